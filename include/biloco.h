@@ -1,0 +1,178 @@
+/*
+ * biloco.h - C ABI of libbiloco.so: the fused NVFP4 GEMM with a binary-sign
+ * low-rank correction on one B200 (sm_100a).
+ *
+ * The operation (BiLoCo README, github jindavid/BiLoCo, sections "Decomposition"
+ * and "Kernel"): a weight is split as W ~= U diag(alpha) V^T + R with sign
+ * factors U in {+-1}^{N x r}, V in {+-1}^{K x r} and an NVFP4 residual R, and the
+ * layer output is
+ *
+ *     y = FP4(x) FP4(R)^T + sum_i alpha_i (x . v_i) u_i            (BF16 out)
+ *
+ * computed in one fused launch: the FP4 product on the tensor cores, the sign
+ * correction on the CUDA cores.
+ *
+ * Conventions for every call
+ *   - Pointers are DEVICE pointers owned by the caller unless stated otherwise;
+ *     the library never frees them.  Calls are asynchronous and ordered on
+ *     `stream` (NULL = the legacy default stream).
+ *   - Return value: BILOCO_OK (0) or a negative BILOCO_ERR_* code.  Argument,
+ *     shape and alignment errors are detected on the host before anything is
+ *     launched.  Errors raised inside a kernel (a bounded wait that expired)
+ *     are reported by biloco_last_error().
+ *   - Row-major everywhere.  "x_bf16" and "y_bf16" point to IEEE bfloat16 data.
+ *   - The library keeps scratch memory per (device, stream), allocated on first
+ *     use and grown when a larger shape arrives; biloco_shutdown() frees it.
+ *     Calls on one stream must not run concurrently with each other from
+ *     several host threads.
+ *
+ * NVFP4 format used throughout (E2M1 elements, one E4M3 scale per 16 elements
+ * along K):
+ *   - element codes: 4-bit E2M1, grid {0, +-0.5, +-1, +-1.5, +-2, +-3, +-4, +-6};
+ *     element 2j of a row in the low nibble of byte j; a zero is always code 0.
+ *   - scale s = E4M3(amax_block / 6) for activations (no tensor scale), and
+ *     s = E4M3(amax_block / (6 g)) for the weight with g = amax(|R|) / 2688
+ *     (g = 1 if R == 0); E4M3 rounding is nearest-even with saturation at 448.
+ *   - code = E2M1(v / S), S = s (activation) or S = s * g (weight), FP32
+ *     division rounded to nearest, E2M1 nearest with ties to the even code,
+ *     |v/S| > 6 saturates; if S == 0 the block's codes are 0.
+ *
+ * Sign packing: bit 1 = -1, bit 0 = +1 (a zero counts as +1), least significant
+ * bit first in little-endian uint32 words; unused tail bits are 0.
+ */
+#ifndef BILOCO_H
+#define BILOCO_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t. */
+typedef struct CUstream_st *biloco_stream_t;
+
+enum {
+  BILOCO_OK = 0,
+  BILOCO_ERR_ARG = -1,     /* NULL pointer where one is required, negative size  */
+  BILOCO_ERR_SHAPE = -2,   /* shape outside the supported limits                  */
+  BILOCO_ERR_ALIGN = -3,   /* pointer not 16-byte aligned                         */
+  BILOCO_ERR_CUDA = -4,    /* a CUDA runtime call or a kernel launch failed       */
+  BILOCO_ERR_TIMEOUT = -5, /* a bounded device-side wait expired (see last_error) */
+  BILOCO_ERR_NOMEM = -6,   /* library scratch could not be allocated              */
+  BILOCO_ERR_DEVICE = -7   /* the current device is not an sm_100 GPU             */
+};
+
+/* Size limits of biloco_gemm. */
+#define BILOCO_MAX_M 128
+#define BILOCO_MAX_R 1024
+
+/* z schedules of biloco_gemm (BiLoCo README, section "Kernel", mode table):
+ *   BILOCO_MODE_AUTO       pick per (M, r, K) from a measured table
+ *   BILOCO_MODE_SHARED_Z   every CTA computes one slice of z = alpha . (V^T x) at
+ *                          entry and publishes it to scratch behind an arrival
+ *                          counter; the GEMM tiles read z in their epilogue
+ *                          (the "side CTAs + arrival flag" schedule)
+ *   BILOCO_MODE_LOCAL_Z    every CTA computes, at entry, the part of z that its own
+ *                          tiles need; no cross-CTA exchange (the "every CTA computes
+ *                          the correction at kernel entry" schedule) */
+enum { BILOCO_MODE_AUTO = 0, BILOCO_MODE_SHARED_Z = 1, BILOCO_MODE_LOCAL_Z = 2 };
+
+/*
+ * biloco_quant_act - BF16 activation -> NVFP4 codes and E4M3 block scales.
+ * (BiLoCo README, section "Kernel": the activation enters the FP4 product as
+ * NVFP4 codes A plus block scales A_sf; no tensor scale is passed.)
+ *
+ *   x_bf16  [M][K] bfloat16, 16-byte aligned
+ *   M, K    M >= 1, K >= 16, K % 16 == 0
+ *   x_fp4   out [M][K/2] bytes (two codes per byte)
+ *   x_sf    out [M][K/16] E4M3 bytes
+ * Bit-exact with the rules in the header comment.
+ */
+int biloco_quant_act(const void *x_bf16, int M, int K, uint8_t *x_fp4, uint8_t *x_sf,
+                     biloco_stream_t stream);
+
+/*
+ * biloco_pack_signs - +-1 matrix -> packed sign words.
+ * (BiLoCo README, section "Kernel": pack_signs(V.T), pack_signs(U.T).)
+ *
+ *   S     [rows][cols] float; bit = 1 where S < 0
+ *   bits  out [rows][ceil(cols/32)] uint32, bit j of word w <-> column 32w + j
+ * For the GEMM: Vbits = pack_signs(V^T) with rows = r, cols = K, and
+ * Ubits = pack_signs(U) with rows = N, cols = r.
+ */
+int biloco_pack_signs(const float *S, int rows, int cols, uint32_t *bits,
+                      biloco_stream_t stream);
+
+/*
+ * biloco_pack_weight - FP32 residual R -> NVFP4 codes, block scales in the
+ * GEMM's tile layout, and the FP32 tensor scale.
+ * (BiLoCo README, section "Decomposition": R is quantised to NVFP4; section
+ * "Kernel": W_fp4, W_sf, w_global_scale.)
+ *
+ *   R       [N][K] float, 16-byte aligned; N % 128 == 0, K % 64 == 0
+ *   W_fp4   out [N][K/2] bytes, 16-byte aligned
+ *   W_sf    out biloco_weight_sf_bytes(N, K) bytes, 16-byte aligned, tile layout:
+ *           the scale of weight row n and 16-element block b (k = 16b .. 16b+15)
+ *           sits at byte
+ *              ((((n/128) * KC + b/16) * 4 + (b%16)/4) * 512)
+ *              + (n%32) * 16 + ((n%128)/32) * 4 + (b%4)
+ *           with KC = ceil(K/256); bytes past K are zero.
+ *   gscale  out device float, the tensor scale g
+ * Runs three kernels; needs no host synchronisation.
+ */
+int biloco_pack_weight(const float *R, int N, int K, uint8_t *W_fp4, uint8_t *W_sf,
+                       float *gscale, biloco_stream_t stream);
+
+/* Bytes of the weight scale array: N * ceil(K/256) * 16. */
+size_t biloco_weight_sf_bytes(int N, int K);
+
+/*
+ * biloco_gemm - y = FP4(x) FP4(R)^T + sum_i alpha_i (x . v_i) u_i, in BF16.
+ * (BiLoCo README, section "Kernel": one launch for decode batches; the FP4 GEMM
+ * on tensor cores, z = alpha . (V x) on CUDA cores from bit-packed V, U z expanded
+ * in the GEMM epilogue before the BF16 store.)
+ *
+ *   x_bf16  [M][K] bfloat16 activation; quantised inside the call exactly like
+ *           biloco_quant_act, and used unquantised (BF16) for the correction
+ *   W_fp4, W_sf, gscale   as written by biloco_pack_weight
+ *   Ubits   [N][ceil(r/32)] uint32 = pack_signs(U)      (may be NULL when r == 0)
+ *   Vbits   [r][K/32] uint32 = pack_signs(V^T)           (may be NULL when r == 0)
+ *   alpha   [r] float                                    (may be NULL when r == 0)
+ *   y_bf16  out [M][N] bfloat16, rounded to nearest-even from FP32
+ *   limits  1 <= M <= 128, N % 128 == 0, K % 64 == 0, 0 <= r <= 1024
+ * Accumulation is FP32 in an unspecified order; results are deterministic for a
+ * fixed shape, mode and GPU.  Two kernels are launched (activation quantiser,
+ * then the fused kernel through programmatic dependent launch).
+ */
+int biloco_gemm(const void *x_bf16, const uint8_t *W_fp4, const uint8_t *W_sf,
+                const float *gscale, const uint32_t *Ubits, const uint32_t *Vbits,
+                const float *alpha, void *y_bf16, int M, int N, int K, int r,
+                biloco_stream_t stream);
+
+/* Select the z schedule for later biloco_gemm calls (process-wide). */
+int biloco_set_mode(int mode);
+/* The schedule biloco_gemm would use for this shape under the current setting. */
+int biloco_resolve_mode(int M, int N, int K, int r);
+
+/*
+ * biloco_last_error - synchronise `stream`, return and clear the first error a
+ * kernel on it recorded (BILOCO_ERR_TIMEOUT when a bounded wait expired), or
+ * BILOCO_OK.  After an error the stream's scratch counters are reset.
+ */
+int biloco_last_error(biloco_stream_t stream);
+
+/* Human-readable name of a status code (static storage). */
+const char *biloco_status_string(int status);
+
+/* Number of kernels biloco_gemm launches per call (for launch accounting). */
+int biloco_gemm_kernel_count(void);
+
+/* Free every stream's scratch.  Safe to call more than once. */
+void biloco_shutdown(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* BILOCO_H */

@@ -1,0 +1,65 @@
+// Host-side declarations shared by the library's translation units.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace biloco {
+
+// Library-owned scratch of one (device, stream) pair.  All regions live in one
+// cudaMalloc block; counters and the status word are zeroed when allocated.
+struct Scratch {
+  int device = -1;
+  cudaStream_t stream = nullptr;
+  void* base = nullptr;
+  size_t bytes = 0;
+  // carved regions
+  int* status = nullptr;            // first device-side error of this stream
+  uint32_t* counters = nullptr;     // rank-block arrivals, z ready/seen, tile tickets
+  size_t counter_words = 0;
+  uint8_t* act_fp4 = nullptr;       // [M][K/2]
+  uint8_t* act_sf = nullptr;        // KC * 2048 scale atoms
+  float* xsum32 = nullptr;          // [M][K/32]
+  float* zpart = nullptr;           // [KB][IB][M][16]
+  float* zfin = nullptr;            // [M][rpad]
+  float* zbsum = nullptr;           // [IB][M]
+  float* slots = nullptr;           // [2 G][BN][128]
+};
+
+struct ScratchNeed {
+  size_t act_fp4, act_sf, xsum32, zpart, zfin, zbsum, slots, counter_words;
+};
+
+// Returns nullptr on allocation failure.
+Scratch* get_scratch(cudaStream_t stream, const ScratchNeed& need);
+
+int num_sms();
+
+// Launchers (return cudaError_t values).
+cudaError_t launch_quant_act_rowmajor(const uint16_t* x, int M, int K, uint8_t* codes, uint8_t* sf,
+                                      cudaStream_t s);
+cudaError_t launch_prep_act(const uint16_t* x, int M, int K, uint8_t* codes, uint8_t* sf_atoms,
+                            float* xsum32, cudaStream_t s);
+cudaError_t launch_pack_weight(const float* R, int N, int K, uint8_t* W_fp4, uint8_t* W_sf,
+                               float* gscale, cudaStream_t s);
+cudaError_t launch_pack_signs(const float* S, int rows, int cols, uint32_t* bits, cudaStream_t s);
+
+struct GemmArgs {
+  const uint16_t* x;
+  const uint8_t* W_fp4;
+  const uint8_t* W_sf;
+  const float* gscale;
+  const uint32_t* Ubits;
+  const uint32_t* Vbits;
+  const float* alpha;
+  uint16_t* y;
+  int M, N, K, r;
+  int mode;   // resolved: 1 shared z, 2 local z
+};
+
+// Validated arguments; launches prep + fused kernels.  Returns a BILOCO_* status.
+int run_gemm(const GemmArgs& a, cudaStream_t s);
+int resolve_mode(int M, int N, int K, int r, int requested);
+
+}  // namespace biloco

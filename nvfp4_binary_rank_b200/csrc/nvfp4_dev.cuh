@@ -1,0 +1,65 @@
+// NVFP4 element and scale conversions on the device (sm_100a).
+//
+// Format (BiLoCo README, section "Kernel": FP4 activation and residual with
+// block scales): E2M1 codes on {0, +-0.5, +-1, +-1.5, +-2, +-3, +-4, +-6}, one
+// E4M3 scale per 16 elements along K.  Rounding: FP32 quotient v/S rounded to
+// nearest, then E2M1 to nearest with ties to the even code and saturation
+// (the hardware cvt.rn.satfinite.e2m1x2.f32); E4M3 scales to nearest-even with
+// saturation at 448 (cvt.rn.satfinite.e4m3x2.f32).  Zero magnitudes are stored
+// as code 0, never as negative zero.
+#pragma once
+
+#include <cstdint>
+
+namespace biloco {
+
+// FP32 -> E4M3 byte, nearest-even, clamped to +-448.
+__device__ __forceinline__ uint32_t e4m3_from_f32(float t) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(t));
+  return r & 0xFFu;
+}
+
+// Exact value of a non-negative E4M3 byte (sign bit ignored; 0x7F never occurs).
+__device__ __forceinline__ float e4m3_to_f32(uint32_t b) {
+  const uint32_t e = (b >> 3) & 15u, m = b & 7u;
+  if (e == 0) return static_cast<float>(m) * 0x1p-9f;          // subnormal: m/8 * 2^-6
+  return __uint_as_float(((e + 120u) << 23) | (m << 20));     // (1+m/8) * 2^(e-7)
+}
+
+// Two FP32 values -> one byte of E2M1 codes, `lo` in the low nibble.
+__device__ __forceinline__ uint32_t e2m1x2(float lo, float hi) {
+  uint16_t r;
+  asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tcvt.u16.u8 %0, t;\n\t}"
+      : "=h"(r)
+      : "f"(hi), "f"(lo));
+  uint32_t b = r & 0xFFu;
+  if ((b & 0x07u) == 0) b &= 0xF0u;     // -0 -> +0 in the low nibble
+  if ((b & 0x70u) == 0) b &= 0x0Fu;     // and in the high nibble
+  return b;
+}
+
+// 16 values and their block scale S (FP32) -> 8 bytes of packed codes.
+__device__ __forceinline__ uint2 encode_block16(const float (&v)[16], float S) {
+  uint2 out = make_uint2(0u, 0u);
+  if (S != 0.0f) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      out.x |= e2m1x2(__fdiv_rn(v[2 * j], S), __fdiv_rn(v[2 * j + 1], S)) << (8 * j);
+      out.y |= e2m1x2(__fdiv_rn(v[8 + 2 * j], S), __fdiv_rn(v[8 + 2 * j + 1], S)) << (8 * j);
+    }
+  }
+  return out;
+}
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint32_t h) { return __uint_as_float(h << 16); }
+
+// Byte offset of the scale of row `row` (< 128 within its 128-row tile) and
+// 16-element block `blk` (block index within the row) inside a run of 512-byte
+// scale atoms: one atom per 64 elements of K, 4 atoms per 256-element chunk.
+__device__ __forceinline__ uint32_t sf_atom_offset(uint32_t row, uint32_t blk) {
+  const uint32_t chunk = blk >> 4, step = (blk >> 2) & 3u, q = blk & 3u;
+  return ((chunk * 4u + step) * 512u) + (row & 31u) * 16u + ((row >> 5) & 3u) * 4u + q;
+}
+
+}  // namespace biloco

@@ -1,0 +1,80 @@
+"""The C-ABI library loads and exports every entry point include/biloco.h declares
+(CPU only: no call here reaches the GPU)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "biloco.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(biloco_[a-z0-9_]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from nvfp4_binary_rank_b200 import build, _lib
+    build.build()
+    return _lib.load()
+
+
+def test_header_declares_the_four_hot_path_calls():
+    names = _declared()
+    for n in ("biloco_quant_act", "biloco_pack_signs", "biloco_pack_weight", "biloco_gemm"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in _declared():
+        assert hasattr(lib, name), name
+
+
+def test_binding_signatures_cover_the_header(lib):
+    from nvfp4_binary_rank_b200 import _lib
+    assert sorted(_lib.SIGNATURES) == _declared()
+
+
+def test_status_strings(lib):
+    from nvfp4_binary_rank_b200 import _lib
+    assert _lib.status_string(0) == "ok"
+    assert "timed out" in _lib.status_string(_lib.ERR_TIMEOUT)
+    assert _lib.status_string(12345) == "unknown status"
+
+
+def test_weight_sf_bytes(lib):
+    from nvfp4_binary_rank_b200 import _lib
+    assert _lib.weight_sf_bytes(5120, 5120) == 5120 * 5120 // 16
+    assert _lib.weight_sf_bytes(128, 320) == 128 * 2 * 16     # K padded to whole 256-chunks
+
+
+def test_host_validation_rejects_bad_arguments_without_a_gpu(lib):
+    # argument and shape checks run before any CUDA call
+    P = ctypes.c_void_p
+    fake = P(0x10000)
+    assert lib.biloco_gemm(None, fake, fake, fake, None, None, None, fake, 1, 128, 64, 0, None) == -1
+    assert lib.biloco_gemm(fake, fake, fake, fake, None, None, None, fake, 0, 128, 64, 0, None) == -2
+    assert lib.biloco_gemm(fake, fake, fake, fake, None, None, None, fake, 129, 128, 64, 0, None) == -2
+    assert lib.biloco_gemm(fake, fake, fake, fake, None, None, None, fake, 1, 100, 64, 0, None) == -2
+    assert lib.biloco_gemm(fake, fake, fake, fake, None, None, None, fake, 1, 128, 96, 0, None) == -2
+    assert lib.biloco_gemm(fake, fake, fake, fake, None, None, None, fake, 1, 128, 64, 1025, None) == -1
+    assert lib.biloco_gemm(fake, fake, fake, fake, fake, fake, fake, fake, 1, 128, 64, 1025, None) == -2
+    assert lib.biloco_gemm(P(0x10008), fake, fake, fake, None, None, None, fake, 1, 128, 64, 0, None) == -3
+    assert lib.biloco_pack_weight(fake, 100, 64, fake, fake, fake, None) == -2
+    assert lib.biloco_quant_act(fake, 1, 24, fake, fake, None) == -2
+    assert lib.biloco_pack_signs(None, 1, 1, fake, None) == -1
+
+
+def test_mode_setting(lib):
+    from nvfp4_binary_rank_b200 import _lib
+    assert lib.biloco_set_mode(7) == -1
+    for m in (_lib.MODE_SHARED_Z, _lib.MODE_LOCAL_Z):
+        assert lib.biloco_set_mode(m) == 0
+        assert lib.biloco_resolve_mode(1, 5120, 5120, 512) == m
+    assert lib.biloco_set_mode(_lib.MODE_AUTO) == 0
+    assert lib.biloco_resolve_mode(1, 5120, 5120, 512) in (_lib.MODE_SHARED_Z, _lib.MODE_LOCAL_Z)

@@ -1,0 +1,130 @@
+"""Parity of biloco_gemm against the FP64 oracle (through the C-ABI).
+
+The GEMM part and the sign correction are pinned separately (r = 0, R = 0)
+because at the workload sizes the correction is about 25x larger than the FP4
+product and would hide an error in it."""
+
+import numpy as np
+import pytest
+import torch
+
+import workloads
+from oracle import biloco as ob
+from gpu_common import (assert_y_close, device_problem, oracle_for, y_errors, y_to_numpy)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def nb():
+    import nvfp4_binary_rank_b200 as nb
+    nb.load()
+    return nb
+
+
+def _run(nb, prob, mode=None):
+    if mode is not None:
+        nb.set_mode(mode)
+    try:
+        y = nb.gemm(prob["x"], prob["W"], prob["sf"], prob["g"], prob["Ub"], prob["Vb"], prob["alpha"])
+        st = nb.last_error()
+        assert st == 0, nb.status_string(st)
+    finally:
+        nb.set_mode(nb.MODE_AUTO)
+    return y_to_numpy(y)
+
+
+def _small(M, N, K, r, seed, outliers=True):
+    return workloads.Workload(f"s{M}_{N}_{K}_{r}", M, N, K, r, seed, outliers=outliers)
+
+
+# --- the FP4 product alone (r = 0) -------------------------------------------
+
+@pytest.mark.parametrize("M,N,K", [(1, 128, 64), (1, 256, 256), (5, 384, 320), (16, 128, 1024),
+                                   (32, 512, 768), (33, 256, 512), (64, 128, 256), (128, 256, 576)])
+def test_fp4_gemm_part(nb, M, N, K):
+    w = _small(M, N, K, 0, seed=M + N + K)
+    d, ref = oracle_for(w)
+    y = _run(nb, device_problem(w, d))
+    assert_y_close(y, ref["gemm"], "r=0 y")
+    # each element within BF16 rounding of the FP64 value (FP32 accumulation error is far below)
+    tol = np.abs(ref["gemm"]) * 2.0 ** -8 + 1e-6 * np.abs(ref["gemm"]).max()
+    assert np.all(np.abs(y - ref["gemm"]) <= tol)
+
+
+# --- the correction alone (R = 0) ---------------------------------------------
+
+@pytest.mark.parametrize("mode", [1, 2])
+@pytest.mark.parametrize("M,N,K,r", [(1, 128, 64, 16), (3, 256, 320, 17), (16, 128, 512, 64),
+                                     (32, 256, 256, 33), (40, 128, 256, 16)])
+def test_correction_part(nb, mode, M, N, K, r):
+    w = _small(M, N, K, r, seed=100 + M + r)
+    d = workloads.make_inputs(w)
+    d["R"] = np.zeros_like(d["R"])
+    ref = ob.biloco_reference(d["x"], d["R"], d["U"], d["V"], d["alpha"])
+    y = _run(nb, device_problem(w, d), mode)
+    assert_y_close(y, ref["corr"], "R=0 y")
+
+
+def test_all_ones_signs_closed_form(nb):
+    w = _small(4, 256, 512, 32, seed=7)
+    d = workloads.make_inputs(w)
+    d["R"] = np.zeros_like(d["R"])
+    d["U"] = np.ones_like(d["U"])
+    d["V"] = np.ones_like(d["V"])
+    y = _run(nb, device_problem(w, d))
+    want = float(d["alpha"].astype(np.float64).sum()) * d["x"].astype(np.float64).sum(axis=1)
+    assert_y_close(y, np.repeat(want[:, None], w.N, axis=1), "U=V=1")
+
+
+# --- full y on the workloads ---------------------------------------------------
+
+@pytest.mark.parametrize("name", ["tiny", "decode", "mlp_up", "mlp_down"])
+def test_workload_y(nb, name):
+    w = workloads.CONFIGS[name]
+    d, ref = oracle_for(w)
+    y = _run(nb, device_problem(w, d))
+    assert_y_close(y, ref["y"], name)
+
+
+@pytest.mark.parametrize("M", workloads.SWEEP_MS)
+@pytest.mark.parametrize("r", workloads.SWEEP_RS)
+def test_sweep_y(nb, M, r):
+    w = workloads.sweep_config(M, r)
+    d, ref = oracle_for(w)
+    y = _run(nb, device_problem(w, d))
+    assert_y_close(y, ref["y"], w.name)
+
+
+@pytest.mark.parametrize("mode", [1, 2])
+@pytest.mark.parametrize("M,N,K,r", [(1, 128, 64, 1), (2, 640, 1344, 100), (17, 384, 832, 255),
+                                     (31, 1280, 2560, 1024), (100, 256, 448, 48)])
+def test_ragged_shapes_both_modes(nb, mode, M, N, K, r):
+    w = _small(M, N, K, r, seed=M * 3 + r)
+    d, ref = oracle_for(w)
+    y = _run(nb, device_problem(w, d), mode)
+    assert_y_close(y, ref["y"], w.name)
+
+
+def test_deterministic_and_reusable(nb):
+    w = workloads.CONFIGS["decode"]
+    d, ref = oracle_for(w)
+    prob = device_problem(w, d)
+    y1 = _run(nb, prob)
+    y2 = _run(nb, prob)
+    np.testing.assert_array_equal(y1, y2)
+
+
+def test_shape_and_alignment_errors(nb):
+    x = torch.zeros((1, 64), dtype=torch.bfloat16, device="cuda")
+    W = torch.zeros((128, 32), dtype=torch.uint8, device="cuda")
+    sf = torch.zeros((nb.weight_sf_bytes(128, 64),), dtype=torch.uint8, device="cuda")
+    g = torch.ones((1,), device="cuda")
+    with pytest.raises(nb.BilocoError) as e:
+        nb.gemm(torch.zeros((129, 64), dtype=torch.bfloat16, device="cuda"),
+                W, sf, g, None, None, None)
+    assert e.value.status == -2
+    buf = torch.zeros((2 * 64 + 8,), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(nb.BilocoError) as e:
+        nb.gemm(buf[1:65].view(1, 64), W, sf, g, None, None, None)
+    assert e.value.status == -3
