@@ -1,0 +1,453 @@
+"""Benchmark of the fused NVFP4 + binary-sign low-rank GEMM on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one pass of the whole hot path over one batch: the activation
+quantiser and the fused GEMM (two kernels, the second launched with
+programmatic dependent launch), i.e. one `biloco_gemm` call.  The default
+workload is the decode shape (M=1, N=K=5120, r=512).  Steps are replayed from
+a CUDA graph; each step reads a different copy of the weight so that the copies
+together exceed the L2 cache, and the device time of exactly K steps is taken
+with CUDA events on the launching stream, bracketed by a barrier and
+synchronisation, max over ranks.
+
+Multi-GPU (torchrun): every rank runs an independent replica of the workload
+(the operation has no exchange step); `value` is the bytes of all ranks over
+the slowest rank's time ("scaling": "weak").
+
+`--impl reference` times the CPU oracle (NumPy/FP64) on a bounded row slice
+of the same workload; only rank 0 runs it.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "fused FP4+binary-lowrank GEMM µs and HBM GB/s (% of peak), M=1–32, r=512"
+UNIT = "GB/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def algo_bytes(M, N, K, r):
+    """Algorithmic HBM bytes of one call: weight codes + E4M3 scales + sign bits +
+    BF16 activation + BF16 output + FP32 alpha."""
+    return N * K // 2 + N * K // 16 + (N + K) * r // 8 + M * K * 2 + M * N * 2 + 4 * r
+
+
+def hbm_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples (every 100 ms) of SM clock and throttle reasons."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.thread.join(timeout=2)
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": float(np.median(sm)) if sm else None,
+                "sm_max_mhz": float(max(mx)) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- GPU arm
+
+def setup_problem(w, n_copies, device):
+    import torch
+    import nvfp4_binary_rank_b200 as nb
+    d = workloads.make_inputs(w)
+    x = torch.from_numpy(d["x_bf16"].astype(np.int16)).view(torch.bfloat16).to(device)
+    R = torch.from_numpy(d["R"]).to(device)
+    W, sf, g = nb.pack_weight(R)
+    copies = [(W, sf, g)] + [(W.clone(), sf.clone(), g.clone()) for _ in range(n_copies - 1)]
+    del R
+    if w.r:
+        Ub = nb.pack_signs(torch.from_numpy(d["U"].astype(np.float32)).to(device))
+        Vb = nb.pack_signs(torch.from_numpy(np.ascontiguousarray(d["V"].T).astype(np.float32)).to(device))
+        alpha = torch.from_numpy(d["alpha"]).to(device)
+    else:
+        Ub = Vb = alpha = None
+    y = torch.empty((w.M, w.N), dtype=torch.bfloat16, device=device)
+    torch.cuda.synchronize()
+    return dict(x=x, copies=copies, Ub=Ub, Vb=Vb, alpha=alpha, y=y, host=d)
+
+
+def n_copies_for(w, l2_bytes):
+    per = w.N * w.K // 2 + w.N * w.K // 16
+    return max(2, int(np.ceil(1.25 * l2_bytes / per)))
+
+
+def time_graph(prob, steps, warmup, stream, dist_ctx):
+    """Device time of exactly `steps` calls replayed from CUDA graphs."""
+    import torch
+    import nvfp4_binary_rank_b200 as nb
+    copies = prob["copies"]
+    nc = len(copies)
+
+    def call(i):
+        W, sf, g = copies[i % nc]
+        nb.gemm(prob["x"], W, sf, g, prob["Ub"], prob["Vb"], prob["alpha"], out=prob["y"])
+
+    with torch.cuda.stream(stream):
+        for i in range(max(warmup, 3)):
+            call(i)
+    stream.synchronize()
+    st = nb.last_error(stream)
+    if st != 0:
+        raise RuntimeError(f"warm-up failed: {nb.status_string(st)}")
+
+    def capture(n):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(n):
+                call(i)
+        return g
+
+    chunk = nc * max(1, 64 // nc)
+    full, rem = divmod(steps, chunk)
+    g_full = capture(chunk) if full else None
+    g_rem = capture(rem) if rem else None
+    # warm replay of the graphs themselves
+    with torch.cuda.stream(stream):
+        if g_full:
+            g_full.replay()
+        if g_rem:
+            g_rem.replay()
+    stream.synchronize()
+
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    dist_ctx.barrier()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        start.record(stream)
+        for _ in range(full):
+            g_full.replay()
+        if g_rem:
+            g_rem.replay()
+        end.record(stream)
+    end.synchronize()
+    torch.cuda.synchronize()
+    dist_ctx.barrier()
+    ms = start.elapsed_time(end)
+    st = nb.last_error(stream)
+    if st != 0:
+        raise RuntimeError(f"timed region failed: {nb.status_string(st)}")
+    del g_full, g_rem
+    return ms
+
+
+def time_e2e(prob, steps, stream):
+    """Same call from pinned host buffers: H2D of x, the call, D2H of y, per step."""
+    import torch
+    import nvfp4_binary_rank_b200 as nb
+    x_host = prob["x"].cpu().pin_memory()
+    y_host = torch.empty(prob["y"].shape, dtype=torch.bfloat16).pin_memory()
+    copies = prob["copies"]
+    nc = len(copies)
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            prob["x"].copy_(x_host, non_blocking=True)
+            W, sf, g = copies[i % nc]
+            nb.gemm(prob["x"], W, sf, g, prob["Ub"], prob["Vb"], prob["alpha"], out=prob["y"])
+            y_host.copy_(prob["y"], non_blocking=True)
+        stream.synchronize()
+        start.record(stream)
+        for i in range(steps):
+            prob["x"].copy_(x_host, non_blocking=True)
+            W, sf, g = copies[i % nc]
+            nb.gemm(prob["x"], W, sf, g, prob["Ub"], prob["Vb"], prob["alpha"], out=prob["y"])
+            y_host.copy_(prob["y"], non_blocking=True)
+        end.record(stream)
+    end.synchronize()
+    return start.elapsed_time(end) / steps, x_host.numel() * 2, y_host.numel() * 2
+
+
+class DistCtx:
+    def __init__(self):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = False
+
+    def init(self):
+        import datetime
+        import torch
+        import torch.distributed as dist
+        if self.world > 1:
+            os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", self.local))
+            self.pg = True
+
+    def barrier(self):
+        if self.pg:
+            import torch.distributed as dist
+            dist.barrier()
+
+    def max(self, v: float) -> float:
+        if not self.pg:
+            return v
+        import torch
+        import torch.distributed as dist
+        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+def measure_config(w, steps, warmup, stream, dist_ctx, l2):
+    import torch
+    prob = setup_problem(w, n_copies_for(w, l2), torch.device("cuda", torch.cuda.current_device()))
+    ms = dist_ctx.max(time_graph(prob, steps, warmup, stream, dist_ctx))
+    us = ms * 1e3 / steps
+    b = algo_bytes(w.M, w.N, w.K, w.r)
+    peak, _ = hbm_peak()
+    out = {"us": round(us, 3), "GBps": round(b / (us * 1e-6) / 1e9, 1),
+           "frac": round(b / (us * 1e-6) / 1e9 / peak, 4), "bytes": b}
+    del prob
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_ours(args):
+    import torch
+    import nvfp4_binary_rank_b200 as nb
+    from nvfp4_binary_rank_b200 import build as _b
+    ctx = DistCtx()
+    torch.cuda.set_device(ctx.local)
+    ctx.init()
+    if ctx.rank == 0:
+        _b.build()
+    ctx.barrier()
+    nb.load()
+    stream = torch.cuda.Stream()
+    l2 = torch.cuda.get_device_properties(ctx.local).L2_cache_size
+    w = workloads.CONFIGS[args.workload]
+    peak, peak_kind = hbm_peak()
+
+    prob = setup_problem(w, n_copies_for(w, l2), torch.device("cuda", ctx.local))
+    with ClockSampler(ctx.local) as clk:
+        ms_local = time_graph(prob, args.steps, args.warmup, stream, ctx)
+    ms = ctx.max(ms_local)
+    us = ms * 1e3 / args.steps
+    b = algo_bytes(w.M, w.N, w.K, w.r)
+    gbs_rank = b / (us * 1e-6) / 1e9
+    value = gbs_rank * ctx.world
+
+    e2e_steps = min(args.steps, 2000)
+    e2e_ms, h2d, d2h = time_e2e(prob, e2e_steps, stream)
+    e2e_ms = ctx.max(e2e_ms)
+    e2e_val = b * ctx.world / (e2e_ms * 1e-3) / 1e9
+    del prob
+    torch.cuda.empty_cache()
+
+    extra = {}
+    if not args.no_extra:
+        sub_steps = max(2000, args.steps // 20)
+        for name, ww in [("mlp_up", workloads.CONFIGS["mlp_up"]),
+                         ("mlp_down", workloads.CONFIGS["mlp_down"]),
+                         ("sweep_M8_r512", workloads.sweep_config(8, 512)),
+                         ("sweep_M32_r512", workloads.sweep_config(32, 512)),
+                         ("sweep_M1_r0", workloads.sweep_config(1, 0))]:
+            extra[name] = measure_config(ww, sub_steps, args.warmup, stream, ctx, l2)
+
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": ctx.world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 6),
+        "us_per_call": round(us, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "nvfp4", "data": "synthetic",
+        "config": {"workload": w.name, "M": w.M, "N": w.N, "K": w.K, "r": w.r,
+                   "seed": w.seed, "parallelism": f"replicas x{ctx.world}",
+                   "l2": f"{n_copies_for(w, l2)} weight copies rotated (> L2 {l2 >> 20} MiB)",
+                   "launch": f"CUDA graph replay, {nb.gemm_kernel_count(w.M)} kernel(s) per step"},
+        "roofline": {"bound": "hbm", "achieved": round(gbs_rank, 1), "peak": peak,
+                     "unit": "GB/s", "frac": round(gbs_rank / peak, 4), "traffic": None,
+                     "peak_kind": peak_kind, "per": "step (all kernels of one call)"},
+        "e2e": {"value": round(e2e_val, 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "us_per_step": round(e2e_ms * 1e3, 3),
+                "api": "nvfp4_binary_rank_b200.gemm, eager, pinned host x/y"},
+        "gpu_launches": nb.gemm_kernel_count(w.M) * args.steps,
+        "clocks": clk.summary(),
+        "extra_configs": extra,
+    }
+    if ctx.world == 1 and ctx.rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, budget_s=12.0)
+    if ctx.rank == 0:
+        print(json.dumps(line), flush=True)
+    ctx.close()
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+
+def _oracle_sample(w, rows):
+    """Inputs for the oracle on output rows [0, rows) of the workload."""
+    from oracle import nvfp4 as on
+    d = workloads.make_inputs(w)
+    wq, ws, g = on.quant_weight(d["R"])
+    return dict(x=d["x"], wq=wq[:rows], ws=ws[:rows], g=g, U=d["U"][:rows], V=d["V"],
+                alpha=d["alpha"])
+
+
+def _oracle_step(s):
+    from oracle import biloco as ob
+    from oracle import nvfp4 as on
+    xq, xs = on.quant_act(s["x"])
+    y = ob.gemm_part(xq, xs, s["wq"], s["ws"], s["g"])
+    if s["alpha"].size:
+        y = y + ob.correction_part(s["x"], s["U"], s["V"], s["alpha"])
+    return y
+
+
+def _threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info()]
+        return int(max(n)) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(w, budget_s=12.0, rows=None):
+    rows = w.N if rows is None else rows
+    s = _oracle_sample(w, rows)
+    b = algo_bytes(w.M, rows, w.K, w.r)
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        _oracle_step(s)
+        n += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = (time.perf_counter() - t0) / n
+    return {"value": round(b / dt / 1e9, 4), "unit": UNIT, "cores": _threads(), "kind": "oracle",
+            "sample": f"{n} full oracle passes (quantise x, FP64 GEMM part from packed weight, "
+                      f"FP64 correction) over {w.name} rows 0..{rows}, {dt * 1e3:.1f} ms each"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    w = workloads.CONFIGS[args.workload]
+    # each step is a bounded row slice so that warm-up + steps stay within ~2 minutes
+    probe = _oracle_sample(w, 128)
+    t0 = time.perf_counter()
+    _oracle_step(probe)
+    t_row = (time.perf_counter() - t0) / 128
+    per_step = 100.0 / max(args.steps + args.warmup, 1)
+    rows = int(max(1, min(w.N, per_step / max(t_row, 1e-9))))
+    s = _oracle_sample(w, rows)
+    for _ in range(args.warmup):
+        _oracle_step(s)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        _oracle_step(s)
+    dt = (time.perf_counter() - t0) / args.steps
+    b = algo_bytes(w.M, rows, w.K, w.r)
+    val = b / dt / 1e9
+    line = {
+        "metric": METRIC, "value": round(val, 4), "unit": UNIT, "n_gpus": int(args.gpus),
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "impl": "reference",
+        "config": {"workload": w.name, "M": w.M, "N": w.N, "K": w.K, "r": w.r, "seed": w.seed,
+                   "rows_per_step": rows},
+        "cpu_baseline": {"value": round(val, 4), "unit": UNIT, "cores": _threads(), "kind": "oracle",
+                         "sample": f"oracle on rows 0..{rows} of {w.name} per step"},
+        "e2e": {"value": round(val, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200000)
+    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(workloads.CONFIGS), default="decode")
+    ap.add_argument("--no-extra", action="store_true", help="skip the other workloads")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

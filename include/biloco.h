@@ -143,8 +143,9 @@ size_t biloco_weight_sf_bytes(int N, int K);
  *   y_bf16  out [M][N] bfloat16, rounded to nearest-even from FP32
  *   limits  1 <= M <= 128, N % 128 == 0, K % 64 == 0, 0 <= r <= 1024
  * Accumulation is FP32 in an unspecified order; results are deterministic for a
- * fixed shape, mode and GPU.  Two kernels are launched (activation quantiser,
- * then the fused kernel through programmatic dependent launch).
+ * fixed shape, mode and GPU.  For M <= 8 one kernel is launched (it quantises
+ * the activation itself); for larger M an activation quantiser runs first and
+ * the fused kernel follows through programmatic dependent launch.
  */
 int biloco_gemm(const void *x_bf16, const uint8_t *W_fp4, const uint8_t *W_sf,
                 const float *gscale, const uint32_t *Ubits, const uint32_t *Vbits,
@@ -166,8 +167,9 @@ int biloco_last_error(biloco_stream_t stream);
 /* Human-readable name of a status code (static storage). */
 const char *biloco_status_string(int status);
 
-/* Number of kernels biloco_gemm launches per call (for launch accounting). */
-int biloco_gemm_kernel_count(void);
+/* Number of kernels biloco_gemm launches per call for a batch of M rows:
+ * 1 when the activation is quantised inside the fused kernel (M <= 8), else 2. */
+int biloco_gemm_kernel_count(int M);
 
 /* Free every stream's scratch.  Safe to call more than once. */
 void biloco_shutdown(void);

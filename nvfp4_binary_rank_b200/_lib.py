@@ -39,7 +39,7 @@ SIGNATURES = {
     "biloco_resolve_mode": (_I, [_I, _I, _I, _I]),
     "biloco_last_error": (_I, [_P]),
     "biloco_status_string": (ctypes.c_char_p, [_I]),
-    "biloco_gemm_kernel_count": (_I, []),
+    "biloco_gemm_kernel_count": (_I, [_I]),
     "biloco_shutdown": (None, []),
 }
 
@@ -172,8 +172,8 @@ def last_error(stream=None) -> int:
     return int(load().biloco_last_error(_stream(stream)))
 
 
-def gemm_kernel_count() -> int:
-    return int(load().biloco_gemm_kernel_count())
+def gemm_kernel_count(M: int) -> int:
+    return int(load().biloco_gemm_kernel_count(M))
 
 
 def shutdown():

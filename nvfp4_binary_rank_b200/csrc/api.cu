@@ -45,7 +45,7 @@ int check_device() {
 
 // Region offsets of one scratch block, every region 256-byte aligned.
 struct Carve {
-  size_t status, counters, act_fp4, act_sf, xsum32, zpart, zfin, zbsum, slots, total;
+  size_t status, counters, act_fp4, act_sf, zpart, zfin, slots, total;
 };
 
 Carve carve(const ScratchNeed& n) {
@@ -60,10 +60,8 @@ Carve carve(const ScratchNeed& n) {
   c.counters = take(n.counter_words * 4);
   c.act_fp4 = take(n.act_fp4);
   c.act_sf = take(n.act_sf);
-  c.xsum32 = take(n.xsum32);
   c.zpart = take(n.zpart);
   c.zfin = take(n.zfin);
-  c.zbsum = take(n.zbsum);
   c.slots = take(n.slots);
   c.total = off;
   return c;
@@ -73,10 +71,8 @@ ScratchNeed max_need(const ScratchNeed& a, const ScratchNeed& b) {
   ScratchNeed m;
   m.act_fp4 = std::max(a.act_fp4, b.act_fp4);
   m.act_sf = std::max(a.act_sf, b.act_sf);
-  m.xsum32 = std::max(a.xsum32, b.xsum32);
   m.zpart = std::max(a.zpart, b.zpart);
   m.zfin = std::max(a.zfin, b.zfin);
-  m.zbsum = std::max(a.zbsum, b.zbsum);
   m.slots = std::max(a.slots, b.slots);
   m.counter_words = std::max(a.counter_words, b.counter_words);
   return m;
@@ -96,10 +92,8 @@ void apply_carve(Scratch& s, const Carve& c, const ScratchNeed& n) {
   s.counter_words = n.counter_words;
   s.act_fp4 = b + c.act_fp4;
   s.act_sf = b + c.act_sf;
-  s.xsum32 = reinterpret_cast<float*>(b + c.xsum32);
   s.zpart = reinterpret_cast<float*>(b + c.zpart);
   s.zfin = reinterpret_cast<float*>(b + c.zfin);
-  s.zbsum = reinterpret_cast<float*>(b + c.zbsum);
   s.slots = reinterpret_cast<float*>(b + c.slots);
 }
 
@@ -120,9 +114,8 @@ Scratch* get_scratch(cudaStream_t stream, const ScratchNeed& need) {
     if (x->s.device == dev && x->s.stream == stream) e = x;
   if (e) {
     const ScratchNeed& h = e->have;
-    if (need.act_fp4 <= h.act_fp4 && need.act_sf <= h.act_sf && need.xsum32 <= h.xsum32 &&
-        need.zpart <= h.zpart && need.zfin <= h.zfin && need.zbsum <= h.zbsum &&
-        need.slots <= h.slots && need.counter_words <= h.counter_words)
+    if (need.act_fp4 <= h.act_fp4 && need.act_sf <= h.act_sf && need.zpart <= h.zpart &&
+        need.zfin <= h.zfin && need.slots <= h.slots && need.counter_words <= h.counter_words)
       return &e->s;
   }
   ScratchNeed want = e ? max_need(e->have, need) : need;
@@ -279,7 +272,7 @@ const char* biloco_status_string(int status) {
   }
 }
 
-int biloco_gemm_kernel_count(void) { return 2; }
+int biloco_gemm_kernel_count(int M) { return gemm_kernel_count_for(M); }
 
 void biloco_shutdown(void) {
   std::lock_guard<std::mutex> lk(g_mu);

@@ -8,18 +8,24 @@
 // BF16 store, all in one launch.)
 //
 // Work decomposition ("swap-AB" + stream-K):
-//   * The MMA's M dimension (128) runs over weight rows n, its N dimension (BN)
-//     over activation rows m, so a decode batch of 1..32 rows wastes nothing on
-//     padding to 128 activation rows.
-//   * A "unit" is one 128-row weight tile times 256 elements of K: 16 KB of E2M1
-//     codes (one 128-byte swizzled row per weight row) plus 2 KB of scales.  The
-//     T * KC units are split into G contiguous ranges, one per CTA (G <= #SMs), so
-//     every SM streams the same number of weight bytes.  A CTA's range covers
-//     parts of at most a few tiles ("segments"); a tile cut between several CTAs
+//   * The MMA's M dimension (128) runs over weight rows n and its N dimension (BN)
+//     over activation rows m, so a decode batch of 1..32 rows is not padded to
+//     128 activation rows.
+//   * A "unit" is one 128-row weight tile times one 256-element chunk of K:
+//     16 KB of E2M1 codes (a 128-byte swizzled row per weight row) plus 2 KB of
+//     scales.  The T * KC units are cut into G contiguous ranges, one per CTA
+//     (G <= #SMs), so every SM streams the same number of weight bytes.  A range
+//     covers parts of one or a few tiles ("segments"); a tile split between CTAs
 //     is summed through FP32 partial slots by the last CTA to arrive (ticket).
-//   * The sign correction of a tile is split over the same contributors by rank
-//     blocks in proportion to their share of the tile's K, so the CUDA-core work
-//     is balanced exactly like the weight stream.
+//   * The sign correction rides on the same units.  Unit (t, c) computes the
+//     chunk-c part of V^T x for tile t's slice of the ranks (every chunk's ranks
+//     are spread over the T tiles), and the U side of a tile is split over its
+//     contributors in rank blocks proportional to their share of the tile's K.
+//     Both halves are therefore balanced exactly like the weight stream.
+//   * Small batches (M <= 8) quantise the activation chunk in the CTA that uses
+//     it, straight from the staged BF16 chunk into the swizzled B tile and its
+//     scale atoms; larger batches take it from a pre-pass kernel (launched before,
+//     overlapped through programmatic dependent launch).
 //
 // Warp roles (14 warps):
 //   warp 0      TMA producer: weight codes (2-D tiled, 128B swizzle), weight scales
@@ -27,15 +33,14 @@
 //   warp 1      TMEM allocator and tcgen05 MMA issuer (kind::mxf4nvf4, block16)
 //   warps 2-5   epilogue: tcgen05.ld of the accumulator, g * acc + correction,
 //               BF16 store or split-K partial + ticket
-//   warps 6-13  CUDA-core sign correction: the V side (z slices) at entry and the
+//   warps 6-13  CUDA cores: activation quantisation (small M), V side per unit,
 //               U side per segment
 //
 // z schedules:
-//   shared z (mode 1)  every CTA computes one (K block, 16-rank block) slice of
-//                      V^T x, publishes it to scratch and bumps an arrival counter;
-//                      the last arrival of a rank block sums its K blocks, applies
-//                      alpha and marks the block ready.  Tiles wait (bounded) for
-//                      all rank blocks before their U side.
+//   shared z (mode 1)  units publish chunk partials of V^T x; once every CTA has
+//                      published (one arrival counter; for larger batches a
+//                      per-tile finaliser sums the chunks first), each CTA reads the
+//                      z ranks of its rank shares.
 //   local z  (mode 2)  every CTA computes, over the whole K, the z ranks its own
 //                      segments need; no cross-CTA traffic.
 //
@@ -46,13 +51,13 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
-#include <unordered_map>
 
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include "../../include/biloco.h"
+
 #include "internal.h"
 #include "nvfp4_dev.cuh"
 #include "ptx.cuh"
@@ -69,16 +74,20 @@ constexpr int kAluWarp0 = 6;
 constexpr int kAluWarps = 8;
 constexpr int kAluThreads = kAluWarps * 32;
 constexpr int kTileRows = 128;             // weight rows per tile = MMA M
-constexpr int kUnitK = 256;                // K elements per unit
+constexpr int kUnitK = 256;                // K elements per unit (chunk)
 constexpr int kUnitBytesA = kTileRows * 128;
 constexpr int kSfBytes = 2048;             // 4 scale atoms of 512 B per unit
-constexpr int kRB = 16;                    // ranks per rank block
+constexpr int kRB = 16;                    // ranks per U-side rank block
 constexpr int kMP = 32;                    // activation rows per CUDA-core pass
-constexpr int kMpad = 36;                  // padded row stride (floats) of staged tiles
-constexpr int kXWords = 8;                 // 32-element words per staged x sub-block
+constexpr int kMpad = 36;                  // padded row stride (floats) of staged z
+constexpr int kXWords = 8;                 // 32-element words per chunk
+constexpr int kSubK = kXWords * 32;        // K elements per staged x chunk
+constexpr int kVRanks = 32;                // V-side ranks per computed sub-range
+constexpr int kVStageRanks = 64;           // V rows staged per unit by TMA (fast path)
 constexpr int kZChunkBlocks = 8;           // rank blocks per staged z chunk
 constexpr int kTmemCols = 512;
 constexpr int kSfTmemBase = 256;           // TMEM column of the scale-factor regions
+constexpr int kInKernelQuantMaxM = 8;
 
 constexpr int kBarAlu = 1;                 // named barrier ids (0 is __syncthreads)
 constexpr int kBarEpi = 2;
@@ -91,20 +100,23 @@ struct FusedParams {
   const uint32_t* Vbits;
   const float* alpha;
   const uint16_t* x;
-  const float* xsum32;
   uint16_t* y;
-  float* zpart;
-  float* zfin;
-  float* zbsum;
-  float* slots;
-  uint32_t* rb_count;
+  float* zpart;        // [KC][M][rpad]
+  float* zfin;         // [M][rpad]
+  float* slots;        // [2 G][BN][128]
   uint32_t* z_ready;
   uint32_t* z_seen;
-  uint32_t* tickets;
+  uint32_t* tickets;   // [T] split-K tickets
+  uint32_t* vtick;     // [T] V-side finaliser tickets
   int* status;
   int M, N, K, r;
-  int KC, T, U, G, KW, KB, IB, rpad, RW;
-  int mode;
+  int KC, T, U, G, KW, rpad, RW;
+  int mode;            // BILOCO_MODE_SHARED_Z or BILOCO_MODE_LOCAL_Z
+  int inq;             // 1: activation quantised in-kernel (no pre-pass)
+  int zdirect;         // 1: consumers sum the chunk partials themselves
+  int fast;            // 1: the producer stages each unit's x chunk and V rows by TMA
+  int unit_alu;        // 1: the CUDA-core warps have per-unit work (quantise and/or V side)
+  int bxr;             // rows of the staged x box (16 or 32)
 };
 
 template <int BN, int ST>
@@ -113,21 +125,33 @@ struct Layout {
   static constexpr int kB = kA + ST * kUnitBytesA;
   static constexpr int kSFA = kB + ST * BN * 128;
   static constexpr int kSFB = kSFA + ST * kSfBytes;
-  static constexpr int kXS = kSFB + ST * kSfBytes;                 // x sub-block [256][kMpad]
-  static constexpr int kXSBytes = kXWords * 32 * kMpad * 4;
-  static constexpr int kZS = kXS + kXSBytes;                        // z chunk [128][kMpad]
-  static constexpr int kZSBytes = kZChunkBlocks * kRB * kMpad * 4;
-  static constexpr int kZB = kZS + kZSBytes;                        // zbsum chunk [8][32]
-  static constexpr int kVS = kZB + kZChunkBlocks * kMP * 4;         // V bits [16][8]
-  static constexpr int kCorr = kVS + kRB * kXWords * 4;             // corr [2][32][128]
-  static constexpr int kRed = kCorr + 2 * kMP * kTileRows * 4;      // k-split partials [8][64]
-  static constexpr int kVOut = kRed + kAluWarps * 64 * 4;           // V-side result [32][16]
-  static constexpr int kBar = kVOut + kMP * kRB * 4;
-  static constexpr int kNumBars = 2 * ST + 7;
+  // per-stage x chunk + V rows staged by TMA (fast path); the cp.async fallback
+  // uses the start of the same region as its double buffer
+  static constexpr int kXRows = (BN <= 16) ? 16 : 32;
+  static constexpr int kXBytes = kXRows * kSubK * 2;
+  static constexpr int kVBytes = kVStageRanks * kXWords * 4;
+  static constexpr int kXStride = kXBytes + kVBytes;
+  static constexpr int kFallbackBytes = 2 * kMP * kSubK * 2 + 2 * kVRanks * kXWords * 4;
+  static constexpr int kXSRegion = (BN <= 32) ? ((ST * kXStride > kFallbackBytes) ? ST * kXStride
+                                                                                   : kFallbackBytes)
+                                              : kFallbackBytes;
+  static constexpr int kXS = kSFB + ST * kSfBytes;
+  static constexpr int kXB = kXS;                                    // fallback x [2][32][256]
+  static constexpr int kVB = kXB + 2 * kMP * kSubK * 2;              // fallback V [2][32][8]
+  static constexpr int kZS = kXS + kXSRegion;                        // z chunk [128][kMpad]
+  static constexpr int kZB = kZS + kZChunkBlocks * kRB * kMpad * 4;  // z block sums [8][32]
+  static constexpr int kCorr = kZB + kZChunkBlocks * kMP * 4;        // corr [2][32][128]
+  static constexpr int kRed = kCorr + 2 * kMP * kTileRows * 4;       // task partials [8][64]
+  static constexpr int kVOut = kRed + kAluWarps * 64 * 4;            // V-side result [32][32]
+  static constexpr int kXsw = kVOut + kMP * kVRanks * 4;             // x sums per warp [8][32]
+  static constexpr int kXsum = kXsw + kAluWarps * kMP * 4;           // x sums [32]
+  static constexpr int kBar = kXsum + kMP * 4;
+  static constexpr int kNumBars = 3 * ST + 7;
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kTotal = kMisc + 64;
   static constexpr int kAlloc = kTotal + 1024;
   static_assert(kB % 1024 == 0 && (BN * 128) % 1024 == 0, "swizzled tiles need 1 KB alignment");
+  static_assert(kXB % 16 == 0 && kVB % 16 == 0, "cp.async destinations need 16-byte alignment");
   static_assert(kAlloc <= 232448, "shared memory budget");
 };
 
@@ -159,8 +183,9 @@ __device__ __forceinline__ float hi_f(uint64_t v) {
   return __uint_as_float(static_cast<uint32_t>(v >> 32));
 }
 
-// Reduce V per-lane values over the 32 lanes of a warp.  Afterwards lane l holds
-// the totals of entries  out_index(l, j)  in v[j], j < max(1, V/32).
+// Reduce V per-lane values over the 32 lanes of a warp (recursive halving).
+// Afterwards lane l holds in v[j] (j < max(1, V/32)) the total of entry
+// reduce_out_index<V>(l, j).
 template <int V>
 __device__ __forceinline__ void warp_reduce_scatter(float (&v)[V], int lane) {
   int half = V / 2;
@@ -169,7 +194,7 @@ __device__ __forceinline__ void warp_reduce_scatter(float (&v)[V], int lane) {
     if (half >= 1) {
       const bool upper = (lane & o) != 0;
 #pragma unroll
-      for (int j = 0; j < V / 2; ++j) {
+      for (int j = 0; j < (V > 1 ? V / 2 : 1); ++j) {
         if (j < half) {
           const float send = upper ? v[j] : v[j + half];
           const float keep = upper ? v[j + half] : v[j];
@@ -187,7 +212,6 @@ __device__ __forceinline__ int reduce_out_index(int lane, int j) {
   if constexpr (V >= 32) {
     return (V / 32) * lane + j;
   } else {
-    // log2(V) halving steps used lane bits 4 .. 5-log2(V)
     constexpr int kLog = (V >= 16) ? 4 : (V >= 8) ? 3 : (V >= 4) ? 2 : (V >= 2) ? 1 : 0;
     return lane >> (5 - kLog);
   }
@@ -203,116 +227,106 @@ __device__ __forceinline__ void fail(const Ctl& c) {
   record_error(c.status, kDevErrTimeout);
 }
 
-// Bounded spin on a global counter.
+// Bounded spin on a global counter (every calling lane polls).
 __device__ __forceinline__ bool spin_until_geq(const uint32_t* p, uint32_t target, const Ctl& c) {
   const uint64_t t0 = globaltimer_ns();
   while (ld_acquire_gpu(p) < target) {
     if (*c.abort_flag) return false;
     if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
-    __nanosleep(64);
+    __nanosleep(32);
   }
   return true;
 }
 
-// One elected thread of a named-barrier group waits on an mbarrier; the whole
-// group learns the outcome.  Returns false (uniformly) on timeout / abort.
-__device__ __forceinline__ bool group_wait(uint32_t bar, uint32_t parity, bool elected, int bar_id,
-                                           int nthreads, volatile int* shared_ok, const Ctl& c) {
-  if (elected) {
-    const bool ok = mbar_wait(bar, parity, c.abort_flag);
-    if (!ok) fail(c);
-    *shared_ok = ok ? 1 : 0;
+// Every thread of a named-barrier group waits on an mbarrier phase; the group
+// then agrees (barrier + OR) on whether anyone gave up, so all leave together.
+__device__ __forceinline__ bool group_wait(uint32_t bar, uint32_t parity, int bar_id, int nthreads,
+                                           const Ctl& c) {
+  const bool ok = mbar_wait(bar, parity, c.abort_flag);
+  const bool any_fail = named_barrier_or(bar_id, nthreads, !ok);
+  if (any_fail) fail(c);
+  return !any_fail;
+}
+
+// Tile t's slice of the ranks on the V side: [t r / T, (t + 1) r / T).
+__device__ __forceinline__ void vside_ranks(const FusedParams& p, int t, int& i_lo, int& i_hi) {
+  i_lo = static_cast<int>(static_cast<long long>(t) * p.r / p.T);
+  i_hi = static_cast<int>(static_cast<long long>(t + 1) * p.r / p.T);
+}
+
+// U-side rank blocks of tile t handled by the segment covering units [ua, ub)
+// of the tile (offsets within the tile): proportional to its share of K.
+__device__ __forceinline__ void rank_share(const FusedParams& p, int ua, int ub, int& b_lo, int& b_hi) {
+  const int IBn = (p.r + kRB - 1) / kRB;
+  b_lo = static_cast<int>(static_cast<long long>(IBn) * ua / p.KC);
+  b_hi = static_cast<int>(static_cast<long long>(IBn) * ub / p.KC);
+}
+
+// ------------------------------------------------------------------ staging
+
+// Activation rows m0 .. m0+mcnt, words [ws, ws + nw) (BF16 as stored) -> xb [32][256].
+__device__ __forceinline__ void stage_x(const FusedParams& p, int m0, int mcnt, int ws, int nw,
+                                        uint16_t* xb, int tid) {
+  const int per_row = nw * 4;                       // 16-byte pieces per row
+  for (int idx = tid; idx < mcnt * per_row; idx += kAluThreads) {
+    const int m = idx / per_row, piece = idx % per_row;
+    cp_async16(smem_u32(xb + m * kSubK + piece * 8),
+               p.x + static_cast<size_t>(m0 + m) * p.K + static_cast<size_t>(ws) * 32 + piece * 8);
   }
-  named_barrier(bar_id, nthreads);
-  const bool ok = *shared_ok != 0;
-  named_barrier(bar_id, nthreads);     // everyone has read shared_ok before it is reused
-  return ok;
+}
+// Sign rows i0 .. i0+nr, words [ws, ws + nw) -> vb [nr][8].
+__device__ __forceinline__ void stage_v(const FusedParams& p, int i0, int nr, int ws, int nw,
+                                        uint32_t* vb, int tid) {
+  for (int idx = tid; idx < nr * nw; idx += kAluThreads) {
+    const int i = idx / nw, wl = idx % nw;
+    cp_async4(smem_u32(vb + i * kXWords + wl), p.Vbits + static_cast<size_t>(i0 + i) * p.KW + ws + wl);
+  }
 }
 
 // ------------------------------------------------------------------ V side
 
-// P[m][i] = sum over words [w0, w1) of sum_{k in word, V[k][i0+i] = -1} x[m0+m][k]
-// for i < 16, m < mcnt (<= 32); returned through red (smem) as res[m * 16 + i]
-// in `out` (smem, [32][16]).  All 256 correction threads call this together.
+// One task (warp) over a staged chunk: for ranks 8 rg .. 8 rg + 7 of the staged
+// sign rows and activation rows MG mg .. MG mg + MG-1, accumulate the x whose
+// sign is -1 over words [wa, wb).  Lane l takes bit l of every word.
 template <int MG>
-__device__ void vside_partial(const FusedParams& p, int m0, int mcnt, int i0, int nr, int w0, int w1,
-                              float* x_s, uint32_t* v_s, float* red_s, float* out, int a, int lane,
-                              int tid) {
-  constexpr int kVals = 8 * MG;           // 8 ranks x MG rows per lane
-  const int mgc = (mcnt + MG - 1) / MG;   // m groups
-  const int groups = 2 * mgc;             // x 2 rank groups of 8
-  int KS = 8 / groups;                    // k splits so that tasks == 8 warps
-  if (KS < 1) KS = 1;
-  const int tasks = groups * KS;
-  const bool active = a < tasks;
-  const int ks = a % KS, rest = a / KS, mg = rest % mgc, rg = rest / mgc;
-
-  uint64_t acc2[8][(MG >= 2) ? MG / 2 : 1];
-  float acc1[8];
-#pragma unroll
-  for (int g = 0; g < 8; ++g) {
-    acc1[g] = 0.0f;
-#pragma unroll
-    for (int j = 0; j < ((MG >= 2) ? MG / 2 : 1); ++j) acc2[g][j] = 0ull;
-  }
+__device__ __forceinline__ void vside_task_accumulate(const uint16_t* xb, const uint32_t* vb, int rg,
+                                                      int mg, int wa, int wb, int lane,
+                                                      uint64_t (&acc2)[8][(MG >= 2) ? MG / 2 : 1],
+                                                      float (&acc1)[8]) {
   const uint32_t lane_bit = 1u << lane;
-
-  for (int ws = w0; ws < w1; ws += kXWords) {
-    const int nw = min(kXWords, w1 - ws);
-    named_barrier(kBarAlu, kAluThreads);          // previous sub-block consumed
-    {
-      const int kk = tid;                          // 256 threads <-> 256 k
-      const bool in = kk < nw * 32;
-      for (int m = 0; m < mcnt; ++m) {
-        float v = 0.0f;
-        if (in) v = bf16_bits_to_f32(__ldg(p.x + static_cast<size_t>(m0 + m) * p.K + ws * 32 + kk));
-        x_s[kk * kMpad + m] = v;
-      }
-      if (tid < kRB * kXWords) {
-        const int i = tid / kXWords, wl = tid % kXWords;
-        uint32_t bits = 0;
-        if (i < nr && wl < nw) bits = __ldg(p.Vbits + static_cast<size_t>(i0 + i) * p.KW + ws + wl);
-        v_s[i * kXWords + wl] = bits;
-      }
-    }
-    named_barrier(kBarAlu, kAluThreads);
-    if (active) {
-      const int wa = (ks * kXWords) / KS, wb = ((ks + 1) * kXWords) / KS;
-      for (int wl = wa; wl < min(wb, nw); ++wl) {
-        const float* xr = x_s + (wl * 32 + lane) * kMpad + mg * MG;
-        float xv[MG];
-        if constexpr (MG >= 4) {
+  const uint16_t* xs = xb + (mg * MG) * kSubK + lane;
+  const uint32_t* vs = vb + (rg * 8) * kXWords;
+  for (int wl = wa; wl < wb; ++wl) {
+    float xv[MG];
 #pragma unroll
-          for (int j = 0; j < MG; j += 4) {
-            const float4 q = *reinterpret_cast<const float4*>(xr + j);
-            xv[j] = q.x; xv[j + 1] = q.y; xv[j + 2] = q.z; xv[j + 3] = q.w;
-          }
-        } else {
+    for (int mm = 0; mm < MG; ++mm) xv[mm] = bf16_bits_to_f32(xs[mm * kSubK + wl * 32]);
 #pragma unroll
-          for (int j = 0; j < MG; ++j) xv[j] = xr[j];
-        }
+    for (int g = 0; g < 8; ++g) {
+      const uint32_t flag = vs[g * kXWords + wl] & lane_bit;
+      if constexpr (MG >= 2) {
 #pragma unroll
-        for (int g = 0; g < 8; ++g) {
-          const uint32_t flag = v_s[(rg * 8 + g) * kXWords + wl] & lane_bit;
-          if constexpr (MG >= 2) {
-#pragma unroll
-            for (int j = 0; j < MG / 2; ++j) padd2(acc2[g][j], xv[2 * j], xv[2 * j + 1], flag);
-          } else {
-            padd1(acc1[g], xv[0], flag);
-          }
-        }
+        for (int q = 0; q < MG / 2; ++q) padd2(acc2[g][q], xv[2 * q], xv[2 * q + 1], flag);
+      } else {
+        padd1(acc1[g], xv[0], flag);
       }
     }
   }
-  // reduce over lanes, then over the k splits (fixed order)
+}
+
+// Reduce a task's accumulators over its lanes and store them in red_slot[.].
+template <int MG>
+__device__ __forceinline__ void vside_task_finish(uint64_t (&acc2)[8][(MG >= 2) ? MG / 2 : 1],
+                                                  float (&acc1)[8], float* red_slot, bool store,
+                                                  int lane) {
+  constexpr int kVals = 8 * MG;
   float vals[kVals];
 #pragma unroll
   for (int g = 0; g < 8; ++g) {
     if constexpr (MG >= 2) {
 #pragma unroll
-      for (int j = 0; j < MG / 2; ++j) {
-        vals[g * MG + 2 * j] = lo_f(acc2[g][j]);
-        vals[g * MG + 2 * j + 1] = hi_f(acc2[g][j]);
+      for (int q = 0; q < MG / 2; ++q) {
+        vals[g * MG + 2 * q] = lo_f(acc2[g][q]);
+        vals[g * MG + 2 * q + 1] = hi_f(acc2[g][q]);
       }
     } else {
       vals[g] = acc1[g];
@@ -320,16 +334,178 @@ __device__ void vside_partial(const FusedParams& p, int m0, int mcnt, int i0, in
   }
   warp_reduce_scatter<kVals>(vals, lane);
   constexpr int kOut = (kVals >= 32) ? kVals / 32 : 1;
-  if (active) {
+  if (store) {
 #pragma unroll
-    for (int j = 0; j < kOut; ++j) {
-      const int e = reduce_out_index<kVals>(lane, j);
-      // lanes that share an index after a partial reduction hold equal totals
-      red_s[a * 64 + e] = vals[j];
+    for (int j = 0; j < kOut; ++j) red_slot[reduce_out_index<kVals>(lane, j)] = vals[j];
+  }
+}
+
+// out[m * kVRanks + i] = sum over the staged words [0, nw) of the x[m][k] whose
+// sign V[k][i] is -1, for m < mcnt (<= 32), i < nr (<= 64).  Whole group.
+template <int MG>
+__device__ void vside_chunk(const uint16_t* xb, const uint32_t* vb, int mcnt, int nr, int nw,
+                            float* red_s, float* out, int a, int lane, int tid) {
+  constexpr int kPairs = (MG >= 2) ? MG / 2 : 1;
+  const int mgc = (mcnt + MG - 1) / MG;
+  const int rgc = (nr + 7) / 8;
+  const int groups = rgc * mgc;
+  int KS = kAluWarps / groups;
+  if (KS < 1) KS = 1;
+  const int tasks = groups * KS;
+  for (int base = 0; base < tasks; base += kAluWarps) {
+    const int task = base + a;
+    const bool active = task < tasks;
+    const int ks = task % KS, rest = task / KS, mg = rest % mgc, rg = rest / mgc;
+    uint64_t acc2[8][kPairs];
+    float acc1[8];
+#pragma unroll
+    for (int g = 0; g < 8; ++g) {
+      acc1[g] = 0.0f;
+#pragma unroll
+      for (int q = 0; q < kPairs; ++q) acc2[g][q] = 0ull;
     }
+    if (active) {
+      const int wa = (ks * kXWords) / KS, wb = min(nw, ((ks + 1) * kXWords) / KS);
+      vside_task_accumulate<MG>(xb, vb, rg, mg, wa, wb, lane, acc2, acc1);
+    }
+    vside_task_finish<MG>(acc2, acc1, red_s + a * 64, active, lane);
+    named_barrier(kBarAlu, kAluThreads);
+    // combine the k splits in order
+    const int nout = min(tasks - base, kAluWarps) / KS;    // (rank group, m group) pairs this round
+    for (int idx = tid; idx < nout * 8 * MG; idx += kAluThreads) {
+      const int pair = idx / (8 * MG), e = idx % (8 * MG);
+      const int pg = base / KS + pair;                     // global pair index
+      const int mgi = pg % mgc, rgi = pg / mgc;
+      const int m = mgi * MG + e % MG, i = rgi * 8 + e / MG;
+      float s = 0.0f;
+      for (int k2 = 0; k2 < KS; ++k2) s += red_s[(pair * KS + k2) * 64 + e];
+      if (m < mcnt && i < nr) out[m * kVRanks + i] = s;
+    }
+    named_barrier(kBarAlu, kAluThreads);
+  }
+}
+
+__device__ void vside_chunk_dispatch(const uint16_t* xb, const uint32_t* vb, int mcnt, int nr, int nw,
+                                     float* red_s, float* out, int a, int lane, int tid) {
+  if (mcnt > 4) vside_chunk<8>(xb, vb, mcnt, nr, nw, red_s, out, a, lane, tid);
+  else if (mcnt > 2) vside_chunk<4>(xb, vb, mcnt, nr, nw, red_s, out, a, lane, tid);
+  else if (mcnt > 1) vside_chunk<2>(xb, vb, mcnt, nr, nw, red_s, out, a, lane, tid);
+  else vside_chunk<1>(xb, vb, mcnt, nr, nw, red_s, out, a, lane, tid);
+}
+
+// xs_s[m] = sum of the staged chunk row m (fixed order: lanes, then warps).
+template <int V>
+__device__ void chunk_xsum(const uint16_t* xb, int mcnt, int nw, float* xsw, float* xs_s, int a,
+                           int lane, int tid) {
+  float v[V];
+  const bool in = tid < nw * 32;
+#pragma unroll
+  for (int m = 0; m < V; ++m) v[m] = (m < mcnt && in) ? bf16_bits_to_f32(xb[m * kSubK + tid]) : 0.0f;
+  warp_reduce_scatter<V>(v, lane);
+  // lanes that share an index after a partial reduction hold the same total
+  xsw[a * kMP + reduce_out_index<V>(lane, 0)] = v[0];
+  named_barrier(kBarAlu, kAluThreads);
+  if (tid < mcnt) {
+    float s = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kAluWarps; ++w) s += xsw[w * kMP + tid];
+    xs_s[tid] = s;
   }
   named_barrier(kBarAlu, kAluThreads);
-  // out[m][i] for i < 16, m < mcnt: sum the KS partial tasks in order
+}
+
+__device__ void chunk_xsum_dispatch(const uint16_t* xb, int mcnt, int nw, float* xsw, float* xs_s,
+                                    int a, int lane, int tid) {
+  if (mcnt > 16) chunk_xsum<32>(xb, mcnt, nw, xsw, xs_s, a, lane, tid);
+  else if (mcnt > 8) chunk_xsum<16>(xb, mcnt, nw, xsw, xs_s, a, lane, tid);
+  else if (mcnt > 4) chunk_xsum<8>(xb, mcnt, nw, xsw, xs_s, a, lane, tid);
+  else if (mcnt > 2) chunk_xsum<4>(xb, mcnt, nw, xsw, xs_s, a, lane, tid);
+  else if (mcnt > 1) chunk_xsum<2>(xb, mcnt, nw, xsw, xs_s, a, lane, tid);
+  else chunk_xsum<1>(xb, mcnt, nw, xsw, xs_s, a, lane, tid);
+}
+
+// ------------------------------------------------------------------ activation quantisation
+
+// Rows m < mcnt of the staged chunk (its first nw words) -> B tile (BN rows x 128 B,
+// 128-byte swizzle: 16-byte piece j of row m sits at piece j ^ (m & 7)) and the
+// chunk's 4 scale atoms.  Blocks past K keep whatever finite codes the stage held;
+// the weight codes there are zero-filled by TMA.
+__device__ void quant_chunk(const uint16_t* xb, int mcnt, int nw, uint8_t* btile, uint8_t* sfb, int tid) {
+  const int nblk = 2 * nw;
+  for (int idx = tid; idx < mcnt * nblk; idx += kAluThreads) {
+    const int m = idx / nblk, blk = idx % nblk;
+    const uint4* src = reinterpret_cast<const uint4*>(xb + m * kSubK + blk * 16);
+    float v[16];
+    bf16x16_to_f32(src[0], src[1], v);
+    uint2 codes;
+    const uint32_t s = quant_act_block(v, codes);
+    const int j = blk * 8;
+    *reinterpret_cast<uint2*>(btile + m * 128 + ((((j >> 4) ^ (m & 7)) << 4) | (j & 15))) = codes;
+    sfb[(blk >> 2) * 512 + (m & 31) * 16 + ((m >> 5) & 3) * 4 + (blk & 3)] = static_cast<uint8_t>(s);
+  }
+}
+
+// ------------------------------------------------------------------ local z (mode 2)
+
+// out[m * kVRanks + i] = sum over ALL of K of the x[m0+m][k] whose sign V[k][i0+i]
+// is -1 (i < nr <= 16), and xs_s[m] = sum_k x[m0+m][k].  Whole group.
+template <int MG>
+__device__ void vside_full_k(const FusedParams& p, int m0, int mcnt, int i0, int nr, uint16_t* xb,
+                             uint32_t* vb, float* red_s, float* xs_s, float* out, int a, int lane,
+                             int tid) {
+  constexpr int kPairs = (MG >= 2) ? MG / 2 : 1;
+  const int mgc = (mcnt + MG - 1) / MG;
+  const int groups = 2 * mgc;
+  int KS = kAluWarps / groups;
+  if (KS < 1) KS = 1;
+  const int tasks = groups * KS;
+  const bool active = a < tasks;
+  const int ks = a % KS, rest = a / KS, mg = rest % mgc, rg = rest / mgc;
+  uint64_t acc2[8][kPairs];
+  float acc1[8];
+#pragma unroll
+  for (int g = 0; g < 8; ++g) {
+    acc1[g] = 0.0f;
+#pragma unroll
+    for (int q = 0; q < kPairs; ++q) acc2[g][q] = 0ull;
+  }
+  float xrun = 0.0f;                                 // this thread's share of sum_k x
+  const int nsb = (p.KW + kXWords - 1) / kXWords;
+  stage_x(p, m0, mcnt, 0, min(kXWords, p.KW), xb, tid);
+  stage_v(p, i0, nr, 0, min(kXWords, p.KW), vb, tid);
+  cp_async_commit();
+  for (int j = 0; j < nsb; ++j) {
+    const int ws = j * kXWords, nw = min(kXWords, p.KW - ws);
+    const uint16_t* xcur = xb + (j & 1) * kMP * kSubK;
+    const uint32_t* vcur = vb + (j & 1) * kVRanks * kXWords;
+    if (j + 1 < nsb) {
+      const int ws2 = ws + kXWords, nw2 = min(kXWords, p.KW - ws2);
+      stage_x(p, m0, mcnt, ws2, nw2, xb + ((j + 1) & 1) * kMP * kSubK, tid);
+      stage_v(p, i0, nr, ws2, nw2, vb + ((j + 1) & 1) * kVRanks * kXWords, tid);
+      cp_async_commit();
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    named_barrier(kBarAlu, kAluThreads);
+    if (active) {
+      const int wa = (ks * kXWords) / KS, wb = min(nw, ((ks + 1) * kXWords) / KS);
+      vside_task_accumulate<MG>(xcur, vcur, rg, mg, wa, wb, lane, acc2, acc1);
+    }
+    // thread tid owns row tid / 8 and every 8th element of it for the x sum
+    {
+      const int m = tid >> 3, part = tid & 7;
+      if (m < mcnt)
+        for (int k = part; k < nw * 32; k += 8) xrun += bf16_bits_to_f32(xcur[m * kSubK + k]);
+    }
+    named_barrier(kBarAlu, kAluThreads);
+  }
+  vside_task_finish<MG>(acc2, acc1, red_s + a * 64, active, lane);
+  xrun += __shfl_xor_sync(0xffffffffu, xrun, 4);
+  xrun += __shfl_xor_sync(0xffffffffu, xrun, 2);
+  xrun += __shfl_xor_sync(0xffffffffu, xrun, 1);
+  if ((tid & 7) == 0) xs_s[tid >> 3] = xrun;
+  named_barrier(kBarAlu, kAluThreads);
   for (int idx = tid; idx < kMP * kRB; idx += kAluThreads) {
     const int m = idx / kRB, i = idx % kRB;
     float s = 0.0f;
@@ -338,136 +514,140 @@ __device__ void vside_partial(const FusedParams& p, int m0, int mcnt, int i0, in
       const int task0 = (rgi * mgc + mgi) * KS;
       for (int k2 = 0; k2 < KS; ++k2) s += red_s[(task0 + k2) * 64 + gg * MG + mm];
     }
-    out[idx] = s;
+    out[m * kVRanks + i] = s;
   }
   named_barrier(kBarAlu, kAluThreads);
 }
 
-__device__ void vside_dispatch(const FusedParams& p, int m0, int mcnt, int i0, int nr, int w0, int w1,
-                               float* x_s, uint32_t* v_s, float* red_s, float* out, int a, int lane,
-                               int tid) {
-  if (mcnt > 4)
-    vside_partial<8>(p, m0, mcnt, i0, nr, w0, w1, x_s, v_s, red_s, out, a, lane, tid);
-  else if (mcnt > 2)
-    vside_partial<4>(p, m0, mcnt, i0, nr, w0, w1, x_s, v_s, red_s, out, a, lane, tid);
-  else if (mcnt > 1)
-    vside_partial<2>(p, m0, mcnt, i0, nr, w0, w1, x_s, v_s, red_s, out, a, lane, tid);
-  else
-    vside_partial<1>(p, m0, mcnt, i0, nr, w0, w1, x_s, v_s, red_s, out, a, lane, tid);
+__device__ void vside_full_k_dispatch(const FusedParams& p, int m0, int mcnt, int i0, int nr,
+                                      uint16_t* xb, uint32_t* vb, float* red_s, float* xs_s, float* out,
+                                      int a, int lane, int tid) {
+  if (mcnt > 4) vside_full_k<8>(p, m0, mcnt, i0, nr, xb, vb, red_s, xs_s, out, a, lane, tid);
+  else if (mcnt > 2) vside_full_k<4>(p, m0, mcnt, i0, nr, xb, vb, red_s, xs_s, out, a, lane, tid);
+  else if (mcnt > 1) vside_full_k<2>(p, m0, mcnt, i0, nr, xb, vb, red_s, xs_s, out, a, lane, tid);
+  else vside_full_k<1>(p, m0, mcnt, i0, nr, xb, vb, red_s, xs_s, out, a, lane, tid);
 }
 
 // ------------------------------------------------------------------ U side
 
-// corr[rs][m][n] for the 128 rows of tile t, m in [m0, m0 + mcnt), ranks of
-// rank blocks [b_lo, b_hi).  z comes from z_s (staged [i][kMpad]) and its block
-// sums from zb_s.  Task a: rows 32 (a & 3) + lane; (a >> 2) selects the m half
-// (mcnt > 16) or the rank-block parity (mcnt <= 16).
-template <int MG>
-__device__ void uside_chunk_accumulate(const FusedParams& p, int t, int blk0, int nblk,
-                                       const float* z_s, uint64_t (&acc2)[MG >= 2 ? MG / 2 : 1],
-                                       float& acc1, int mbase, int rs, int RS, int a, int lane) {
-  const int n = t * kTileRows + (a & 3) * 32 + lane;
-  const uint32_t* urow = p.Ubits + static_cast<size_t>(n) * p.RW;
-  for (int bl = 0; bl < nblk; ++bl) {
-    const int blk = blk0 + bl;
-    if (RS == 2 && (blk & 1) != rs) continue;
-    const uint32_t word = __ldg(urow + (blk >> 1)) >> ((blk & 1) * 16);
-    const float* zr = z_s + (bl * kRB) * kMpad + mbase;
-#pragma unroll
-    for (int ii = 0; ii < kRB; ++ii) {
-      const uint32_t flag = word & (1u << ii);
-      if constexpr (MG >= 4) {
-#pragma unroll
-        for (int j = 0; j < MG; j += 4) {
-          const float4 q = *reinterpret_cast<const float4*>(zr + ii * kMpad + j);
-          padd2(acc2[j / 2], q.x, q.y, flag);
-          padd2(acc2[j / 2 + 1], q.z, q.w, flag);
-        }
-      } else if constexpr (MG == 2) {
-        const float2 q = *reinterpret_cast<const float2*>(zr + ii * kMpad);
-        padd2(acc2[0], q.x, q.y, flag);
-      } else {
-        padd1(acc1, zr[ii * kMpad], flag);
-      }
-    }
-  }
-}
+struct AluBufs {
+  uint16_t* xb;
+  uint32_t* vb;
+  float* z_s;
+  float* zb_s;
+  float* corr_s;
+  float* red_s;
+  float* vout;
+  float* xsw;
+  float* xs_s;
+};
 
+// corr[rs][m][row] for the 128 rows of tile t, rows m0 .. m0+mcnt of the batch and
+// the ranks of rank blocks [b_lo, b_hi).  Task a: rows 32 (a & 3) + lane; (a >> 2)
+// picks the upper/lower 16 batch rows (mcnt > 16) or the rank-block parity (else).
 template <int MG>
-__device__ bool uside_pass(const FusedParams& p, int t, int b_lo, int b_hi, int m0, int mcnt,
-                           float* z_s, float* zb_s, float* corr_s, float* x_s, uint32_t* v_s,
-                           float* red_s, float* vout, int a, int lane, int tid) {
+__device__ void uside_pass(const FusedParams& p, int t, int b_lo, int b_hi, int m0, int mcnt,
+                           const AluBufs& B, int a, int lane, int tid) {
+  constexpr int kPairs = (MG >= 2) ? MG / 2 : 1;
   const int RS = (mcnt > 16) ? 1 : 2;
   const int rs = (RS == 2) ? (a >> 2) : 0;
-  const int mbase = (RS == 1) ? (a >> 2) * 16 : 0;      // m offset within the pass
+  const int mbase = (RS == 1) ? (a >> 2) * 16 : 0;
   const int mwidth = (RS == 1) ? 16 : MG;
-  uint64_t acc2[MG >= 2 ? MG / 2 : 1];
+  const int row = (a & 3) * 32 + lane;
+  const uint32_t* urow = p.Ubits + static_cast<size_t>(t * kTileRows + row) * p.RW;
+  const int IBn = (p.r + kRB - 1) / kRB;
+  uint64_t acc2[kPairs];
 #pragma unroll
-  for (int j = 0; j < (MG >= 2 ? MG / 2 : 1); ++j) acc2[j] = 0ull;
+  for (int j = 0; j < kPairs; ++j) acc2[j] = 0ull;
   float acc1 = 0.0f;
   float zsum[MG];
 #pragma unroll
   for (int j = 0; j < MG; ++j) zsum[j] = 0.0f;
 
-  for (int c0 = b_lo; c0 < b_hi; c0 += kZChunkBlocks) {
-    const int nblk = min(kZChunkBlocks, b_hi - c0);
-    named_barrier(kBarAlu, kAluThreads);     // previous chunk consumed
+  // chunks of 8 rank blocks starting on an even block (whole 32-bit sign words)
+  for (int c0 = b_lo & ~1; c0 < b_hi; c0 += kZChunkBlocks) {
+    const int nblk = min(kZChunkBlocks, IBn - c0);
+    uint32_t uw[kZChunkBlocks / 2];
+#pragma unroll
+    for (int q = 0; q < kZChunkBlocks / 2; ++q)
+      uw[q] = (2 * q < nblk && c0 + 2 * q < b_hi) ? __ldg(urow + (c0 >> 1) + q) : 0u;
+    named_barrier(kBarAlu, kAluThreads);            // previous chunk consumed
     if (p.mode == BILOCO_MODE_SHARED_Z) {
-      // stage z[m][16 c0 .. 16 (c0 + nblk)) -> z_s[i][m], block sums -> zb_s[bl][m]
       const int nr = nblk * kRB;
       for (int idx = tid; idx < nr * kMP; idx += kAluThreads) {
         const int m = idx / nr, i = idx % nr;
+        const int rank = c0 * kRB + i;
         float v = 0.0f;
-        if (m < mcnt) v = __ldcg(p.zfin + static_cast<size_t>(m0 + m) * p.rpad + c0 * kRB + i);
-        z_s[i * kMpad + m] = v;
+        if (m < mcnt && rank < p.r && c0 + i / kRB >= b_lo && c0 + i / kRB < b_hi) {
+          if (p.zdirect) {
+            float s = 0.0f;
+            const float* src = p.zpart + static_cast<size_t>(m0 + m) * p.rpad + rank;
+            const size_t stride = static_cast<size_t>(p.M) * p.rpad;
+#pragma unroll 4
+            for (int c = 0; c < p.KC; ++c) s += __ldcg(src + c * stride);
+            v = __fmul_rn(__ldg(p.alpha + rank), s);
+          } else {
+            v = __ldcg(p.zfin + static_cast<size_t>(m0 + m) * p.rpad + rank);
+          }
+        }
+        B.z_s[i * kMpad + m] = v;
       }
-      for (int idx = tid; idx < nblk * kMP; idx += kAluThreads) {
-        const int bl = idx / kMP, m = idx % kMP;
-        zb_s[bl * kMP + m] = (m < mcnt) ? __ldcg(p.zbsum + static_cast<size_t>(c0 + bl) * p.M + m0 + m)
-                                        : 0.0f;
-      }
-      named_barrier(kBarAlu, kAluThreads);
     } else {
-      // local z: compute each rank block over the whole K right here
+      // local z: each needed rank block over the whole K, computed right here
       for (int bl = 0; bl < nblk; ++bl) {
         const int blk = c0 + bl;
+        if (blk < b_lo || blk >= b_hi) continue;      // uniform over the group
         const int i0 = blk * kRB, nr = min(kRB, p.r - i0);
-        vside_dispatch(p, m0, mcnt, i0, nr, 0, p.KW, x_s, v_s, red_s, vout, a, lane, tid);
-        // z = alpha_i * (sum_k x - 2 P)
+        vside_full_k_dispatch(p, m0, mcnt, i0, nr, B.xb, B.vb, B.red_s, B.xs_s, B.vout, a, lane, tid);
         for (int idx = tid; idx < kMP * kRB; idx += kAluThreads) {
           const int m = idx / kRB, i = idx % kRB;
           float z = 0.0f;
-          if (m < mcnt && i < nr) {
-            float xs = 0.0f;
-            for (int w = 0; w < p.KW; ++w)
-              xs += __ldg(p.xsum32 + static_cast<size_t>(m0 + m) * p.KW + w);
-            z = __fmul_rn(__ldg(p.alpha + i0 + i), xs - 2.0f * vout[idx]);
-          }
-          z_s[(bl * kRB + i) * kMpad + m] = z;
-        }
-        named_barrier(kBarAlu, kAluThreads);
-        for (int idx = tid; idx < kMP; idx += kAluThreads) {
-          float s = 0.0f;
-          for (int i = 0; i < kRB; ++i) s += z_s[(bl * kRB + i) * kMpad + idx];
-          zb_s[bl * kMP + idx] = s;
+          if (m < mcnt && i < nr)
+            z = __fmul_rn(__ldg(p.alpha + i0 + i), B.xs_s[m] - 2.0f * B.vout[m * kVRanks + i]);
+          B.z_s[(bl * kRB + i) * kMpad + m] = z;
         }
         named_barrier(kBarAlu, kAluThreads);
       }
     }
-    // accumulate this chunk
-    uside_chunk_accumulate<MG>(p, t, c0, nblk, z_s, acc2, acc1, mbase, rs, RS, a, lane);
+    named_barrier(kBarAlu, kAluThreads);
+    // block sums of the staged z, then the sign accumulation
+    for (int idx = tid; idx < nblk * kMP; idx += kAluThreads) {
+      const int bl = idx / kMP, m = idx % kMP;
+      float s = 0.0f;
 #pragma unroll
-    for (int j = 0; j < MG; ++j) {
-      if (j < mwidth) {
-        float s = 0.0f;
-        for (int bl = 0; bl < nblk; ++bl)
-          if (RS == 1 || ((c0 + bl) & 1) == rs) s += zb_s[bl * kMP + mbase + j];
-        zsum[j] += s;
+      for (int i = 0; i < kRB; ++i) s += B.z_s[(bl * kRB + i) * kMpad + m];
+      B.zb_s[bl * kMP + m] = s;
+    }
+    named_barrier(kBarAlu, kAluThreads);
+#pragma unroll
+    for (int bl = 0; bl < kZChunkBlocks; ++bl) {
+      const int blk = c0 + bl;
+      if (bl >= nblk || blk < b_lo || blk >= b_hi) continue;
+      if (RS == 2 && (blk & 1) != rs) continue;
+      const uint32_t word = uw[bl >> 1] >> ((bl & 1) * 16);
+      const float* zr = B.z_s + (bl * kRB) * kMpad + mbase;
+#pragma unroll
+      for (int ii = 0; ii < kRB; ++ii) {
+        const uint32_t flag = word & (1u << ii);
+        if constexpr (MG >= 4) {
+#pragma unroll
+          for (int j = 0; j < MG; j += 4) {
+            const float4 q = *reinterpret_cast<const float4*>(zr + ii * kMpad + j);
+            padd2(acc2[j / 2], q.x, q.y, flag);
+            padd2(acc2[j / 2 + 1], q.z, q.w, flag);
+          }
+        } else if constexpr (MG == 2) {
+          const float2 q = *reinterpret_cast<const float2*>(zr + ii * kMpad);
+          padd2(acc2[0], q.x, q.y, flag);
+        } else {
+          padd1(acc1, zr[ii * kMpad], flag);
+        }
       }
+#pragma unroll
+      for (int j = 0; j < MG; ++j)
+        if (j < mwidth) zsum[j] += B.zb_s[bl * kMP + mbase + j];
     }
   }
-  // corr = zsum - 2 * acc, written as corr_s[rs][m][row]
-  const int row = (a & 3) * 32 + lane;
   float accf[MG];
 #pragma unroll
   for (int j = 0; j < MG; ++j) {
@@ -478,26 +658,33 @@ __device__ bool uside_pass(const FusedParams& p, int t, int b_lo, int b_hi, int 
   for (int j = 0; j < MG; ++j) {
     const int m = mbase + j;
     if (j < mwidth && m < kMP) {
-      corr_s[(rs * kMP + m) * kTileRows + row] = zsum[j] - 2.0f * accf[j];
-      if (RS == 1) corr_s[(1 * kMP + m) * kTileRows + row] = 0.0f;
+      B.corr_s[(rs * kMP + m) * kTileRows + row] = zsum[j] - 2.0f * accf[j];
+      if (RS == 1) B.corr_s[(1 * kMP + m) * kTileRows + row] = 0.0f;
     }
   }
-  return true;
 }
 
 __device__ void uside_dispatch(const FusedParams& p, int t, int b_lo, int b_hi, int m0, int mcnt,
-                               float* z_s, float* zb_s, float* corr_s, float* x_s, uint32_t* v_s,
-                               float* red_s, float* vout, int a, int lane, int tid) {
-  if (mcnt > 8)
-    uside_pass<16>(p, t, b_lo, b_hi, m0, mcnt, z_s, zb_s, corr_s, x_s, v_s, red_s, vout, a, lane, tid);
-  else if (mcnt > 4)
-    uside_pass<8>(p, t, b_lo, b_hi, m0, mcnt, z_s, zb_s, corr_s, x_s, v_s, red_s, vout, a, lane, tid);
-  else if (mcnt > 2)
-    uside_pass<4>(p, t, b_lo, b_hi, m0, mcnt, z_s, zb_s, corr_s, x_s, v_s, red_s, vout, a, lane, tid);
-  else if (mcnt > 1)
-    uside_pass<2>(p, t, b_lo, b_hi, m0, mcnt, z_s, zb_s, corr_s, x_s, v_s, red_s, vout, a, lane, tid);
-  else
-    uside_pass<1>(p, t, b_lo, b_hi, m0, mcnt, z_s, zb_s, corr_s, x_s, v_s, red_s, vout, a, lane, tid);
+                               const AluBufs& B, int a, int lane, int tid) {
+  if (mcnt > 8) uside_pass<16>(p, t, b_lo, b_hi, m0, mcnt, B, a, lane, tid);
+  else if (mcnt > 4) uside_pass<8>(p, t, b_lo, b_hi, m0, mcnt, B, a, lane, tid);
+  else if (mcnt > 2) uside_pass<4>(p, t, b_lo, b_hi, m0, mcnt, B, a, lane, tid);
+  else if (mcnt > 1) uside_pass<2>(p, t, b_lo, b_hi, m0, mcnt, B, a, lane, tid);
+  else uside_pass<1>(p, t, b_lo, b_hi, m0, mcnt, B, a, lane, tid);
+}
+
+// Warm L2 with the sign rows of U this CTA's U side will read.
+__device__ void prefetch_u_rows(const FusedParams& p, int u0, int u1, int tid) {
+  const int t_first = u0 / p.KC, t_last = (u1 - 1) / p.KC;
+  for (int t = t_first; t <= t_last && t < t_first + 2; ++t) {
+    int b_lo, b_hi;
+    rank_share(p, max(u0, t * p.KC) - t * p.KC, min(u1, (t + 1) * p.KC) - t * p.KC, b_lo, b_hi);
+    if (b_hi <= b_lo) continue;
+    const int wlo = b_lo / 2, whi = (b_hi + 1) / 2;
+    for (int row = tid; row < kTileRows; row += kAluThreads)
+      for (int w = wlo; w < whi; w += 32)
+        prefetch_l2(p.Ubits + static_cast<size_t>(t * kTileRows + row) * p.RW + w);
+  }
 }
 
 // ------------------------------------------------------------------ the kernel
@@ -505,6 +692,7 @@ __device__ void uside_dispatch(const FusedParams& p, int t, int b_lo, int b_hi, 
 template <int BN, int ST>
 __global__ void __launch_bounds__(kThreads, 1)
 fused_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
+             const __grid_constant__ CUtensorMap tmap_xs, const __grid_constant__ CUtensorMap tmap_v,
              const __grid_constant__ FusedParams p) {
   using L = Layout<BN, ST>;
   extern __shared__ uint8_t smem_raw[];
@@ -520,10 +708,9 @@ fused_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
   const uint32_t corrf_bar = smem_u32(&bars[2 * ST + 4]);
   const uint32_t corre_bar = smem_u32(&bars[2 * ST + 5]);
   const uint32_t drain_bar = smem_u32(&bars[2 * ST + 6]);
+  auto xfull_bar = [&](int s) { return smem_u32(&bars[2 * ST + 7 + s]); };
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
-  volatile int* epi_ok = reinterpret_cast<volatile int*>(smem + L::kMisc + 8);
-  volatile int* alu_ok = reinterpret_cast<volatile int*>(smem + L::kMisc + 12);
   volatile int* epi_last = reinterpret_cast<volatile int*>(smem + L::kMisc + 16);
   volatile int* alu_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 20);
   const Ctl ctl{abort_flag, p.status};
@@ -532,12 +719,20 @@ fused_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
   const int u0 = first_unit(g, p.G, p.U), u1 = first_unit(g + 1, p.G, p.U);
   const int t_first = u0 / p.KC, t_last = (u1 - 1) / p.KC;
   const int nseg = t_last - t_first + 1;
+  const int nunits = u1 - u0;
   const int npass = (p.M + kMP - 1) / kMP;
 
   if (threadIdx.x == 0) {
+    prefetch_tmap(&tmap_w);
+    if (!p.inq) prefetch_tmap(&tmap_x);
+    if (p.fast) {
+      prefetch_tmap(&tmap_xs);
+      if (p.r > 0) prefetch_tmap(&tmap_v);
+    }
     for (int s = 0; s < ST; ++s) {
-      mbar_init(full_bar(s), 1);
-      mbar_init(empty_bar(s), 1);
+      mbar_init(full_bar(s), p.inq ? 2 : 1);     // + the quantiser's arrival when in-kernel
+      mbar_init(empty_bar(s), p.fast ? 2 : 1);   // + the CUDA cores releasing the staged x
+      mbar_init(xfull_bar(s), 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(accf_bar(b), 1);
@@ -553,10 +748,6 @@ fused_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
     tmem_alloc(smem_u32(tmem_holder), kTmemCols);
     tmem_relinquish();
   }
-  if (warp == 0 && lane == 0) {
-    prefetch_tmap(&tmap_w);
-    prefetch_tmap(&tmap_x);
-  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -565,10 +756,25 @@ fused_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
     if (lane == 0) {
-      const int nunits = u1 - u0;
       const int pre = min(ST, nunits);
-      const uint32_t stage_bytes = kUnitBytesA + BN * 128 + 2 * kSfBytes;
-      // weight bytes do not depend on the activation quantiser: start them first
+      const uint32_t stage_bytes = kUnitBytesA + kSfBytes + (p.inq ? 0u : BN * 128 + kSfBytes);
+      const bool vstage = p.fast && p.r > 0 && p.mode == BILOCO_MODE_SHARED_Z;
+      const uint32_t xstage_bytes = static_cast<uint32_t>(p.bxr * kSubK * 2) + (vstage ? L::kVBytes : 0u);
+      auto issue_x = [&](int k, int s) {
+        const int u = u0 + k, t = u / p.KC, c = u % p.KC;
+        mbar_arrive_expect_tx(xfull_bar(s), xstage_bytes);
+        tma_load_2d(smem_u32(smem + L::kXS + s * L::kXStride), &tmap_xs, xfull_bar(s), c * kSubK, 0);
+        if (vstage) {
+          int i_lo, i_hi;
+          vside_ranks(p, t, i_lo, i_hi);
+          tma_load_2d(smem_u32(smem + L::kXS + s * L::kXStride + L::kXBytes), &tmap_v, xfull_bar(s),
+                      c * kXWords, i_lo);
+        }
+      };
+      // the CUDA cores' inputs first, then the weight bytes (they do not depend on
+      // the activation)
+      if (p.fast)
+        for (int k = 0; k < pre; ++k) issue_x(k, k);
       for (int k = 0; k < pre; ++k) {
         const int u = u0 + k, t = u / p.KC, c = u % p.KC;
         mbar_arrive_expect_tx(full_bar(k), stage_bytes);
@@ -577,12 +783,14 @@ fused_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
         bulk_load(smem_u32(smem + L::kSFA + k * kSfBytes),
                   p.w_sf + (static_cast<size_t>(t) * p.KC + c) * kSfBytes, kSfBytes, full_bar(k));
       }
-      griddep_wait();
-      for (int k = 0; k < pre; ++k) {
-        const int c = (u0 + k) % p.KC;
-        tma_load_2d(smem_u32(smem + L::kB + k * BN * 128), &tmap_x, full_bar(k), c * 128, 0);
-        bulk_load(smem_u32(smem + L::kSFB + k * kSfBytes), p.x_sf + static_cast<size_t>(c) * kSfBytes,
-                  kSfBytes, full_bar(k));
+      if (!p.inq) {
+        griddep_wait();
+        for (int k = 0; k < pre; ++k) {
+          const int c = (u0 + k) % p.KC;
+          tma_load_2d(smem_u32(smem + L::kB + k * BN * 128), &tmap_x, full_bar(k), c * 128, 0);
+          bulk_load(smem_u32(smem + L::kSFB + k * kSfBytes), p.x_sf + static_cast<size_t>(c) * kSfBytes,
+                    kSfBytes, full_bar(k));
+        }
       }
       int issued = pre;
       for (int k = pre; k < nunits; ++k) {
@@ -592,20 +800,24 @@ fused_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
           break;
         }
         const int u = u0 + k, t = u / p.KC, c = u % p.KC;
+        if (p.fast) issue_x(k, s);
         mbar_arrive_expect_tx(full_bar(s), stage_bytes);
         tma_load_2d(smem_u32(smem + L::kA + s * kUnitBytesA), &tmap_w, full_bar(s), c * 128,
                     t * kTileRows);
         bulk_load(smem_u32(smem + L::kSFA + s * kSfBytes),
                   p.w_sf + (static_cast<size_t>(t) * p.KC + c) * kSfBytes, kSfBytes, full_bar(s));
-        tma_load_2d(smem_u32(smem + L::kB + s * BN * 128), &tmap_x, full_bar(s), c * 128, 0);
-        bulk_load(smem_u32(smem + L::kSFB + s * kSfBytes), p.x_sf + static_cast<size_t>(c) * kSfBytes,
-                  kSfBytes, full_bar(s));
+        if (!p.inq) {
+          tma_load_2d(smem_u32(smem + L::kB + s * BN * 128), &tmap_x, full_bar(s), c * 128, 0);
+          bulk_load(smem_u32(smem + L::kSFB + s * kSfBytes), p.x_sf + static_cast<size_t>(c) * kSfBytes,
+                    kSfBytes, full_bar(s));
+        }
         ++issued;
       }
       // never leave the CTA with copies in flight: wait for the last fills
       for (int k = max(0, issued - ST); k < issued; ++k) {
         const uint64_t t0 = globaltimer_ns();
-        while (!mbar_try_wait(full_bar(k % ST), (k / ST) & 1)) {
+        while (!mbar_try_wait(full_bar(k % ST), (k / ST) & 1) ||
+               (p.fast && !mbar_try_wait(xfull_bar(k % ST), (k / ST) & 1))) {
           if (globaltimer_ns() - t0 > kWaitLimitNs) {
             record_error(p.status, kDevErrTimeout);
             break;
@@ -613,6 +825,7 @@ fused_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
         }
       }
     }
+    __syncwarp();
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
@@ -668,9 +881,9 @@ fused_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
         }
       }
     }
+    __syncwarp();
   } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + 4) {
     // ---------------------------------------------------------------- epilogue
-    const int et = threadIdx.x - kEpiWarp0 * 32;      // 0..127
     const int q = warp & 3;                            // TMEM lane quarter of this warp
     const int row = q * 32 + lane;                     // weight row within the tile
     const float gs = __ldg(p.gscale);
@@ -683,7 +896,7 @@ fused_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
       const bool sole = hf == hl;
       const int which = (t == t_first) ? 0 : 1;
       float* my_slot = p.slots + static_cast<size_t>(2 * g + which) * BN * kTileRows;
-      if (!group_wait(accf_bar(b), (seg >> 1) & 1, et == 0, kBarEpi, kEpiThreads, epi_ok, ctl)) break;
+      if (!group_wait(accf_bar(b), (seg >> 1) & 1, kBarEpi, kEpiThreads, ctl)) break;
       tc_fence_after();
       bool ok = true;
       for (int pass = 0; pass < npass; ++pass) {
@@ -710,7 +923,7 @@ fused_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
 #pragma unroll
         for (int j = 0; j < kMP; ++j) v[j] = __fmul_rn(gs, v[j]);
         if (p.r > 0) {
-          if (!group_wait(corrf_bar, corr_round & 1, et == 0, kBarEpi, kEpiThreads, epi_ok, ctl)) {
+          if (!group_wait(corrf_bar, corr_round & 1, kBarEpi, kEpiThreads, ctl)) {
             ok = false;
             break;
           }
@@ -725,7 +938,8 @@ fused_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
           uint16_t* yb = p.y + static_cast<size_t>(t) * kTileRows + row;
 #pragma unroll
           for (int j = 0; j < kMP; ++j)
-            if (j < mcnt) yb[static_cast<size_t>(m0 + j) * p.N] = __bfloat16_as_ushort(__float2bfloat16_rn(v[j]));
+            if (j < mcnt)
+              yb[static_cast<size_t>(m0 + j) * p.N] = __bfloat16_as_ushort(__float2bfloat16_rn(v[j]));
         } else {
 #pragma unroll
           for (int j = 0; j < kMP; ++j)
@@ -736,25 +950,40 @@ fused_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
       mbar_arrive(acce_bar(b));
       if (!ok) break;
       if (!sole) {
+        // publish this partial; the last contributor of the tile sums all of them
         __threadfence();
         named_barrier(kBarEpi, kEpiThreads);
-        if (et == 0) {
-          const uint32_t contributors = static_cast<uint32_t>(hl - hf + 1);
-          const uint32_t old = atomicAdd(p.tickets + t, 1u);
-          const bool last = (old == contributors - 1);
-          if (last) atomicExch(p.tickets + t, 0u);
-          __threadfence();
-          *epi_last = last ? 1 : 0;
+        if (warp == kEpiWarp0) {
+          if (lane == 0) {
+            const uint32_t contributors = static_cast<uint32_t>(hl - hf + 1);
+            const uint32_t old = atomicAdd(p.tickets + t, 1u);
+            const bool last = (old == contributors - 1);
+            if (last) atomicExch(p.tickets + t, 0u);
+            __threadfence();
+            *epi_last = last ? 1 : 0;
+          }
+          __syncwarp();
         }
         named_barrier(kBarEpi, kEpiThreads);
         const bool last = *epi_last != 0;
         named_barrier(kBarEpi, kEpiThreads);
         if (last) {
+#pragma unroll 2
           for (int m = 0; m < p.M; ++m) {
             float s = 0.0f;
-            for (int h = hf; h <= hl; ++h) {
-              const int wh = (t == first_unit(h, p.G, p.U) / p.KC) ? 0 : 1;
-              s += __ldcg(p.slots + (static_cast<size_t>(2 * h + wh) * BN + m) * kTileRows + row);
+            for (int h0 = hf; h0 <= hl; h0 += 8) {
+              float part[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const int h = h0 + e;
+                part[e] = 0.0f;
+                if (h <= hl) {
+                  const int wh = (t == first_unit(h, p.G, p.U) / p.KC) ? 0 : 1;
+                  part[e] = __ldcg(p.slots + (static_cast<size_t>(2 * h + wh) * BN + m) * kTileRows + row);
+                }
+              }
+#pragma unroll
+              for (int e = 0; e < 8; ++e) s += part[e];
             }
             p.y[static_cast<size_t>(m) * p.N + static_cast<size_t>(t) * kTileRows + row] =
                 __bfloat16_as_ushort(__float2bfloat16_rn(s));
@@ -762,117 +991,250 @@ fused_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
         }
       }
     }
-  } else if (warp >= kAluWarp0 && warp < kAluWarp0 + kAluWarps && p.r > 0) {
-    // ---------------------------------------------------------------- sign correction
+  } else if (warp >= kAluWarp0 && warp < kAluWarp0 + kAluWarps && (p.r > 0 || p.inq)) {
+    // ---------------------------------------------------------------- CUDA-core work
     const int tid = threadIdx.x - kAluWarp0 * 32;   // 0..255
     const int a = warp - kAluWarp0;                  // task slot 0..7
-    float* x_s = reinterpret_cast<float*>(smem + L::kXS);
-    float* z_s = reinterpret_cast<float*>(smem + L::kZS);
-    float* zb_s = reinterpret_cast<float*>(smem + L::kZB);
-    uint32_t* v_s = reinterpret_cast<uint32_t*>(smem + L::kVS);
-    float* corr_s = reinterpret_cast<float*>(smem + L::kCorr);
-    float* red_s = reinterpret_cast<float*>(smem + L::kRed);
-    float* vout = reinterpret_cast<float*>(smem + L::kVOut);
+    AluBufs B;
+    B.xb = reinterpret_cast<uint16_t*>(smem + L::kXB);
+    B.vb = reinterpret_cast<uint32_t*>(smem + L::kVB);
+    B.z_s = reinterpret_cast<float*>(smem + L::kZS);
+    B.zb_s = reinterpret_cast<float*>(smem + L::kZB);
+    B.corr_s = reinterpret_cast<float*>(smem + L::kCorr);
+    B.red_s = reinterpret_cast<float*>(smem + L::kRed);
+    B.vout = reinterpret_cast<float*>(smem + L::kVOut);
+    B.xsw = reinterpret_cast<float*>(smem + L::kXsw);
+    B.xs_s = reinterpret_cast<float*>(smem + L::kXsum);
+    const bool shared_z = p.r > 0 && p.mode == BILOCO_MODE_SHARED_Z;
     bool ok = true;
 
-    if (p.mode == BILOCO_MODE_SHARED_Z) {
-      // V side: this CTA's slices (kb, ib) of V^T x
-      const int items = p.KB * p.IB;
-      float* part = vout;                    // [32][16] V-side result
-      for (int item = g; item < items; item += p.G) {
-        const int kb = item / p.IB, ib = item % p.IB;
-        const int w0 = static_cast<int>(static_cast<long long>(kb) * p.KW / p.KB);
-        const int w1 = static_cast<int>(static_cast<long long>(kb + 1) * p.KW / p.KB);
-        const int i0 = ib * kRB, nr = min(kRB, p.r - i0);
-        for (int pass = 0; pass < npass; ++pass) {
-          const int m0 = pass * kMP, mcnt = min(kMP, p.M - m0);
-          vside_dispatch(p, m0, mcnt, i0, nr, w0, w1, x_s, v_s, red_s, part, a, lane, tid);
-          for (int idx = tid; idx < mcnt * kRB; idx += kAluThreads) {
-            const int m = idx / kRB, i = idx % kRB;
-            float xs = 0.0f;
-            for (int w = w0; w < w1; ++w) xs += __ldg(p.xsum32 + static_cast<size_t>(m0 + m) * p.KW + w);
-            p.zpart[((static_cast<size_t>(kb) * p.IB + ib) * p.M + m0 + m) * kRB + i] =
-                xs - 2.0f * part[m * kRB + i];
-          }
+    if (p.r > 0) prefetch_u_rows(p, u0, u1, tid);
+    if (p.inq) {
+      // B tile rows >= M and unused scale bytes stay zero for the whole launch
+      constexpr int kPer = (BN * 128 + kSfBytes) / 16;
+      for (int idx = tid; idx < ST * kPer; idx += kAluThreads) {
+        const int s = idx / kPer, o = idx % kPer;
+        uint4* dst = (o < BN * 8) ? reinterpret_cast<uint4*>(smem + L::kB + s * BN * 128) + o
+                                  : reinterpret_cast<uint4*>(smem + L::kSFB + s * kSfBytes) + (o - BN * 8);
+        *dst = make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+
+    if (p.fast) {
+      // ---- per unit, on the x chunk and V rows the producer staged: quantise
+      // (small M), x sums and the V side, then release the staging slot
+      for (int k = 0; k < nunits && ok; ++k) {
+        const int u = u0 + k, t = u / p.KC, c = u % p.KC, s = k % ST;
+        const int nw = min(kXWords, p.KW - c * kXWords);
+        const uint16_t* xcur = reinterpret_cast<const uint16_t*>(smem + L::kXS + s * L::kXStride);
+        const uint32_t* vcur = reinterpret_cast<const uint32_t*>(smem + L::kXS + s * L::kXStride + L::kXBytes);
+        if (!group_wait(xfull_bar(s), (k / ST) & 1, kBarAlu, kAluThreads, ctl)) {
+          ok = false;
+          break;
         }
-        // publish; the last K block of this rank block finalises it
-        __threadfence();
-        named_barrier(kBarAlu, kAluThreads);
-        if (tid == 0) {
-          const uint32_t old = atomicAdd(p.rb_count + ib, 1u);
-          const bool last = old == static_cast<uint32_t>(p.KB - 1);
-          if (last) atomicExch(p.rb_count + ib, 0u);
-          __threadfence();
-          *alu_flag = last ? 1 : 0;
-        }
-        named_barrier(kBarAlu, kAluThreads);
-        const bool last = *alu_flag != 0;
-        named_barrier(kBarAlu, kAluThreads);
-        if (last) {
-          // warp-uniform trip count: the shuffles below need all 32 lanes
-          for (int base = 0; base < p.M * kRB; base += kAluThreads) {
-            const int idx = base + tid;
-            const bool live = idx < p.M * kRB;
-            const int m = idx / kRB, i = idx % kRB;
-            float z = 0.0f;
-            if (live) {
-              float s = 0.0f;
-              for (int kb2 = 0; kb2 < p.KB; ++kb2)
-                s += __ldcg(p.zpart + ((static_cast<size_t>(kb2) * p.IB + ib) * p.M + m) * kRB + i);
-              z = (i < nr) ? __fmul_rn(__ldg(p.alpha + i0 + i), s) : 0.0f;
-              p.zfin[static_cast<size_t>(m) * p.rpad + i0 + i] = z;
-            }
-            // block sum over the 16 ranks (16 consecutive threads share m)
-            float bs = z;
-#pragma unroll
-            for (int o = 8; o >= 1; o >>= 1) bs += __shfl_xor_sync(0xffffffffu, bs, o);
-            if (live && i == 0) p.zbsum[static_cast<size_t>(ib) * p.M + m] = bs;
-          }
-          __threadfence();
+        const int mcnt = p.M;                          // fast path: M <= 32, one pass
+        if (p.inq) {
+          quant_chunk(xcur, mcnt, nw, smem + L::kB + s * BN * 128, smem + L::kSFB + s * kSfBytes, tid);
+          fence_proxy_async_smem();
           named_barrier(kBarAlu, kAluThreads);
-          if (tid == 0) atomicAdd(p.z_ready, 1u);
+          if (a == 0) {
+            if (lane == 0) mbar_arrive(full_bar(s));
+            __syncwarp();
+          }
+        }
+        if (shared_z) {
+          int i_lo, i_hi;
+          vside_ranks(p, t, i_lo, i_hi);
+          chunk_xsum_dispatch(xcur, mcnt, nw, B.xsw, B.xs_s, a, lane, tid);
+          for (int r0 = i_lo; r0 < i_hi; r0 += kVRanks) {
+            const int nr = min(kVRanks, i_hi - r0);
+            vside_chunk_dispatch(xcur, vcur + (r0 - i_lo) * kXWords, mcnt, nr, nw, B.red_s, B.vout, a,
+                                 lane, tid);
+            for (int idx = tid; idx < mcnt * nr; idx += kAluThreads) {
+              const int m = idx / nr, i = idx % nr;
+              p.zpart[(static_cast<size_t>(c) * p.M + m) * p.rpad + r0 + i] =
+                  B.xs_s[m] - 2.0f * B.vout[m * kVRanks + i];
+            }
+            named_barrier(kBarAlu, kAluThreads);
+          }
+        }
+        named_barrier(kBarAlu, kAluThreads);           // every read of the slot is done
+        if (a == 0) {
+          if (lane == 0) mbar_arrive(empty_bar(s));
+          __syncwarp();
         }
       }
-      // wait until every rank block is final, then count ourselves out
-      if (tid == 0) {
-        bool okw = spin_until_geq(p.z_ready, static_cast<uint32_t>(p.IB), ctl);
-        if (!okw) fail(ctl);
-        *alu_ok = okw ? 1 : 0;
-        if (okw) {
+    } else if (p.unit_alu) {
+      // ---- per unit: stage the chunk, quantise it (small M), V side (shared z).
+      // A job is (unit, batch pass, V rank sub-range); the next job is prefetched.
+      auto nsub_of = [&](int t) {
+        if (!shared_z) return 1;
+        int i_lo, i_hi;
+        vside_ranks(p, t, i_lo, i_hi);
+        return max(1, (i_hi - i_lo + kVRanks - 1) / kVRanks);
+      };
+      auto stage_job = [&](int k, int jk, int buf) {
+        const int u = u0 + k, t = u / p.KC, c = u % p.KC;
+        const int nw = min(kXWords, p.KW - c * kXWords);
+        const int nsub = nsub_of(t);
+        const int pass = jk / nsub, sub = jk % nsub;
+        const int m0 = pass * kMP, mcnt = min(kMP, p.M - m0);
+        stage_x(p, m0, mcnt, c * kXWords, nw, B.xb + buf * kMP * kSubK, tid);
+        if (shared_z) {
+          int i_lo, i_hi;
+          vside_ranks(p, t, i_lo, i_hi);
+          const int r0 = i_lo + sub * kVRanks, nr = min(kVRanks, i_hi - r0);
+          if (nr > 0) stage_v(p, r0, nr, c * kXWords, nw, B.vb + buf * kVRanks * kXWords, tid);
+        }
+      };
+      int buf = 0;
+      stage_job(0, 0, 0);
+      cp_async_commit();
+      for (int k = 0; k < nunits && ok; ++k) {
+        const int u = u0 + k, t = u / p.KC, c = u % p.KC, s = k % ST;
+        const int nw = min(kXWords, p.KW - c * kXWords);
+        const int nsub = nsub_of(t);
+        const int njobs = npass * nsub;
+        int i_lo = 0, i_hi = 0;
+        if (shared_z) vside_ranks(p, t, i_lo, i_hi);
+        for (int jk = 0; jk < njobs && ok; ++jk) {
+          const bool more = (jk + 1 < njobs) || (k + 1 < nunits);
+          if (more) {
+            if (jk + 1 < njobs) stage_job(k, jk + 1, buf ^ 1);
+            else stage_job(k + 1, 0, buf ^ 1);
+            cp_async_commit();
+            cp_async_wait<1>();
+          } else {
+            cp_async_wait<0>();
+          }
+          named_barrier(kBarAlu, kAluThreads);
+          const uint16_t* xcur = B.xb + buf * kMP * kSubK;
+          const int pass = jk / nsub, sub = jk % nsub;
+          const int m0 = pass * kMP, mcnt = min(kMP, p.M - m0);
+          if (p.inq && jk == 0) {
+            // the stage must be free before its B tile is rewritten
+            if (k >= ST && !group_wait(empty_bar(s), ((k / ST) - 1) & 1, kBarAlu, kAluThreads, ctl)) {
+              ok = false;
+              break;
+            }
+            quant_chunk(xcur, mcnt, nw, smem + L::kB + s * BN * 128, smem + L::kSFB + s * kSfBytes, tid);
+            fence_proxy_async_smem();
+            named_barrier(kBarAlu, kAluThreads);
+            if (a == 0) {
+              if (lane == 0) mbar_arrive(full_bar(s));
+              __syncwarp();
+            }
+          }
+          if (shared_z) {
+            const int r0 = i_lo + sub * kVRanks, nr = min(kVRanks, i_hi - r0);
+            if (sub == 0) chunk_xsum_dispatch(xcur, mcnt, nw, B.xsw, B.xs_s, a, lane, tid);
+            if (nr > 0) {
+              vside_chunk_dispatch(xcur, B.vb + buf * kVRanks * kXWords, mcnt, nr, nw, B.red_s, B.vout, a,
+                                   lane, tid);
+              for (int idx = tid; idx < mcnt * nr; idx += kAluThreads) {
+                const int m = idx / nr, i = idx % nr;
+                p.zpart[(static_cast<size_t>(c) * p.M + m0 + m) * p.rpad + r0 + i] =
+                    B.xs_s[m] - 2.0f * B.vout[m * kVRanks + i];
+              }
+            }
+          }
+          named_barrier(kBarAlu, kAluThreads);     // buffer `buf` may be refilled
+          buf ^= 1;
+        }
+      }
+      if (!ok) cp_async_wait<0>();
+    }
+
+    if (shared_z && ok) {
+      // ---- publish the chunk partials; finalise (larger M) or count in (direct)
+      __threadfence();
+      named_barrier(kBarAlu, kAluThreads);
+      if (p.zdirect) {
+        if (a == 0) {
+          if (lane == 0) atomicAdd(p.z_ready, 1u);
+          __syncwarp();
+        }
+      } else {
+        for (int seg = 0; seg < nseg; ++seg) {
+          const int t = t_first + seg;
+          if (a == 0) {
+            if (lane == 0) {
+              const int hf = owner_cta(static_cast<long long>(t) * p.KC, p.G, p.U);
+              const int hl = owner_cta(static_cast<long long>(t + 1) * p.KC - 1, p.G, p.U);
+              const uint32_t old = atomicAdd(p.vtick + t, 1u);
+              const bool last = old == static_cast<uint32_t>(hl - hf);
+              if (last) atomicExch(p.vtick + t, 0u);
+              __threadfence();
+              *alu_flag = last ? 1 : 0;
+            }
+            __syncwarp();
+          }
+          named_barrier(kBarAlu, kAluThreads);
+          const bool last = *alu_flag != 0;
+          named_barrier(kBarAlu, kAluThreads);
+          if (last) {
+            int i_lo, i_hi;
+            vside_ranks(p, t, i_lo, i_hi);
+            const int nr = i_hi - i_lo;
+            const size_t stride = static_cast<size_t>(p.M) * p.rpad;
+            for (int idx = tid; idx < p.M * nr; idx += kAluThreads) {
+              const int m = idx / nr, i = i_lo + idx % nr;
+              const float* src = p.zpart + static_cast<size_t>(m) * p.rpad + i;
+              float s = 0.0f;
+#pragma unroll 4
+              for (int c = 0; c < p.KC; ++c) s += __ldcg(src + c * stride);
+              p.zfin[static_cast<size_t>(m) * p.rpad + i] = __fmul_rn(__ldg(p.alpha + i), s);
+            }
+            __threadfence();
+            named_barrier(kBarAlu, kAluThreads);
+            if (a == 0) {
+              if (lane == 0) atomicAdd(p.z_ready, 1u);
+              __syncwarp();
+            }
+          }
+        }
+      }
+      // wait until every partial (or every finished tile slice) is visible
+      const uint32_t target = static_cast<uint32_t>(p.zdirect ? p.G : p.T);
+      bool okw = true;
+      if (a == 0) {
+        okw = spin_until_geq(p.z_ready, target, ctl);
+        __syncwarp();
+        if (lane == 0 && okw) {
           const uint32_t old = atomicAdd(p.z_seen, 1u);
           if (old == static_cast<uint32_t>(p.G - 1)) {
             atomicExch(p.z_ready, 0u);
             atomicExch(p.z_seen, 0u);
           }
         }
+        __syncwarp();
       }
-      named_barrier(kBarAlu, kAluThreads);
-      ok = *alu_ok != 0;
-      named_barrier(kBarAlu, kAluThreads);
+      const bool any_fail = named_barrier_or(kBarAlu, kAluThreads, !okw);
+      if (any_fail) fail(ctl);
+      ok = !any_fail;
     }
 
-    // U side, one (segment, pass) at a time, handed to the epilogue through corr_s
-    const int IBn = (p.r + kRB - 1) / kRB;
-    int corr_round = 0;
-    for (int seg = 0; seg < nseg && ok; ++seg) {
-      const int t = t_first + seg;
-      const int ua = max(u0, t * p.KC) - t * p.KC, ub = min(u1, (t + 1) * p.KC) - t * p.KC;
-      const int b_lo = static_cast<int>(static_cast<long long>(IBn) * ua / p.KC);
-      const int b_hi = static_cast<int>(static_cast<long long>(IBn) * ub / p.KC);
-      for (int pass = 0; pass < npass; ++pass) {
-        const int m0 = pass * kMP, mcnt = min(kMP, p.M - m0);
-        if (corr_round > 0 &&
-            !group_wait(corre_bar, (corr_round - 1) & 1, tid == 0, kBarAlu, kAluThreads, alu_ok, ctl)) {
-          ok = false;
-          break;
+    if (p.r > 0) {
+      // ---- U side, one (segment, pass) at a time, handed to the epilogue via corr_s
+      int corr_round = 0;
+      for (int seg = 0; seg < nseg && ok; ++seg) {
+        const int t = t_first + seg;
+        int b_lo, b_hi;
+        rank_share(p, max(u0, t * p.KC) - t * p.KC, min(u1, (t + 1) * p.KC) - t * p.KC, b_lo, b_hi);
+        for (int pass = 0; pass < npass; ++pass) {
+          const int m0 = pass * kMP, mcnt = min(kMP, p.M - m0);
+          if (corr_round > 0 &&
+              !group_wait(corre_bar, (corr_round - 1) & 1, kBarAlu, kAluThreads, ctl)) {
+            ok = false;
+            break;
+          }
+          uside_dispatch(p, t, b_lo, b_hi, m0, mcnt, B, a, lane, tid);
+          mbar_arrive(corrf_bar);
+          ++corr_round;
         }
-        uside_dispatch(p, t, b_lo, b_hi, m0, mcnt, z_s, zb_s, corr_s, x_s, v_s, red_s, vout, a, lane, tid);
-        mbar_arrive(corrf_bar);
-        ++corr_round;
       }
+      if (ok && corr_round > 0) group_wait(corre_bar, (corr_round - 1) & 1, kBarAlu, kAluThreads, ctl);
     }
-    if (ok && corr_round > 0)
-      group_wait(corre_bar, (corr_round - 1) & 1, tid == 0, kBarAlu, kAluThreads, alu_ok, ctl);
   }
 
   // ------------------------------------------------------------------ teardown
@@ -917,9 +1279,23 @@ bool make_tmap(CUtensorMap* m, const void* base, uint64_t inner_bytes, uint64_t 
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2-D tensor without swizzle: [rows][inner elements of elem_bytes], box [box_rows][box_inner].
+bool make_tmap_plain(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint32_t elem_bytes,
+                     uint64_t inner, uint64_t rows, uint32_t box_inner, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {inner, rows};
+  const cuuint64_t strides[1] = {inner * elem_bytes};
+  const cuuint32_t box[2] = {box_inner, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int BN, int ST>
-cudaError_t launch_fused(const CUtensorMap& tw, const CUtensorMap& tx, const FusedParams& fp,
-                         cudaStream_t s) {
+cudaError_t launch_fused(const CUtensorMap& tw, const CUtensorMap& tx, const CUtensorMap& txs,
+                         const CUtensorMap& tv, const FusedParams& fp, cudaStream_t s, bool pdl) {
   using L = Layout<BN, ST>;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
@@ -937,8 +1313,8 @@ cudaError_t launch_fused(const CUtensorMap& tw, const CUtensorMap& tx, const Fus
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, fused_kernel<BN, ST>, tw, tx, fp);
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, fused_kernel<BN, ST>, tw, tx, txs, tv, fp);
 }
 
 int pick_bn(int M) {
@@ -956,6 +1332,8 @@ int resolve_mode(int M, int N, int K, int r, int requested) {
   return BILOCO_MODE_SHARED_Z;
 }
 
+int gemm_kernel_count_for(int M) { return M <= kInKernelQuantMaxM ? 1 : 2; }
+
 int run_gemm(const GemmArgs& a, cudaStream_t s) {
   const int M = a.M, N = a.N, K = a.K, r = a.r;
   const int KC = (K + kUnitK - 1) / kUnitK;
@@ -963,31 +1341,51 @@ int run_gemm(const GemmArgs& a, cudaStream_t s) {
   const int U = T * KC;
   const int G = std::min(num_sms(), U);
   const int KW = K / 32;
-  const int IB = (r + kRB - 1) / kRB;
-  const int KB = (IB > 0) ? std::max(1, std::min(KW, G / IB)) : 1;
-  const int rpad = std::max(IB, 1) * kRB;
+  const int rpad = std::max((r + kRB - 1) / kRB, 1) * kRB;
   const int BN = pick_bn(M);
+  const bool inq = M <= kInKernelQuantMaxM;
+  const bool zdirect = (M <= 2) || (M * KC <= 64);
+  const bool shared_z = r > 0 && a.mode == BILOCO_MODE_SHARED_Z;
+  const bool unit_alu = inq || shared_z;
+  const int ranks_per_tile = (r + T - 1) / T;
+  const bool fast = unit_alu && BN <= 32 && K % 128 == 0 && (!shared_z || ranks_per_tile <= kVStageRanks);
 
   ScratchNeed need;
-  need.act_fp4 = static_cast<size_t>(M) * K / 2;
-  need.act_sf = static_cast<size_t>(KC) * kSfBytes;
-  need.xsum32 = static_cast<size_t>(M) * KW * 4;
-  need.zpart = static_cast<size_t>(std::max(KB * IB, 1)) * M * kRB * 4;
-  need.zfin = static_cast<size_t>(M) * rpad * 4;
-  need.zbsum = static_cast<size_t>(std::max(IB, 1)) * M * 4;
+  need.act_fp4 = inq ? 16 : static_cast<size_t>(M) * K / 2;
+  need.act_sf = inq ? 16 : static_cast<size_t>(KC) * kSfBytes;
+  need.zpart = r ? static_cast<size_t>(KC) * M * rpad * 4 : 16;
+  need.zfin = r ? static_cast<size_t>(M) * rpad * 4 : 16;
   need.slots = static_cast<size_t>(2 * G) * BN * kTileRows * 4;
-  need.counter_words = static_cast<size_t>(std::max(IB, 1)) + 2 + T;
+  need.counter_words = 2 + 2 * static_cast<size_t>(T);
   Scratch* sc = get_scratch(s, need);
   if (!sc) return BILOCO_ERR_NOMEM;
 
-  cudaError_t e = launch_prep_act(a.x, M, K, sc->act_fp4, sc->act_sf, sc->xsum32, s);
-  if (e != cudaSuccess) return BILOCO_ERR_CUDA;
+  cudaError_t e = cudaSuccess;
+  if (!inq) {
+    e = launch_prep_act(a.x, M, K, sc->act_fp4, sc->act_sf, s);
+    if (e != cudaSuccess) return BILOCO_ERR_CUDA;
+  }
 
-  CUtensorMap tw, tx;
+  CUtensorMap tw, tx, txs, tv;
   if (!make_tmap(&tw, a.W_fp4, static_cast<uint64_t>(K) / 2, static_cast<uint64_t>(N), kTileRows))
     return BILOCO_ERR_CUDA;
-  if (!make_tmap(&tx, sc->act_fp4, static_cast<uint64_t>(K) / 2, static_cast<uint64_t>(M), BN))
+  if (inq) {
+    tx = tw;                                           // not read when quantising in-kernel
+  } else if (!make_tmap(&tx, sc->act_fp4, static_cast<uint64_t>(K) / 2, static_cast<uint64_t>(M), BN)) {
     return BILOCO_ERR_CUDA;
+  }
+  const int bxr = BN <= 16 ? 16 : 32;
+  txs = tw;
+  tv = tw;
+  if (fast) {
+    if (!make_tmap_plain(&txs, a.x, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, static_cast<uint64_t>(K),
+                         static_cast<uint64_t>(M), kSubK, static_cast<uint32_t>(bxr)))
+      return BILOCO_ERR_CUDA;
+    if (shared_z && !make_tmap_plain(&tv, a.Vbits, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4,
+                                     static_cast<uint64_t>(KW), static_cast<uint64_t>(r), kXWords,
+                                     kVStageRanks))
+      return BILOCO_ERR_CUDA;
+  }
 
   FusedParams fp = {};
   fp.w_sf = a.W_sf;
@@ -997,28 +1395,32 @@ int run_gemm(const GemmArgs& a, cudaStream_t s) {
   fp.Vbits = a.Vbits;
   fp.alpha = a.alpha;
   fp.x = a.x;
-  fp.xsum32 = sc->xsum32;
   fp.y = a.y;
   fp.zpart = sc->zpart;
   fp.zfin = sc->zfin;
-  fp.zbsum = sc->zbsum;
   fp.slots = sc->slots;
-  fp.rb_count = sc->counters;
-  fp.z_ready = sc->counters + std::max(IB, 1);
-  fp.z_seen = fp.z_ready + 1;
-  fp.tickets = fp.z_seen + 1;
+  fp.z_ready = sc->counters;
+  fp.z_seen = sc->counters + 1;
+  fp.tickets = sc->counters + 2;
+  fp.vtick = sc->counters + 2 + T;
   fp.status = sc->status;
   fp.M = M; fp.N = N; fp.K = K; fp.r = r;
-  fp.KC = KC; fp.T = T; fp.U = U; fp.G = G; fp.KW = KW; fp.KB = KB; fp.IB = IB;
+  fp.KC = KC; fp.T = T; fp.U = U; fp.G = G; fp.KW = KW;
   fp.rpad = rpad;
   fp.RW = (r + 31) / 32;
   fp.mode = a.mode;
+  fp.inq = inq ? 1 : 0;
+  fp.zdirect = zdirect ? 1 : 0;
+  fp.fast = fast ? 1 : 0;
+  fp.unit_alu = unit_alu ? 1 : 0;
+  fp.bxr = bxr;
 
+  const bool pdl = !inq;
   switch (BN) {
-    case 16: e = launch_fused<16, 6>(tw, tx, fp, s); break;
-    case 32: e = launch_fused<32, 5>(tw, tx, fp, s); break;
-    case 64: e = launch_fused<64, 4>(tw, tx, fp, s); break;
-    default: e = launch_fused<128, 3>(tw, tx, fp, s); break;
+    case 16: e = launch_fused<16, 5>(tw, tx, txs, tv, fp, s, pdl); break;
+    case 32: e = launch_fused<32, 3>(tw, tx, txs, tv, fp, s, pdl); break;
+    case 64: e = launch_fused<64, 4>(tw, tx, txs, tv, fp, s, pdl); break;
+    default: e = launch_fused<128, 3>(tw, tx, txs, tv, fp, s, pdl); break;
   }
   return e == cudaSuccess ? BILOCO_OK : BILOCO_ERR_CUDA;
 }

@@ -20,15 +20,13 @@ struct Scratch {
   size_t counter_words = 0;
   uint8_t* act_fp4 = nullptr;       // [M][K/2]
   uint8_t* act_sf = nullptr;        // KC * 2048 scale atoms
-  float* xsum32 = nullptr;          // [M][K/32]
-  float* zpart = nullptr;           // [KB][IB][M][16]
-  float* zfin = nullptr;            // [M][rpad]
-  float* zbsum = nullptr;           // [IB][M]
-  float* slots = nullptr;           // [2 G][BN][128]
+  float* zpart = nullptr;           // [KC][M][rpad] z partial sums per 256-element chunk
+  float* zfin = nullptr;            // [M][rpad] finished z
+  float* slots = nullptr;           // [2 G][BN][128] split-K partials
 };
 
 struct ScratchNeed {
-  size_t act_fp4, act_sf, xsum32, zpart, zfin, zbsum, slots, counter_words;
+  size_t act_fp4, act_sf, zpart, zfin, slots, counter_words;
 };
 
 // Returns nullptr on allocation failure.
@@ -40,7 +38,7 @@ int num_sms();
 cudaError_t launch_quant_act_rowmajor(const uint16_t* x, int M, int K, uint8_t* codes, uint8_t* sf,
                                       cudaStream_t s);
 cudaError_t launch_prep_act(const uint16_t* x, int M, int K, uint8_t* codes, uint8_t* sf_atoms,
-                            float* xsum32, cudaStream_t s);
+                            cudaStream_t s);
 cudaError_t launch_pack_weight(const float* R, int N, int K, uint8_t* W_fp4, uint8_t* W_sf,
                                float* gscale, cudaStream_t s);
 cudaError_t launch_pack_signs(const float* S, int rows, int cols, uint32_t* bits, cudaStream_t s);
@@ -61,5 +59,6 @@ struct GemmArgs {
 // Validated arguments; launches prep + fused kernels.  Returns a BILOCO_* status.
 int run_gemm(const GemmArgs& a, cudaStream_t s);
 int resolve_mode(int M, int N, int K, int r, int requested);
+int gemm_kernel_count_for(int M);
 
 }  // namespace biloco

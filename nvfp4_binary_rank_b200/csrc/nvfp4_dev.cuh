@@ -54,6 +54,31 @@ __device__ __forceinline__ uint2 encode_block16(const float (&v)[16], float S) {
 
 __device__ __forceinline__ float bf16_bits_to_f32(uint32_t h) { return __uint_as_float(h << 16); }
 
+__device__ __forceinline__ float amax16(const float (&v)[16]) {
+  float a = 0.0f;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) a = fmaxf(a, fabsf(v[j]));
+  return a;
+}
+
+// Activation block (no tensor scale): s = E4M3(amax / 6), codes = E2M1(x / s).
+__device__ __forceinline__ uint32_t quant_act_block(const float (&v)[16], uint2& codes) {
+  const float t = __fdiv_rn(amax16(v), 6.0f);
+  const uint32_t s = e4m3_from_f32(t);
+  codes = encode_block16(v, e4m3_to_f32(s));
+  return s;
+}
+
+// 16 BF16 values from 32 bytes (16-byte aligned) of shared or global memory.
+__device__ __forceinline__ void bf16x16_to_f32(const uint4& a, const uint4& b, float (&v)[16]) {
+  const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    v[2 * j] = bf16_bits_to_f32(w[j] & 0xFFFFu);
+    v[2 * j + 1] = bf16_bits_to_f32(w[j] >> 16);
+  }
+}
+
 // Byte offset of the scale of row `row` (< 128 within its 128-row tile) and
 // 16-element block `blk` (block index within the row) inside a run of 512-byte
 // scale atoms: one atom per 64 elements of K, 4 atoms per 256-element chunk.

@@ -20,28 +20,7 @@ constexpr int kQuantThreads = 256;
 __device__ __forceinline__ void load_bf16_block(const uint16_t* x, int K, int m, int blk,
                                                 float (&v)[16]) {
   const uint4* p = reinterpret_cast<const uint4*>(x + static_cast<size_t>(m) * K + blk * 16);
-  const uint4 a = __ldg(p), b = __ldg(p + 1);
-  const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    v[2 * j] = bf16_bits_to_f32(w[j] & 0xFFFFu);
-    v[2 * j + 1] = bf16_bits_to_f32(w[j] >> 16);
-  }
-}
-
-__device__ __forceinline__ float amax16(const float (&v)[16]) {
-  float a = 0.0f;
-#pragma unroll
-  for (int j = 0; j < 16; ++j) a = fmaxf(a, fabsf(v[j]));
-  return a;
-}
-
-// Activation block: s = E4M3(amax/6), codes = E2M1(x/s).
-__device__ __forceinline__ uint32_t quant_act_block(const float (&v)[16], uint2& codes) {
-  const float t = __fdiv_rn(amax16(v), 6.0f);
-  const uint32_t s = e4m3_from_f32(t);
-  codes = encode_block16(v, e4m3_to_f32(s));
-  return s;
+  bf16x16_to_f32(__ldg(p), __ldg(p + 1), v);
 }
 
 __global__ void __launch_bounds__(kQuantThreads)
@@ -59,34 +38,22 @@ quant_act_rowmajor_kernel(const uint16_t* __restrict__ x, int M, int K, uint8_t*
   sf[static_cast<size_t>(m) * nb + b] = static_cast<uint8_t>(s);
 }
 
-// Same quantiser, scales written into the GEMM's scale atoms, plus the FP32 sum
-// of every 32-element word of x (used by the sign correction).  Triggers the
+// Same quantiser, scales written into the GEMM's scale atoms.  Triggers the
 // dependent fused kernel at entry so that its prologue and weight stream overlap.
 __global__ void __launch_bounds__(kQuantThreads)
 prep_act_kernel(const uint16_t* __restrict__ x, int M, int K, uint8_t* __restrict__ codes,
-                uint8_t* __restrict__ sf_atoms, float* __restrict__ xsum32) {
+                uint8_t* __restrict__ sf_atoms) {
   griddep_launch_dependents();
   const int nb = K / 16;
   const long long id = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const bool live = id < static_cast<long long>(M) * nb;
-  int m = 0, b = 0;
-  float sum = 0.0f;
-  if (live) {
-    m = static_cast<int>(id / nb);
-    b = static_cast<int>(id % nb);
-    float v[16];
-    load_bf16_block(x, K, m, b, v);
-#pragma unroll
-    for (int j = 0; j < 16; ++j) sum += v[j];
-    uint2 c;
-    const uint32_t s = quant_act_block(v, c);
-    *reinterpret_cast<uint2*>(codes + static_cast<size_t>(m) * (K / 2) + b * 8) = c;
-    sf_atoms[sf_atom_offset(static_cast<uint32_t>(m), static_cast<uint32_t>(b))] =
-        static_cast<uint8_t>(s);
-  }
-  // blocks 2j and 2j+1 of a row sit in adjacent lanes (nb is even): pair them
-  const float other = __shfl_xor_sync(0xffffffffu, sum, 1);
-  if (live && (b & 1) == 0) xsum32[static_cast<size_t>(m) * (K / 32) + b / 2] = sum + other;
+  if (id >= static_cast<long long>(M) * nb) return;
+  const int m = static_cast<int>(id / nb), b = static_cast<int>(id % nb);
+  float v[16];
+  load_bf16_block(x, K, m, b, v);
+  uint2 c;
+  const uint32_t s = quant_act_block(v, c);
+  *reinterpret_cast<uint2*>(codes + static_cast<size_t>(m) * (K / 2) + b * 8) = c;
+  sf_atoms[sf_atom_offset(static_cast<uint32_t>(m), static_cast<uint32_t>(b))] = static_cast<uint8_t>(s);
 }
 
 // ---- weight packer: amax(|R|) -> g -> codes and tile-layout scales
@@ -169,9 +136,9 @@ cudaError_t launch_quant_act_rowmajor(const uint16_t* x, int M, int K, uint8_t* 
 }
 
 cudaError_t launch_prep_act(const uint16_t* x, int M, int K, uint8_t* codes, uint8_t* sf_atoms,
-                            float* xsum32, cudaStream_t s) {
+                            cudaStream_t s) {
   const long long n = static_cast<long long>(M) * (K / 16);
-  prep_act_kernel<<<grid_for(n), kQuantThreads, 0, s>>>(x, M, K, codes, sf_atoms, xsum32);
+  prep_act_kernel<<<grid_for(n), kQuantThreads, 0, s>>>(x, M, K, codes, sf_atoms);
   return cudaGetLastError();
 }
 
