@@ -64,9 +64,13 @@ enum {
   BILOCO_ERR_DEVICE = -7   /* the current device is not an sm_100 GPU             */
 };
 
-/* Size limits of biloco_gemm. */
+/* Size limits of biloco_gemm.  The weight is cut into (N/128) * ceil(K/256) units
+ * of 128 rows x 256 elements; at most BILOCO_MAX_UNITS of them (16.7 M units is
+ * 275 GB of codes, more than any single GPU holds). */
 #define BILOCO_MAX_M 128
 #define BILOCO_MAX_R 1024
+#define BILOCO_MAX_N (1 << 24)
+#define BILOCO_MAX_UNITS (1 << 24)
 
 /* z schedules of biloco_gemm (BiLoCo README, section "Kernel", mode table):
  *   BILOCO_MODE_AUTO       pick per (M, r, K) from a measured table
@@ -141,7 +145,8 @@ size_t biloco_weight_sf_bytes(int N, int K);
  *   Vbits   [r][K/32] uint32 = pack_signs(V^T)           (may be NULL when r == 0)
  *   alpha   [r] float                                    (may be NULL when r == 0)
  *   y_bf16  out [M][N] bfloat16, rounded to nearest-even from FP32
- *   limits  1 <= M <= 128, N % 128 == 0, K % 64 == 0, 0 <= r <= 1024
+ *   limits  1 <= M <= 128, N % 128 == 0, N <= 2^24, K % 64 == 0, 0 <= r <= 1024,
+ *           (N/128) * ceil(K/256) <= 2^24
  * Accumulation is FP32 in an unspecified order; results are deterministic for a
  * fixed shape, mode and GPU.  For M <= 8 one kernel is launched (it quantises
  * the activation itself); for larger M an activation quantiser runs first and

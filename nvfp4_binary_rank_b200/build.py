@@ -3,29 +3,32 @@
     python -m nvfp4_binary_rank_b200.build          # incremental
     python -m nvfp4_binary_rank_b200.build --force  # rebuild
 
-The library links the CUDA runtime dynamically so that, inside a process that
+Every .cu file under csrc/ is compiled to an object in parallel (the fused
+kernel instances live in separate files for that reason), then linked.  The
+library links the CUDA runtime dynamically so that, inside a process that
 already imported PyTorch, it shares PyTorch's runtime (one current device, one
 context).  Nothing here needs a GPU.
 """
 
 from __future__ import annotations
 
+import glob
 import os
 import shutil
 import subprocess
 import sys
+from concurrent.futures import ThreadPoolExecutor
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libbiloco.so")
-SOURCES = ["api.cu", "quant.cu", "gemm.cu"]
-HEADERS = ["ptx.cuh", "nvfp4_dev.cuh", "internal.h"]
+OBJ = os.path.join(PKG, "_build")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
-FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-cudart", "shared",
-         "--expt-relaxed-constexpr", "-I", INCLUDE]
+FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
+         "-I", INCLUDE]
 
 
 def nvcc() -> str:
@@ -35,30 +38,53 @@ def nvcc() -> str:
     raise RuntimeError("nvcc not found")
 
 
-def _stale() -> bool:
-    if not os.path.exists(LIB):
-        return True
-    t = os.path.getmtime(LIB)
-    deps = [os.path.join(CSRC, f) for f in SOURCES + HEADERS] + [os.path.join(INCLUDE, "biloco.h")]
-    return any(os.path.getmtime(d) > t for d in deps)
+def sources():
+    return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
+
+
+def _headers():
+    return (glob.glob(os.path.join(CSRC, "*.h")) + glob.glob(os.path.join(CSRC, "*.cuh"))
+            + [os.path.join(INCLUDE, "biloco.h")])
+
+
+def _obj_of(src):
+    return os.path.join(OBJ, os.path.basename(src)[:-3] + ".o")
+
+
+def _compile(src, force, verbose):
+    obj = _obj_of(src)
+    newest_dep = max(os.path.getmtime(p) for p in _headers() + [src])
+    if not force and os.path.exists(obj) and os.path.getmtime(obj) >= newest_dep:
+        return obj
+    cmd = [nvcc(), *ARCH, *FLAGS, "-c", src, "-o", obj + ".tmp"]
+    if verbose:
+        print(" ".join(cmd), flush=True)
+    res = subprocess.run(cmd, capture_output=True, text=True)
+    if res.returncode != 0:
+        sys.stderr.write(res.stdout + res.stderr)
+        raise RuntimeError(f"nvcc failed on {os.path.basename(src)}")
+    os.replace(obj + ".tmp", obj)
+    return obj
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and not _stale():
+    os.makedirs(OBJ, exist_ok=True)
+    srcs = sources()
+    with ThreadPoolExecutor(max_workers=max(1, min(len(srcs), os.cpu_count() or 1))) as ex:
+        objs = list(ex.map(lambda s: _compile(s, force, verbose), srcs))
+    if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= max(os.path.getmtime(o) for o in objs):
         return LIB
-    tmp = LIB + ".tmp"
-    cmd = [nvcc(), *ARCH, *FLAGS, "-shared", "-o", tmp,
-           *[os.path.join(CSRC, f) for f in SOURCES],
+    cmd = [nvcc(), *ARCH, "-shared", "-cudart", "shared", "-o", LIB + ".tmp", *objs,
            "-Xlinker", "-rpath,/usr/local/cuda/lib64"]
     if verbose:
         print(" ".join(cmd), flush=True)
     res = subprocess.run(cmd, capture_output=True, text=True)
     if res.returncode != 0:
         sys.stderr.write(res.stdout + res.stderr)
-        raise RuntimeError("nvcc failed building libbiloco.so")
-    os.replace(tmp, LIB)
+        raise RuntimeError("nvcc failed linking libbiloco.so")
+    os.replace(LIB + ".tmp", LIB)
     return LIB
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose=True))
+    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))

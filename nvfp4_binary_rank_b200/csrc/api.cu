@@ -200,7 +200,8 @@ int biloco_gemm(const void* x_bf16, const uint8_t* W_fp4, const uint8_t* W_sf, c
   if (!x_bf16 || !W_fp4 || !W_sf || !gscale || !y_bf16) return BILOCO_ERR_ARG;
   if (r > 0 && (!Ubits || !Vbits || !alpha)) return BILOCO_ERR_ARG;
   if (M < 1 || M > BILOCO_MAX_M || N < 128 || N % 128 || K < 64 || K % 64 || r < 0 ||
-      r > BILOCO_MAX_R)
+      r > BILOCO_MAX_R || N > BILOCO_MAX_N ||
+      static_cast<long long>(N / 128) * ((K + 255) / 256) > BILOCO_MAX_UNITS)
     return BILOCO_ERR_SHAPE;
   if (!aligned16(x_bf16) || !aligned16(W_fp4) || !aligned16(W_sf) || !aligned16(y_bf16) ||
       (reinterpret_cast<uintptr_t>(gscale) & 3u) || (r > 0 && (!aligned16(Ubits) || !aligned16(Vbits) ||

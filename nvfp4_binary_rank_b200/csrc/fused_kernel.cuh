@@ -47,18 +47,16 @@
 // Every wait (mbarrier or global counter) is bounded; on expiry the kernel records
 // BILOCO_ERR_TIMEOUT in the stream's status word, drains its own copies and MMAs,
 // frees its TMEM and returns.
+#pragma once
+
 #include <cstdint>
-#include <cstdio>
-#include <cstring>
-#include <mutex>
 
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include "../../include/biloco.h"
-
-#include "internal.h"
+#include "fused_params.h"
 #include "nvfp4_dev.cuh"
 #include "ptx.cuh"
 
@@ -92,32 +90,7 @@ constexpr int kInKernelQuantMaxM = 8;
 constexpr int kBarAlu = 1;                 // named barrier ids (0 is __syncthreads)
 constexpr int kBarEpi = 2;
 
-struct FusedParams {
-  const uint8_t* w_sf;
-  const uint8_t* x_sf;
-  const float* gscale;
-  const uint32_t* Ubits;
-  const uint32_t* Vbits;
-  const float* alpha;
-  const uint16_t* x;
-  uint16_t* y;
-  float* zpart;        // [KC][M][rpad]
-  float* zfin;         // [M][rpad]
-  float* slots;        // [2 G][BN][128]
-  uint32_t* z_ready;
-  uint32_t* z_seen;
-  uint32_t* tickets;   // [T] split-K tickets
-  uint32_t* vtick;     // [T] V-side finaliser tickets
-  int* status;
-  int M, N, K, r;
-  int KC, T, U, G, KW, rpad, RW;
-  int mode;            // BILOCO_MODE_SHARED_Z or BILOCO_MODE_LOCAL_Z
-  int inq;             // 1: activation quantised in-kernel (no pre-pass)
-  int zdirect;         // 1: consumers sum the chunk partials themselves
-  int fast;            // 1: the producer stages each unit's x chunk and V rows by TMA
-  int unit_alu;        // 1: the CUDA-core warps have per-unit work (quantise and/or V side)
-  int bxr;             // rows of the staged x box (16 or 32)
-};
+
 
 template <int BN, int ST>
 struct Layout {
@@ -141,12 +114,12 @@ struct Layout {
   static constexpr int kZS = kXS + kXSRegion;                        // z chunk [128][kMpad]
   static constexpr int kZB = kZS + kZChunkBlocks * kRB * kMpad * 4;  // z block sums [8][32]
   static constexpr int kCorr = kZB + kZChunkBlocks * kMP * 4;        // corr [2][32][128]
-  static constexpr int kRed = kCorr + 2 * kMP * kTileRows * 4;       // task partials [8][64]
-  static constexpr int kVOut = kRed + kAluWarps * 64 * 4;            // V-side result [32][32]
+  static constexpr int kRed = kCorr + 2 * kMP * kTileRows * 4;       // task partials [8][256]
+  static constexpr int kVOut = kRed + kAluWarps * 256 * 4;           // V-side result [32][32]
   static constexpr int kXsw = kVOut + kMP * kVRanks * 4;             // x sums per warp [8][32]
   static constexpr int kXsum = kXsw + kAluWarps * kMP * 4;           // x sums [32]
   static constexpr int kBar = kXsum + kMP * 4;
-  static constexpr int kNumBars = 3 * ST + 7;
+  static constexpr int kNumBars = 3 * ST + 8;
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kTotal = kMisc + 64;
   static constexpr int kAlloc = kTotal + 1024;
@@ -157,11 +130,13 @@ struct Layout {
 
 // ------------------------------------------------------------------ small helpers
 
-__device__ __forceinline__ int owner_cta(long long u, int G, int U) {
-  return static_cast<int>(((u + 1) * G - 1) / U);
+// Stream-K bookkeeping in 32-bit unsigned arithmetic: the host limits T * KC to
+// 2^24 units and G to the SM count, so every product stays below 2^32.
+__device__ __forceinline__ int owner_cta(uint32_t u, int G, int U) {
+  return static_cast<int>(((u + 1u) * static_cast<uint32_t>(G) - 1u) / static_cast<uint32_t>(U));
 }
 __device__ __forceinline__ int first_unit(int h, int G, int U) {
-  return static_cast<int>(static_cast<long long>(h) * U / G);
+  return static_cast<int>(static_cast<uint32_t>(h) * static_cast<uint32_t>(U) / static_cast<uint32_t>(G));
 }
 
 // Predicated packed add: acc += (a, b) when flag != 0.
@@ -242,7 +217,10 @@ __device__ __forceinline__ bool spin_until_geq(const uint32_t* p, uint32_t targe
 // then agrees (barrier + OR) on whether anyone gave up, so all leave together.
 __device__ __forceinline__ bool group_wait(uint32_t bar, uint32_t parity, int bar_id, int nthreads,
                                            const Ctl& c) {
-  const bool ok = mbar_wait(bar, parity, c.abort_flag);
+  // one lane per warp polls (the others would only load the shared-memory pipe)
+  bool ok = true;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, c.abort_flag);
+  ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
   const bool any_fail = named_barrier_or(bar_id, nthreads, !ok);
   if (any_fail) fail(c);
   return !any_fail;
@@ -250,16 +228,16 @@ __device__ __forceinline__ bool group_wait(uint32_t bar, uint32_t parity, int ba
 
 // Tile t's slice of the ranks on the V side: [t r / T, (t + 1) r / T).
 __device__ __forceinline__ void vside_ranks(const FusedParams& p, int t, int& i_lo, int& i_hi) {
-  i_lo = static_cast<int>(static_cast<long long>(t) * p.r / p.T);
-  i_hi = static_cast<int>(static_cast<long long>(t + 1) * p.r / p.T);
+  i_lo = static_cast<int>(static_cast<uint32_t>(t) * static_cast<uint32_t>(p.r) / static_cast<uint32_t>(p.T));
+  i_hi = static_cast<int>(static_cast<uint32_t>(t + 1) * static_cast<uint32_t>(p.r) / static_cast<uint32_t>(p.T));
 }
 
 // U-side rank blocks of tile t handled by the segment covering units [ua, ub)
 // of the tile (offsets within the tile): proportional to its share of K.
 __device__ __forceinline__ void rank_share(const FusedParams& p, int ua, int ub, int& b_lo, int& b_hi) {
   const int IBn = (p.r + kRB - 1) / kRB;
-  b_lo = static_cast<int>(static_cast<long long>(IBn) * ua / p.KC);
-  b_hi = static_cast<int>(static_cast<long long>(IBn) * ub / p.KC);
+  b_lo = static_cast<int>(static_cast<uint32_t>(IBn) * static_cast<uint32_t>(ua) / static_cast<uint32_t>(p.KC));
+  b_hi = static_cast<int>(static_cast<uint32_t>(IBn) * static_cast<uint32_t>(ub) / static_cast<uint32_t>(p.KC));
 }
 
 // ------------------------------------------------------------------ staging
@@ -343,7 +321,7 @@ __device__ __forceinline__ void vside_task_finish(uint64_t (&acc2)[8][(MG >= 2) 
 // out[m * kVRanks + i] = sum over the staged words [0, nw) of the x[m][k] whose
 // sign V[k][i] is -1, for m < mcnt (<= 32), i < nr (<= 64).  Whole group.
 template <int MG>
-__device__ void vside_chunk(const uint16_t* xb, const uint32_t* vb, int mcnt, int nr, int nw,
+__device__ __forceinline__ void vside_chunk(const uint16_t* xb, const uint32_t* vb, int mcnt, int nr, int nw,
                             float* red_s, float* out, int a, int lane, int tid) {
   constexpr int kPairs = (MG >= 2) ? MG / 2 : 1;
   const int mgc = (mcnt + MG - 1) / MG;
@@ -385,17 +363,10 @@ __device__ void vside_chunk(const uint16_t* xb, const uint32_t* vb, int mcnt, in
   }
 }
 
-__device__ void vside_chunk_dispatch(const uint16_t* xb, const uint32_t* vb, int mcnt, int nr, int nw,
-                                     float* red_s, float* out, int a, int lane, int tid) {
-  if (mcnt > 4) vside_chunk<8>(xb, vb, mcnt, nr, nw, red_s, out, a, lane, tid);
-  else if (mcnt > 2) vside_chunk<4>(xb, vb, mcnt, nr, nw, red_s, out, a, lane, tid);
-  else if (mcnt > 1) vside_chunk<2>(xb, vb, mcnt, nr, nw, red_s, out, a, lane, tid);
-  else vside_chunk<1>(xb, vb, mcnt, nr, nw, red_s, out, a, lane, tid);
-}
 
 // xs_s[m] = sum of the staged chunk row m (fixed order: lanes, then warps).
 template <int V>
-__device__ void chunk_xsum(const uint16_t* xb, int mcnt, int nw, float* xsw, float* xs_s, int a,
+__device__ __forceinline__ void chunk_xsum(const uint16_t* xb, int mcnt, int nw, float* xsw, float* xs_s, int a,
                            int lane, int tid) {
   float v[V];
   const bool in = tid < nw * 32;
@@ -414,15 +385,6 @@ __device__ void chunk_xsum(const uint16_t* xb, int mcnt, int nw, float* xsw, flo
   named_barrier(kBarAlu, kAluThreads);
 }
 
-__device__ void chunk_xsum_dispatch(const uint16_t* xb, int mcnt, int nw, float* xsw, float* xs_s,
-                                    int a, int lane, int tid) {
-  if (mcnt > 16) chunk_xsum<32>(xb, mcnt, nw, xsw, xs_s, a, lane, tid);
-  else if (mcnt > 8) chunk_xsum<16>(xb, mcnt, nw, xsw, xs_s, a, lane, tid);
-  else if (mcnt > 4) chunk_xsum<8>(xb, mcnt, nw, xsw, xs_s, a, lane, tid);
-  else if (mcnt > 2) chunk_xsum<4>(xb, mcnt, nw, xsw, xs_s, a, lane, tid);
-  else if (mcnt > 1) chunk_xsum<2>(xb, mcnt, nw, xsw, xs_s, a, lane, tid);
-  else chunk_xsum<1>(xb, mcnt, nw, xsw, xs_s, a, lane, tid);
-}
 
 // ------------------------------------------------------------------ activation quantisation
 
@@ -430,7 +392,7 @@ __device__ void chunk_xsum_dispatch(const uint16_t* xb, int mcnt, int nw, float*
 // 128-byte swizzle: 16-byte piece j of row m sits at piece j ^ (m & 7)) and the
 // chunk's 4 scale atoms.  Blocks past K keep whatever finite codes the stage held;
 // the weight codes there are zero-filled by TMA.
-__device__ void quant_chunk(const uint16_t* xb, int mcnt, int nw, uint8_t* btile, uint8_t* sfb, int tid) {
+__device__ __forceinline__ void quant_chunk(const uint16_t* xb, int mcnt, int nw, uint8_t* btile, uint8_t* sfb, int tid) {
   const int nblk = 2 * nw;
   for (int idx = tid; idx < mcnt * nblk; idx += kAluThreads) {
     const int m = idx / nblk, blk = idx % nblk;
@@ -445,12 +407,145 @@ __device__ void quant_chunk(const uint16_t* xb, int mcnt, int nw, uint8_t* btile
   }
 }
 
+// ------------------------------------------------------------------ batched V side
+
+// The V side of a batch of staged units as independent warp tasks: task =
+// (unit j, group of 8 ranks rg, group of MG batch rows mg), over the unit's whole
+// chunk.  Lane l takes bit l of every 32-element word; the task's 8*MG sums are
+// reduced over the lanes, its row sums of x over the whole warp, and the lanes
+// store zpart = sum_k x - 2 * sum_{sign -1} x directly.  No group barrier.
+template <int MG, typename UnitInfo>
+__device__ __forceinline__ void vside_batch(const FusedParams& p, int nb, int mcnt, int rgu, UnitInfo info,
+                                            float* xs_w, int a, int lane) {
+  constexpr int kPairs = (MG >= 2) ? MG / 2 : 1;
+  constexpr int kVals = 8 * MG;
+  const int mgc = (mcnt + MG - 1) / MG;
+  const int tasks = nb * rgu * mgc;
+  const uint32_t lane_bit = 1u << lane;
+  for (int task = a; task < tasks; task += kAluWarps) {
+    const int j = task / (rgu * mgc), rest = task % (rgu * mgc), rg = rest / mgc, mg = rest % mgc;
+    const uint16_t* xc;
+    const uint32_t* vrows;
+    int c, i_lo, nr, nw;
+    info(j, xc, vrows, c, i_lo, nr, nw);
+    if (rg * 8 >= nr) continue;                      // uniform over the warp
+    uint64_t acc2[8][kPairs];
+    float acc1[8];
+    float xacc[MG];
+#pragma unroll
+    for (int g = 0; g < 8; ++g) {
+      acc1[g] = 0.0f;
+#pragma unroll
+      for (int q = 0; q < kPairs; ++q) acc2[g][q] = 0ull;
+    }
+#pragma unroll
+    for (int mm = 0; mm < MG; ++mm) xacc[mm] = 0.0f;
+    const uint16_t* xs = xc + (mg * MG) * kSubK + lane;
+    const uint32_t* vs = vrows + (rg * 8) * kXWords;
+    for (int w = 0; w < nw; ++w) {
+      float xv[MG];
+#pragma unroll
+      for (int mm = 0; mm < MG; ++mm) {
+        xv[mm] = bf16_bits_to_f32(xs[mm * kSubK + w * 32]);
+        xacc[mm] += xv[mm];
+      }
+#pragma unroll
+      for (int g = 0; g < 8; ++g) {
+        const uint32_t flag = vs[g * kXWords + w] & lane_bit;
+        if constexpr (MG >= 2) {
+#pragma unroll
+          for (int q = 0; q < MG / 2; ++q) padd2(acc2[g][q], xv[2 * q], xv[2 * q + 1], flag);
+        } else {
+          padd1(acc1[g], xv[0], flag);
+        }
+      }
+    }
+    // row sums of x over the warp (every lane gets all MG of them)
+#pragma unroll
+    for (int mm = 0; mm < MG; ++mm) {
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) xacc[mm] += __shfl_xor_sync(0xffffffffu, xacc[mm], o);
+    }
+    if (lane == 0) {
+#pragma unroll
+      for (int mm = 0; mm < MG; ++mm) xs_w[a * kMP + mm] = xacc[mm];
+    }
+    float vals[kVals];
+#pragma unroll
+    for (int g = 0; g < 8; ++g) {
+      if constexpr (MG >= 2) {
+#pragma unroll
+        for (int q = 0; q < MG / 2; ++q) {
+          vals[g * MG + 2 * q] = lo_f(acc2[g][q]);
+          vals[g * MG + 2 * q + 1] = hi_f(acc2[g][q]);
+        }
+      } else {
+        vals[g] = acc1[g];
+      }
+    }
+    warp_reduce_scatter<kVals>(vals, lane);
+    __syncwarp();
+    constexpr int kOut = (kVals >= 32) ? kVals / 32 : 1;
+#pragma unroll
+    for (int jj = 0; jj < kOut; ++jj) {
+      const int e = reduce_out_index<kVals>(lane, jj);
+      const int g = e / MG, mm = e % MG;
+      const int m = mg * MG + mm, i = rg * 8 + g;
+      if (m < mcnt && i < nr)
+        p.zpart[(static_cast<size_t>(c) * p.M + m) * p.rpad + i_lo + i] = xs_w[a * kMP + mm] - 2.0f * vals[jj];
+    }
+    __syncwarp();
+  }
+}
+
+// ------------------------------------------------------------------ small-batch fast path
+
+// V side for M <= 8 with lanes over ranks: lane l < nrg takes rank g0 + l of the
+// staged rows, lane 31 sums x itself (an all-ones sign word), warp a takes word a
+// of the chunk.  out[m * 64 + i] = sum of the x whose sign is -1 (i < nr),
+// xs[m] = sum of x over the chunk.  Whole group.
+template <int MG>
+__device__ __forceinline__ void vside_lane_rank(const uint16_t* xc, const uint32_t* vrows, int mcnt, int nr,
+                                                int nw, float* part, float* out, float* xs, int a, int lane,
+                                                int tid) {
+  for (int g0 = 0; g0 < nr; g0 += 31) {
+    const int nrg = min(31, nr - g0);
+    float acc[MG];
+#pragma unroll
+    for (int mm = 0; mm < MG; ++mm) acc[mm] = 0.0f;
+    if (a < nw) {
+      const uint32_t word = (lane < nrg) ? vrows[(g0 + lane) * kXWords + a] : (lane == 31 ? 0xFFFFFFFFu : 0u);
+      const uint16_t* xr = xc + a * 32;
+#pragma unroll 8
+      for (int j = 0; j < 32; ++j) {
+        const uint32_t flag = word & (1u << j);
+#pragma unroll
+        for (int mm = 0; mm < MG; ++mm) padd1(acc[mm], bf16_bits_to_f32(xr[mm * kSubK + j]), flag);
+      }
+    }
+#pragma unroll
+    for (int mm = 0; mm < MG; ++mm) part[(a * 32 + lane) * MG + mm] = acc[mm];
+    named_barrier(kBarAlu, kAluThreads);
+    if (tid < 32 * MG) {
+      const int l = tid / MG, mm = tid % MG;
+      float sum = 0.0f;
+#pragma unroll
+      for (int w = 0; w < kAluWarps; ++w) sum += part[(w * 32 + l) * MG + mm];
+      if (mm < mcnt) {
+        if (l < nrg) out[mm * 64 + g0 + l] = sum;
+        else if (l == 31 && g0 == 0) xs[mm] = sum;
+      }
+    }
+    named_barrier(kBarAlu, kAluThreads);
+  }
+}
+
 // ------------------------------------------------------------------ local z (mode 2)
 
 // out[m * kVRanks + i] = sum over ALL of K of the x[m0+m][k] whose sign V[k][i0+i]
 // is -1 (i < nr <= 16), and xs_s[m] = sum_k x[m0+m][k].  Whole group.
 template <int MG>
-__device__ void vside_full_k(const FusedParams& p, int m0, int mcnt, int i0, int nr, uint16_t* xb,
+__device__ __forceinline__ void vside_full_k(const FusedParams& p, int m0, int mcnt, int i0, int nr, uint16_t* xb,
                              uint32_t* vb, float* red_s, float* xs_s, float* out, int a, int lane,
                              int tid) {
   constexpr int kPairs = (MG >= 2) ? MG / 2 : 1;
@@ -519,14 +614,6 @@ __device__ void vside_full_k(const FusedParams& p, int m0, int mcnt, int i0, int
   named_barrier(kBarAlu, kAluThreads);
 }
 
-__device__ void vside_full_k_dispatch(const FusedParams& p, int m0, int mcnt, int i0, int nr,
-                                      uint16_t* xb, uint32_t* vb, float* red_s, float* xs_s, float* out,
-                                      int a, int lane, int tid) {
-  if (mcnt > 4) vside_full_k<8>(p, m0, mcnt, i0, nr, xb, vb, red_s, xs_s, out, a, lane, tid);
-  else if (mcnt > 2) vside_full_k<4>(p, m0, mcnt, i0, nr, xb, vb, red_s, xs_s, out, a, lane, tid);
-  else if (mcnt > 1) vside_full_k<2>(p, m0, mcnt, i0, nr, xb, vb, red_s, xs_s, out, a, lane, tid);
-  else vside_full_k<1>(p, m0, mcnt, i0, nr, xb, vb, red_s, xs_s, out, a, lane, tid);
-}
 
 // ------------------------------------------------------------------ U side
 
@@ -545,8 +632,8 @@ struct AluBufs {
 // corr[rs][m][row] for the 128 rows of tile t, rows m0 .. m0+mcnt of the batch and
 // the ranks of rank blocks [b_lo, b_hi).  Task a: rows 32 (a & 3) + lane; (a >> 2)
 // picks the upper/lower 16 batch rows (mcnt > 16) or the rank-block parity (else).
-template <int MG>
-__device__ void uside_pass(const FusedParams& p, int t, int b_lo, int b_hi, int m0, int mcnt,
+template <int MG, int MGV>
+__device__ __forceinline__ void uside_pass(const FusedParams& p, int t, int b_lo, int b_hi, int m0, int mcnt,
                            const AluBufs& B, int a, int lane, int tid) {
   constexpr int kPairs = (MG >= 2) ? MG / 2 : 1;
   const int RS = (mcnt > 16) ? 1 : 2;
@@ -574,23 +661,42 @@ __device__ void uside_pass(const FusedParams& p, int t, int b_lo, int b_hi, int 
     named_barrier(kBarAlu, kAluThreads);            // previous chunk consumed
     if (p.mode == BILOCO_MODE_SHARED_Z) {
       const int nr = nblk * kRB;
-      for (int idx = tid; idx < nr * kMP; idx += kAluThreads) {
-        const int m = idx / nr, i = idx % nr;
-        const int rank = c0 * kRB + i;
-        float v = 0.0f;
-        if (m < mcnt && rank < p.r && c0 + i / kRB >= b_lo && c0 + i / kRB < b_hi) {
-          if (p.zdirect) {
-            float s = 0.0f;
-            const float* src = p.zpart + static_cast<size_t>(m0 + m) * p.rpad + rank;
-            const size_t stride = static_cast<size_t>(p.M) * p.rpad;
-#pragma unroll 4
-            for (int c = 0; c < p.KC; ++c) s += __ldcg(src + c * stride);
-            v = __fmul_rn(__ldg(p.alpha + rank), s);
-          } else {
-            v = __ldcg(p.zfin + static_cast<size_t>(m0 + m) * p.rpad + rank);
-          }
+      const int r_lo = max(c0, b_lo) * kRB, r_hi = min(min(c0 + nblk, b_hi) * kRB, p.r);
+      const int nv = max(0, r_hi - r_lo);                 // ranks of this chunk in the share
+      if (p.zdirect) {
+        // every chunk partial of every needed (m, rank), copied asynchronously in one
+        // round (mcnt * KC <= 64, nv <= 128), then summed in chunk order
+        float* zst = B.corr_s;
+        const int i = tid & 127;
+        if (i < nv) {
+          const size_t stride = static_cast<size_t>(p.M) * p.rpad;
+          const float* src = p.zpart + static_cast<size_t>(m0) * p.rpad + r_lo + i;
+          for (int cc = tid >> 7; cc < p.KC; cc += 2)
+            for (int m = 0; m < mcnt; ++m)
+              cp_async4(smem_u32(zst + (cc * mcnt + m) * nv + i), src + cc * stride + static_cast<size_t>(m) * p.rpad);
         }
-        B.z_s[i * kMpad + m] = v;
+        cp_async_commit();
+        cp_async_wait<0>();
+        named_barrier(kBarAlu, kAluThreads);
+        for (int m = tid >> 7; m < kMP; m += 2) {
+          const int rank = c0 * kRB + i;
+          float v = 0.0f;
+          if (i < nr && m < mcnt && rank >= r_lo && rank < r_hi) {
+            float sum = 0.0f;
+            for (int cc = 0; cc < p.KC; ++cc) sum += zst[(cc * mcnt + m) * nv + rank - r_lo];
+            v = __fmul_rn(__ldg(p.alpha + rank), sum);
+          }
+          if (i < nr) B.z_s[i * kMpad + m] = v;
+        }
+      } else {
+        const int i = tid & 127;
+        for (int m = tid >> 7; m < kMP; m += 2) {
+          const int rank = c0 * kRB + i;
+          float v = 0.0f;
+          if (i < nr && m < mcnt && rank >= r_lo && rank < r_hi)
+            v = __ldcg(p.zfin + static_cast<size_t>(m0 + m) * p.rpad + rank);
+          if (i < nr) B.z_s[i * kMpad + m] = v;
+        }
       }
     } else {
       // local z: each needed rank block over the whole K, computed right here
@@ -598,7 +704,7 @@ __device__ void uside_pass(const FusedParams& p, int t, int b_lo, int b_hi, int 
         const int blk = c0 + bl;
         if (blk < b_lo || blk >= b_hi) continue;      // uniform over the group
         const int i0 = blk * kRB, nr = min(kRB, p.r - i0);
-        vside_full_k_dispatch(p, m0, mcnt, i0, nr, B.xb, B.vb, B.red_s, B.xs_s, B.vout, a, lane, tid);
+        vside_full_k<MGV>(p, m0, mcnt, i0, nr, B.xb, B.vb, B.red_s, B.xs_s, B.vout, a, lane, tid);
         for (int idx = tid; idx < kMP * kRB; idx += kAluThreads) {
           const int m = idx / kRB, i = idx % kRB;
           float z = 0.0f;
@@ -664,17 +770,9 @@ __device__ void uside_pass(const FusedParams& p, int t, int b_lo, int b_hi, int 
   }
 }
 
-__device__ void uside_dispatch(const FusedParams& p, int t, int b_lo, int b_hi, int m0, int mcnt,
-                               const AluBufs& B, int a, int lane, int tid) {
-  if (mcnt > 8) uside_pass<16>(p, t, b_lo, b_hi, m0, mcnt, B, a, lane, tid);
-  else if (mcnt > 4) uside_pass<8>(p, t, b_lo, b_hi, m0, mcnt, B, a, lane, tid);
-  else if (mcnt > 2) uside_pass<4>(p, t, b_lo, b_hi, m0, mcnt, B, a, lane, tid);
-  else if (mcnt > 1) uside_pass<2>(p, t, b_lo, b_hi, m0, mcnt, B, a, lane, tid);
-  else uside_pass<1>(p, t, b_lo, b_hi, m0, mcnt, B, a, lane, tid);
-}
 
 // Warm L2 with the sign rows of U this CTA's U side will read.
-__device__ void prefetch_u_rows(const FusedParams& p, int u0, int u1, int tid) {
+__device__ __forceinline__ void prefetch_u_rows(const FusedParams& p, int u0, int u1, int tid) {
   const int t_first = u0 / p.KC, t_last = (u1 - 1) / p.KC;
   for (int t = t_first; t <= t_last && t < t_first + 2; ++t) {
     int b_lo, b_hi;
@@ -689,12 +787,15 @@ __device__ void prefetch_u_rows(const FusedParams& p, int u0, int u1, int tid) {
 
 // ------------------------------------------------------------------ the kernel
 
-template <int BN, int ST>
+template <int BN, int ST, int MC>
 __global__ void __launch_bounds__(kThreads, 1)
 fused_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
              const __grid_constant__ CUtensorMap tmap_xs, const __grid_constant__ CUtensorMap tmap_v,
              const __grid_constant__ FusedParams p) {
   using L = Layout<BN, ST>;
+  constexpr int MGV = (MC < 8) ? MC : 8;       // V side: batch rows per task
+  constexpr int MGU = (MC < 16) ? MC : 16;     // U side: batch rows per task
+  constexpr int XV = (MC < 32) ? MC : 32;      // x sums: rows per warp reduction
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -709,6 +810,7 @@ fused_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
   const uint32_t corre_bar = smem_u32(&bars[2 * ST + 5]);
   const uint32_t drain_bar = smem_u32(&bars[2 * ST + 6]);
   auto xfull_bar = [&](int s) { return smem_u32(&bars[2 * ST + 7 + s]); };
+  const uint32_t done_bar = smem_u32(&bars[3 * ST + 7]);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
   volatile int* epi_last = reinterpret_cast<volatile int*>(smem + L::kMisc + 16);
@@ -741,6 +843,7 @@ fused_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
     mbar_init(corrf_bar, kAluThreads);
     mbar_init(corre_bar, kEpiThreads);
     mbar_init(drain_bar, 1);
+    mbar_init(done_bar, kWarps);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -891,8 +994,8 @@ fused_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
     for (int seg = 0; seg < nseg; ++seg) {
       const int t = t_first + seg;
       const int b = seg & 1;
-      const int hf = owner_cta(static_cast<long long>(t) * p.KC, p.G, p.U);
-      const int hl = owner_cta(static_cast<long long>(t + 1) * p.KC - 1, p.G, p.U);
+      const int hf = owner_cta(static_cast<uint32_t>(t * p.KC), p.G, p.U);
+      const int hl = owner_cta(static_cast<uint32_t>((t + 1) * p.KC - 1), p.G, p.U);
       const bool sole = hf == hl;
       const int which = (t == t_first) ? 0 : 1;
       float* my_slot = p.slots + static_cast<size_t>(2 * g + which) * BN * kTileRows;
@@ -968,25 +1071,62 @@ fused_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
         const bool last = *epi_last != 0;
         named_barrier(kBarEpi, kEpiThreads);
         if (last) {
-#pragma unroll 2
-          for (int m = 0; m < p.M; ++m) {
-            float s = 0.0f;
-            for (int h0 = hf; h0 <= hl; h0 += 8) {
-              float part[8];
+          // this row's partials of every contributor in rounds of 32 independent
+          // loads, each batch row summed in contributor order
+          const int nh = hl - hf + 1;
+          // every contributor after the first starts its range inside tile t, so only
+          // the first one may hold this tile in its second slot
+          const int wh_first = (t == first_unit(hf, p.G, p.U) / p.KC) ? 0 : 1;
+          auto slot_of = [&](int h) { return 2 * h + ((h == hf) ? wh_first : 0); };
+          if (nh <= 32) {
+            const int rows_per_round = 32 / nh;
+            for (int m0 = 0; m0 < p.M; m0 += rows_per_round) {
+              const int mrows = min(p.M - m0, rows_per_round);
+              float part[32];
+              {
+                int e = 0, mm = 0;
 #pragma unroll
-              for (int e = 0; e < 8; ++e) {
-                const int h = h0 + e;
-                part[e] = 0.0f;
-                if (h <= hl) {
-                  const int wh = (t == first_unit(h, p.G, p.U) / p.KC) ? 0 : 1;
-                  part[e] = __ldcg(p.slots + (static_cast<size_t>(2 * h + wh) * BN + m) * kTileRows + row);
+                for (int q = 0; q < 32; ++q) {
+                  part[q] = 0.0f;
+                  if (mm < mrows) {
+                    part[q] = __ldcg(p.slots + (static_cast<size_t>(slot_of(hf + e)) * BN + m0 + mm) * kTileRows + row);
+                  }
+                  if (++e == nh) { e = 0; ++mm; }
                 }
               }
+              int e = 0, mm = 0;
+              float sum = 0.0f;
 #pragma unroll
-              for (int e = 0; e < 8; ++e) s += part[e];
+              for (int q = 0; q < 32; ++q) {
+                if (mm < mrows) {
+                  sum += part[q];
+                  if (e == nh - 1) {
+                    p.y[static_cast<size_t>(m0 + mm) * p.N + static_cast<size_t>(t) * kTileRows + row] =
+                        __bfloat16_as_ushort(__float2bfloat16_rn(sum));
+                    sum = 0.0f;
+                  }
+                }
+                if (++e == nh) { e = 0; ++mm; }
+              }
             }
-            p.y[static_cast<size_t>(m) * p.N + static_cast<size_t>(t) * kTileRows + row] =
-                __bfloat16_as_ushort(__float2bfloat16_rn(s));
+          } else {
+            for (int m = 0; m < p.M; ++m) {
+              float tot = 0.0f;
+              for (int h0 = hf; h0 <= hl; h0 += 32) {
+                float part[32];
+#pragma unroll
+                for (int q = 0; q < 32; ++q) {
+                  part[q] = 0.0f;
+                  const int h = h0 + q;
+                  if (h <= hl)
+                    part[q] = __ldcg(p.slots + (static_cast<size_t>(slot_of(h)) * BN + m) * kTileRows + row);
+                }
+#pragma unroll
+                for (int q = 0; q < 32; ++q) tot += part[q];
+              }
+              p.y[static_cast<size_t>(m) * p.N + static_cast<size_t>(t) * kTileRows + row] =
+                  __bfloat16_as_ushort(__float2bfloat16_rn(tot));
+            }
           }
         }
       }
@@ -1021,46 +1161,69 @@ fused_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
     }
 
     if (p.fast) {
-      // ---- per unit, on the x chunk and V rows the producer staged: quantise
-      // (small M), x sums and the V side, then release the staging slot
-      for (int k = 0; k < nunits && ok; ++k) {
-        const int u = u0 + k, t = u / p.KC, c = u % p.KC, s = k % ST;
-        const int nw = min(kXWords, p.KW - c * kXWords);
-        const uint16_t* xcur = reinterpret_cast<const uint16_t*>(smem + L::kXS + s * L::kXStride);
-        const uint32_t* vcur = reinterpret_cast<const uint32_t*>(smem + L::kXS + s * L::kXStride + L::kXBytes);
-        if (!group_wait(xfull_bar(s), (k / ST) & 1, kBarAlu, kAluThreads, ctl)) {
-          ok = false;
-          break;
+      // ---- on the x chunks and V rows the producer staged, a batch of up to ST
+      // units at a time (one per stage): quantise all of them (small M), release
+      // them to the MMA, then the V side of each, then free the stages.
+      for (int k0 = 0; k0 < nunits && ok; k0 += ST) {
+        const int nb = min(ST, nunits - k0);
+        for (int j = 0; j < nb && ok; ++j) {
+          const int k = k0 + j;
+          if (!group_wait(xfull_bar(k % ST), (k / ST) & 1, kBarAlu, kAluThreads, ctl)) ok = false;
         }
+        if (!ok) break;
         const int mcnt = p.M;                          // fast path: M <= 32, one pass
         if (p.inq) {
-          quant_chunk(xcur, mcnt, nw, smem + L::kB + s * BN * 128, smem + L::kSFB + s * kSfBytes, tid);
+          // one thread per element pair; the 8 pairs of a 16-element block sit in 8
+          // consecutive lanes (block max by shuffles)
+          const int per_unit = mcnt * 128;
+          for (int idx = tid; idx < nb * per_unit; idx += kAluThreads) {
+            const int j = idx / per_unit, rem = idx % per_unit, m = rem >> 7, pr = rem & 127;
+            const int k = k0 + j, s = k % ST, c = (u0 + k) % p.KC;
+            const int nw = min(kXWords, p.KW - c * kXWords);
+            const uint32_t w2 = *reinterpret_cast<const uint32_t*>(smem + L::kXS + s * L::kXStride +
+                                                                   m * (kSubK * 2) + pr * 4);
+            const float v0 = bf16_bits_to_f32(w2 & 0xFFFFu), v1 = bf16_bits_to_f32(w2 >> 16);
+            float amax = fmaxf(fabsf(v0), fabsf(v1));
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
+            const uint32_t sb = e4m3_from_f32(__fdiv_rn(amax, 6.0f));
+            const float S = e4m3_to_f32(sb);
+            const E2M1Thresholds th = e2m1_thresholds(S);
+            const uint32_t byte = e2m1_code_bf16(v0, th, S == 0.0f) | (e2m1_code_bf16(v1, th, S == 0.0f) << 4);
+            if (pr < nw * 16) {
+              smem[L::kB + s * BN * 128 + m * 128 + ((((pr >> 4) ^ (m & 7)) << 4) | (pr & 15))] =
+                  static_cast<uint8_t>(byte);
+              if ((pr & 7) == 0)
+                smem[L::kSFB + s * kSfBytes + (pr >> 5) * 512 + (m & 31) * 16 + ((m >> 5) & 3) * 4 +
+                     ((pr >> 3) & 3)] = static_cast<uint8_t>(sb);
+            }
+          }
           fence_proxy_async_smem();
           named_barrier(kBarAlu, kAluThreads);
           if (a == 0) {
-            if (lane == 0) mbar_arrive(full_bar(s));
+            if (lane < nb) mbar_arrive(full_bar((k0 + lane) % ST));
             __syncwarp();
           }
         }
         if (shared_z) {
-          int i_lo, i_hi;
-          vside_ranks(p, t, i_lo, i_hi);
-          chunk_xsum_dispatch(xcur, mcnt, nw, B.xsw, B.xs_s, a, lane, tid);
-          for (int r0 = i_lo; r0 < i_hi; r0 += kVRanks) {
-            const int nr = min(kVRanks, i_hi - r0);
-            vside_chunk_dispatch(xcur, vcur + (r0 - i_lo) * kXWords, mcnt, nr, nw, B.red_s, B.vout, a,
-                                 lane, tid);
-            for (int idx = tid; idx < mcnt * nr; idx += kAluThreads) {
-              const int m = idx / nr, i = idx % nr;
-              p.zpart[(static_cast<size_t>(c) * p.M + m) * p.rpad + r0 + i] =
-                  B.xs_s[m] - 2.0f * B.vout[m * kVRanks + i];
-            }
-            named_barrier(kBarAlu, kAluThreads);
-          }
+          const int rgu = (p.r + p.T - 1) / p.T / 8 + 1;         // rank groups of 8 per unit (upper bound)
+          auto info = [&](int j, const uint16_t*& xc, const uint32_t*& vrows, int& c, int& i_lo, int& nr,
+                          int& nw) {
+            const int k = k0 + j, u = u0 + k, t = u / p.KC, s = k % ST;
+            c = u % p.KC;
+            nw = min(kXWords, p.KW - c * kXWords);
+            xc = reinterpret_cast<const uint16_t*>(smem + L::kXS + s * L::kXStride);
+            vrows = reinterpret_cast<const uint32_t*>(smem + L::kXS + s * L::kXStride + L::kXBytes);
+            int i_hi;
+            vside_ranks(p, t, i_lo, i_hi);
+            nr = i_hi - i_lo;
+          };
+          vside_batch<MGV>(p, nb, mcnt, rgu, info, B.xsw, a, lane);
         }
-        named_barrier(kBarAlu, kAluThreads);           // every read of the slot is done
+        named_barrier(kBarAlu, kAluThreads);           // every read of the batch's slots is done
         if (a == 0) {
-          if (lane == 0) mbar_arrive(empty_bar(s));
+          if (lane < nb) mbar_arrive(empty_bar((k0 + lane) % ST));
           __syncwarp();
         }
       }
@@ -1127,10 +1290,10 @@ fused_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
           }
           if (shared_z) {
             const int r0 = i_lo + sub * kVRanks, nr = min(kVRanks, i_hi - r0);
-            if (sub == 0) chunk_xsum_dispatch(xcur, mcnt, nw, B.xsw, B.xs_s, a, lane, tid);
+            if (sub == 0) chunk_xsum<XV>(xcur, mcnt, nw, B.xsw, B.xs_s, a, lane, tid);
             if (nr > 0) {
-              vside_chunk_dispatch(xcur, B.vb + buf * kVRanks * kXWords, mcnt, nr, nw, B.red_s, B.vout, a,
-                                   lane, tid);
+              vside_chunk<MGV>(xcur, B.vb + buf * kVRanks * kXWords, mcnt, nr, nw, B.red_s, B.vout, a, lane,
+                               tid);
               for (int idx = tid; idx < mcnt * nr; idx += kAluThreads) {
                 const int m = idx / nr, i = idx % nr;
                 p.zpart[(static_cast<size_t>(c) * p.M + m0 + m) * p.rpad + r0 + i] =
@@ -1159,8 +1322,8 @@ fused_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
           const int t = t_first + seg;
           if (a == 0) {
             if (lane == 0) {
-              const int hf = owner_cta(static_cast<long long>(t) * p.KC, p.G, p.U);
-              const int hl = owner_cta(static_cast<long long>(t + 1) * p.KC - 1, p.G, p.U);
+              const int hf = owner_cta(static_cast<uint32_t>(t * p.KC), p.G, p.U);
+              const int hl = owner_cta(static_cast<uint32_t>((t + 1) * p.KC - 1), p.G, p.U);
               const uint32_t old = atomicAdd(p.vtick + t, 1u);
               const bool last = old == static_cast<uint32_t>(hl - hf);
               if (last) atomicExch(p.vtick + t, 0u);
@@ -1176,14 +1339,41 @@ fused_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
             int i_lo, i_hi;
             vside_ranks(p, t, i_lo, i_hi);
             const int nr = i_hi - i_lo;
+            const int per_c = p.M * nr;                     // values per chunk partial
             const size_t stride = static_cast<size_t>(p.M) * p.rpad;
-            for (int idx = tid; idx < p.M * nr; idx += kAluThreads) {
+            float* acc_s = B.corr_s;                        // running sums [M][nr]
+            float* stg = B.corr_s + 4096;                   // one round of partials
+            const int cpr = max(1, 4096 / max(per_c, 1));   // chunks per round
+            for (int idx = tid; idx < per_c; idx += kAluThreads) acc_s[idx] = 0.0f;
+            for (int c0r = 0; c0r < p.KC; c0r += cpr) {
+              const int ncr = min(cpr, p.KC - c0r);
+              const int total = ncr * per_c;
+              float tmp[16];
+#pragma unroll
+              for (int q = 0; q < 16; ++q) {
+                const int idx = tid + q * kAluThreads;
+                tmp[q] = 0.0f;
+                if (idx < total) {
+                  const int cc = idx / per_c, rem = idx % per_c, m = rem / nr, i = rem % nr;
+                  tmp[q] = __ldcg(p.zpart + (c0r + cc) * stride + static_cast<size_t>(m) * p.rpad + i_lo + i);
+                }
+              }
+#pragma unroll
+              for (int q = 0; q < 16; ++q) {
+                const int idx = tid + q * kAluThreads;
+                if (idx < total) stg[idx] = tmp[q];
+              }
+              named_barrier(kBarAlu, kAluThreads);
+              for (int idx = tid; idx < per_c; idx += kAluThreads) {
+                float sum = acc_s[idx];
+                for (int cc = 0; cc < ncr; ++cc) sum += stg[cc * per_c + idx];
+                acc_s[idx] = sum;
+              }
+              named_barrier(kBarAlu, kAluThreads);
+            }
+            for (int idx = tid; idx < per_c; idx += kAluThreads) {
               const int m = idx / nr, i = i_lo + idx % nr;
-              const float* src = p.zpart + static_cast<size_t>(m) * p.rpad + i;
-              float s = 0.0f;
-#pragma unroll 4
-              for (int c = 0; c < p.KC; ++c) s += __ldcg(src + c * stride);
-              p.zfin[static_cast<size_t>(m) * p.rpad + i] = __fmul_rn(__ldg(p.alpha + i), s);
+              p.zfin[static_cast<size_t>(m) * p.rpad + i] = __fmul_rn(__ldg(p.alpha + i), acc_s[idx]);
             }
             __threadfence();
             named_barrier(kBarAlu, kAluThreads);
@@ -1198,8 +1388,8 @@ fused_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
       const uint32_t target = static_cast<uint32_t>(p.zdirect ? p.G : p.T);
       bool okw = true;
       if (a == 0) {
-        okw = spin_until_geq(p.z_ready, target, ctl);
-        __syncwarp();
+        if (lane == 0) okw = spin_until_geq(p.z_ready, target, ctl);
+        okw = __shfl_sync(0xffffffffu, okw ? 1 : 0, 0) != 0;
         if (lane == 0 && okw) {
           const uint32_t old = atomicAdd(p.z_seen, 1u);
           if (old == static_cast<uint32_t>(p.G - 1)) {
@@ -1228,7 +1418,7 @@ fused_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
             ok = false;
             break;
           }
-          uside_dispatch(p, t, b_lo, b_hi, m0, mcnt, B, a, lane, tid);
+          uside_pass<MGU, MGV>(p, t, b_lo, b_hi, m0, mcnt, B, a, lane, tid);
           mbar_arrive(corrf_bar);
           ++corr_round;
         }
@@ -1238,191 +1428,24 @@ fused_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
   }
 
   // ------------------------------------------------------------------ teardown
+  // Each warp reports once it no longer touches TMEM or the staging buffers;
+  // warp 1 frees TMEM after all of them (bounded wait).
+  __syncwarp();
   tc_fence_before();
-  __syncthreads();
+  if (lane == 0) mbar_arrive(done_bar);
   if (warp == 1) {
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(done_bar, 0)) {
+      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        record_error(p.status, kDevErrTimeout);
+        break;
+      }
+    }
+    __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
 }
 
-// ------------------------------------------------------------------ host side
-
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(ptr);
-  });
-  return fn;
-}
-
-// 2-D byte tensor [rows][inner_bytes], box [box_rows][128 B], 128-byte swizzle.
-bool make_tmap(CUtensorMap* m, const void* base, uint64_t inner_bytes, uint64_t rows, uint32_t box_rows) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[2] = {inner_bytes, rows};
-  const cuuint64_t strides[1] = {inner_bytes};
-  const cuuint32_t box[2] = {128, box_rows};
-  const cuuint32_t estr[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-// 2-D tensor without swizzle: [rows][inner elements of elem_bytes], box [box_rows][box_inner].
-bool make_tmap_plain(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint32_t elem_bytes,
-                     uint64_t inner, uint64_t rows, uint32_t box_inner, uint32_t box_rows) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[2] = {inner, rows};
-  const cuuint64_t strides[1] = {inner * elem_bytes};
-  const cuuint32_t box[2] = {box_inner, box_rows};
-  const cuuint32_t estr[2] = {1, 1};
-  return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-template <int BN, int ST>
-cudaError_t launch_fused(const CUtensorMap& tw, const CUtensorMap& tx, const CUtensorMap& txs,
-                         const CUtensorMap& tv, const FusedParams& fp, cudaStream_t s, bool pdl) {
-  using L = Layout<BN, ST>;
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(fused_kernel<BN, ST>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    L::kAlloc);
-  });
-  if (attr_err != cudaSuccess) return attr_err;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(fp.G));
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = L::kAlloc;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, fused_kernel<BN, ST>, tw, tx, txs, tv, fp);
-}
-
-int pick_bn(int M) {
-  if (M <= 16) return 16;
-  if (M <= 32) return 32;
-  if (M <= 64) return 64;
-  return 128;
-}
-
 }  // namespace
-
-int resolve_mode(int M, int N, int K, int r, int requested) {
-  (void)M; (void)N; (void)K; (void)r;
-  if (requested == BILOCO_MODE_SHARED_Z || requested == BILOCO_MODE_LOCAL_Z) return requested;
-  return BILOCO_MODE_SHARED_Z;
-}
-
-int gemm_kernel_count_for(int M) { return M <= kInKernelQuantMaxM ? 1 : 2; }
-
-int run_gemm(const GemmArgs& a, cudaStream_t s) {
-  const int M = a.M, N = a.N, K = a.K, r = a.r;
-  const int KC = (K + kUnitK - 1) / kUnitK;
-  const int T = N / kTileRows;
-  const int U = T * KC;
-  const int G = std::min(num_sms(), U);
-  const int KW = K / 32;
-  const int rpad = std::max((r + kRB - 1) / kRB, 1) * kRB;
-  const int BN = pick_bn(M);
-  const bool inq = M <= kInKernelQuantMaxM;
-  const bool zdirect = (M <= 2) || (M * KC <= 64);
-  const bool shared_z = r > 0 && a.mode == BILOCO_MODE_SHARED_Z;
-  const bool unit_alu = inq || shared_z;
-  const int ranks_per_tile = (r + T - 1) / T;
-  const bool fast = unit_alu && BN <= 32 && K % 128 == 0 && (!shared_z || ranks_per_tile <= kVStageRanks);
-
-  ScratchNeed need;
-  need.act_fp4 = inq ? 16 : static_cast<size_t>(M) * K / 2;
-  need.act_sf = inq ? 16 : static_cast<size_t>(KC) * kSfBytes;
-  need.zpart = r ? static_cast<size_t>(KC) * M * rpad * 4 : 16;
-  need.zfin = r ? static_cast<size_t>(M) * rpad * 4 : 16;
-  need.slots = static_cast<size_t>(2 * G) * BN * kTileRows * 4;
-  need.counter_words = 2 + 2 * static_cast<size_t>(T);
-  Scratch* sc = get_scratch(s, need);
-  if (!sc) return BILOCO_ERR_NOMEM;
-
-  cudaError_t e = cudaSuccess;
-  if (!inq) {
-    e = launch_prep_act(a.x, M, K, sc->act_fp4, sc->act_sf, s);
-    if (e != cudaSuccess) return BILOCO_ERR_CUDA;
-  }
-
-  CUtensorMap tw, tx, txs, tv;
-  if (!make_tmap(&tw, a.W_fp4, static_cast<uint64_t>(K) / 2, static_cast<uint64_t>(N), kTileRows))
-    return BILOCO_ERR_CUDA;
-  if (inq) {
-    tx = tw;                                           // not read when quantising in-kernel
-  } else if (!make_tmap(&tx, sc->act_fp4, static_cast<uint64_t>(K) / 2, static_cast<uint64_t>(M), BN)) {
-    return BILOCO_ERR_CUDA;
-  }
-  const int bxr = BN <= 16 ? 16 : 32;
-  txs = tw;
-  tv = tw;
-  if (fast) {
-    if (!make_tmap_plain(&txs, a.x, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, static_cast<uint64_t>(K),
-                         static_cast<uint64_t>(M), kSubK, static_cast<uint32_t>(bxr)))
-      return BILOCO_ERR_CUDA;
-    if (shared_z && !make_tmap_plain(&tv, a.Vbits, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4,
-                                     static_cast<uint64_t>(KW), static_cast<uint64_t>(r), kXWords,
-                                     kVStageRanks))
-      return BILOCO_ERR_CUDA;
-  }
-
-  FusedParams fp = {};
-  fp.w_sf = a.W_sf;
-  fp.x_sf = sc->act_sf;
-  fp.gscale = a.gscale;
-  fp.Ubits = a.Ubits;
-  fp.Vbits = a.Vbits;
-  fp.alpha = a.alpha;
-  fp.x = a.x;
-  fp.y = a.y;
-  fp.zpart = sc->zpart;
-  fp.zfin = sc->zfin;
-  fp.slots = sc->slots;
-  fp.z_ready = sc->counters;
-  fp.z_seen = sc->counters + 1;
-  fp.tickets = sc->counters + 2;
-  fp.vtick = sc->counters + 2 + T;
-  fp.status = sc->status;
-  fp.M = M; fp.N = N; fp.K = K; fp.r = r;
-  fp.KC = KC; fp.T = T; fp.U = U; fp.G = G; fp.KW = KW;
-  fp.rpad = rpad;
-  fp.RW = (r + 31) / 32;
-  fp.mode = a.mode;
-  fp.inq = inq ? 1 : 0;
-  fp.zdirect = zdirect ? 1 : 0;
-  fp.fast = fast ? 1 : 0;
-  fp.unit_alu = unit_alu ? 1 : 0;
-  fp.bxr = bxr;
-
-  const bool pdl = !inq;
-  switch (BN) {
-    case 16: e = launch_fused<16, 5>(tw, tx, txs, tv, fp, s, pdl); break;
-    case 32: e = launch_fused<32, 3>(tw, tx, txs, tv, fp, s, pdl); break;
-    case 64: e = launch_fused<64, 4>(tw, tx, txs, tv, fp, s, pdl); break;
-    default: e = launch_fused<128, 3>(tw, tx, txs, tv, fp, s, pdl); break;
-  }
-  return e == cudaSuccess ? BILOCO_OK : BILOCO_ERR_CUDA;
-}
-
 }  // namespace biloco

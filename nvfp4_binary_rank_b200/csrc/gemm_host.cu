@@ -1,0 +1,190 @@
+// Host side of the fused GEMM: shape decomposition, scratch, tensor maps and the
+// choice of kernel instance.
+#include <algorithm>
+#include <cstdint>
+#include <mutex>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "../../include/biloco.h"
+#include "fused_launch.h"
+#include "fused_params.h"
+#include "internal.h"
+
+namespace biloco {
+
+namespace {
+
+constexpr int kTileRows = 128;
+constexpr int kUnitK = 256;
+constexpr int kSfBytes = 2048;
+constexpr int kRB = 16;
+constexpr int kSubK = 256;
+constexpr int kXWords = 8;
+constexpr int kVStageRanks = 64;
+constexpr int kInKernelQuantMaxM = 8;
+
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// 2-D byte tensor [rows][inner_bytes], box [box_rows][128 B], 128-byte swizzle.
+bool make_tmap(CUtensorMap* m, const void* base, uint64_t inner_bytes, uint64_t rows, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {inner_bytes, rows};
+  const cuuint64_t strides[1] = {inner_bytes};
+  const cuuint32_t box[2] = {128, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 2-D tensor without swizzle: [rows][inner elements of elem_bytes], box [box_rows][box_inner].
+bool make_tmap_plain(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint32_t elem_bytes,
+                     uint64_t inner, uint64_t rows, uint32_t box_inner, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {inner, rows};
+  const cuuint64_t strides[1] = {inner * elem_bytes};
+  const cuuint32_t box[2] = {box_inner, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+
+int pick_bn(int M) {
+  if (M <= 16) return 16;
+  if (M <= 32) return 32;
+  if (M <= 64) return 64;
+  return 128;
+}
+
+cudaError_t launch_for(int M, const CUtensorMap& tw, const CUtensorMap& tx, const CUtensorMap& txs,
+                       const CUtensorMap& tv, const FusedParams& fp, cudaStream_t s, bool pdl) {
+  if (M <= 1) return launch_fused_16_1(tw, tx, txs, tv, fp, s, pdl);
+  if (M <= 2) return launch_fused_16_2(tw, tx, txs, tv, fp, s, pdl);
+  if (M <= 4) return launch_fused_16_4(tw, tx, txs, tv, fp, s, pdl);
+  if (M <= 8) return launch_fused_16_8(tw, tx, txs, tv, fp, s, pdl);
+  if (M <= 16) return launch_fused_16_16(tw, tx, txs, tv, fp, s, pdl);
+  if (M <= 32) return launch_fused_32_32(tw, tx, txs, tv, fp, s, pdl);
+  if (M <= 64) return launch_fused_64_32(tw, tx, txs, tv, fp, s, pdl);
+  return launch_fused_128_32(tw, tx, txs, tv, fp, s, pdl);
+}
+
+}  // namespace
+
+int resolve_mode(int M, int N, int K, int r, int requested) {
+  (void)M; (void)N; (void)K; (void)r;
+  if (requested == BILOCO_MODE_SHARED_Z || requested == BILOCO_MODE_LOCAL_Z) return requested;
+  return BILOCO_MODE_SHARED_Z;
+}
+
+int gemm_kernel_count_for(int M) { return M <= kInKernelQuantMaxM ? 1 : 2; }
+
+int run_gemm(const GemmArgs& a, cudaStream_t s) {
+  const int M = a.M, N = a.N, K = a.K, r = a.r;
+  const int KC = (K + kUnitK - 1) / kUnitK;
+  const int T = N / kTileRows;
+  const int U = T * KC;
+  const int G = std::min(num_sms(), U);
+  const int KW = K / 32;
+  const int rpad = std::max((r + kRB - 1) / kRB, 1) * kRB;
+  const int BN = pick_bn(M);
+  const bool inq = M <= kInKernelQuantMaxM;
+  const bool zdirect = (M <= 2) || (M * KC <= 64);
+  const bool shared_z = r > 0 && a.mode == BILOCO_MODE_SHARED_Z;
+  const bool unit_alu = inq || shared_z;
+  const int ranks_per_tile = (r + T - 1) / T;
+  const bool fast = unit_alu && BN <= 32 && K % 128 == 0 && (!shared_z || ranks_per_tile <= kVStageRanks);
+
+  ScratchNeed need;
+  need.act_fp4 = inq ? 16 : static_cast<size_t>(M) * K / 2;
+  need.act_sf = inq ? 16 : static_cast<size_t>(KC) * kSfBytes;
+  need.zpart = r ? static_cast<size_t>(KC) * M * rpad * 4 : 16;
+  need.zfin = r ? static_cast<size_t>(M) * rpad * 4 : 16;
+  need.slots = static_cast<size_t>(2 * G) * BN * kTileRows * 4;
+  need.counter_words = 2 + 2 * static_cast<size_t>(T);
+  Scratch* sc = get_scratch(s, need);
+  if (!sc) return BILOCO_ERR_NOMEM;
+
+  cudaError_t e = cudaSuccess;
+  if (!inq) {
+    e = launch_prep_act(a.x, M, K, sc->act_fp4, sc->act_sf, s);
+    if (e != cudaSuccess) return BILOCO_ERR_CUDA;
+  }
+
+  CUtensorMap tw, tx, txs, tv;
+  if (!make_tmap(&tw, a.W_fp4, static_cast<uint64_t>(K) / 2, static_cast<uint64_t>(N), kTileRows))
+    return BILOCO_ERR_CUDA;
+  if (inq) {
+    tx = tw;                                           // not read when quantising in-kernel
+  } else if (!make_tmap(&tx, sc->act_fp4, static_cast<uint64_t>(K) / 2, static_cast<uint64_t>(M), BN)) {
+    return BILOCO_ERR_CUDA;
+  }
+  const int bxr = BN <= 16 ? 16 : 32;
+  txs = tw;
+  tv = tw;
+  if (fast) {
+    if (!make_tmap_plain(&txs, a.x, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, static_cast<uint64_t>(K),
+                         static_cast<uint64_t>(M), kSubK, static_cast<uint32_t>(bxr)))
+      return BILOCO_ERR_CUDA;
+    if (shared_z && !make_tmap_plain(&tv, a.Vbits, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4,
+                                     static_cast<uint64_t>(KW), static_cast<uint64_t>(r), kXWords,
+                                     kVStageRanks))
+      return BILOCO_ERR_CUDA;
+  }
+
+  FusedParams fp = {};
+  fp.w_sf = a.W_sf;
+  fp.x_sf = sc->act_sf;
+  fp.gscale = a.gscale;
+  fp.Ubits = a.Ubits;
+  fp.Vbits = a.Vbits;
+  fp.alpha = a.alpha;
+  fp.x = a.x;
+  fp.y = a.y;
+  fp.zpart = sc->zpart;
+  fp.zfin = sc->zfin;
+  fp.slots = sc->slots;
+  fp.z_ready = sc->counters;
+  fp.z_seen = sc->counters + 1;
+  fp.tickets = sc->counters + 2;
+  fp.vtick = sc->counters + 2 + T;
+  fp.status = sc->status;
+  fp.M = M; fp.N = N; fp.K = K; fp.r = r;
+  fp.KC = KC; fp.T = T; fp.U = U; fp.G = G; fp.KW = KW;
+  fp.rpad = rpad;
+  fp.RW = (r + 31) / 32;
+  fp.mode = a.mode;
+  fp.inq = inq ? 1 : 0;
+  fp.zdirect = zdirect ? 1 : 0;
+  fp.fast = fast ? 1 : 0;
+  fp.unit_alu = unit_alu ? 1 : 0;
+  fp.bxr = bxr;
+
+  const bool pdl = !inq;
+  e = launch_for(M, tw, tx, txs, tv, fp, s, pdl);
+  return e == cudaSuccess ? BILOCO_OK : BILOCO_ERR_CUDA;
+}
+
+}  // namespace biloco

@@ -61,11 +61,50 @@ __device__ __forceinline__ float amax16(const float (&v)[16]) {
   return a;
 }
 
+// E2M1 code of a BF16 value v under block scale S, without dividing.
+//
+// The format asks for E2M1_RNE(RN_fp32(v / S)).  S is an E4M3 value (at most 4
+// significant bits) and every E2M1 rounding boundary t in {.25, .75, 1.25, 1.75,
+// 2.5, 3.5, 5} has at most 3, so t * S is exact in FP32.  A BF16 |v| has at most 8
+// significant bits, so it is either equal to t * S or at least one BF16 step
+// (relative 2^-8) away from it, far outside the FP32 rounding of the quotient.
+// Hence RN(|v| / S) > t  <=>  |v| > t * S  and  RN(|v| / S) == t  <=>  |v| == t * S,
+// and comparing |v| with the seven exact products gives the same code as the
+// division.  At an exact boundary the even code wins (ties to even), i.e. the
+// boundaries .75, 1.75 and 3.5 round up and the others round down.
+struct E2M1Thresholds {
+  float t[7];
+};
+__device__ __forceinline__ E2M1Thresholds e2m1_thresholds(float S) {
+  E2M1Thresholds th;
+  th.t[0] = 0.25f * S; th.t[1] = 0.75f * S; th.t[2] = 1.25f * S; th.t[3] = 1.75f * S;
+  th.t[4] = 2.5f * S;  th.t[5] = 3.5f * S;  th.t[6] = 5.0f * S;
+  return th;
+}
+__device__ __forceinline__ uint32_t e2m1_code_bf16(float v, const E2M1Thresholds& th, bool zero_scale) {
+  const float a = fabsf(v);
+  uint32_t c = (a > th.t[0]) + (a >= th.t[1]) + (a > th.t[2]) + (a >= th.t[3]) + (a > th.t[4]) +
+               (a >= th.t[5]) + (a > th.t[6]);
+  if (zero_scale) c = 0;
+  return (c != 0 && v < 0.0f) ? (c | 8u) : c;
+}
+
 // Activation block (no tensor scale): s = E4M3(amax / 6), codes = E2M1(x / s).
+// Inputs are BF16 values, so the division-free rounding above applies.
 __device__ __forceinline__ uint32_t quant_act_block(const float (&v)[16], uint2& codes) {
   const float t = __fdiv_rn(amax16(v), 6.0f);
   const uint32_t s = e4m3_from_f32(t);
-  codes = encode_block16(v, e4m3_to_f32(s));
+  const float S = e4m3_to_f32(s);
+  const E2M1Thresholds th = e2m1_thresholds(S);
+  codes = make_uint2(0u, 0u);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    codes.x |= (e2m1_code_bf16(v[2 * j], th, S == 0.0f) | (e2m1_code_bf16(v[2 * j + 1], th, S == 0.0f) << 4))
+               << (8 * j);
+    codes.y |= (e2m1_code_bf16(v[8 + 2 * j], th, S == 0.0f) |
+                (e2m1_code_bf16(v[8 + 2 * j + 1], th, S == 0.0f) << 4))
+               << (8 * j);
+  }
   return s;
 }
 
