@@ -157,6 +157,43 @@ int biloco_gemm(const void *x_bf16, const uint8_t *W_fp4, const uint8_t *W_sf,
                 const float *alpha, void *y_bf16, int M, int N, int K, int r,
                 biloco_stream_t stream);
 
+/*
+ * biloco_gemm_noalloc - biloco_gemm with no device allocation.
+ * The BiLoCo pages have no counterpart of this call: it exists for callers that
+ * cannot let the library allocate, e.g. an engine that has reserved nearly all of
+ * HBM for its own pools, or a decode loop that cannot have its stream stalled
+ * while biloco_gemm grows its per-stream scratch (synchronise, free, cudaMalloc).
+ *
+ * Same arguments, limits, results and error codes as biloco_gemm; the results
+ * equal biloco_gemm's for the same shape and mode.  Its scratch is one static
+ * device array of BILOCO_NOALLOC_SCRATCH_BYTES per device, part of the library's
+ * device code; the call never calls cudaMalloc or cudaFree.  Extra limits,
+ * checked on the host before anything is launched (BILOCO_ERR_SHAPE otherwise):
+ *   N <= BILOCO_NOALLOC_MAX_N, and the call's scratch fits the array.  That
+ *   scratch is 16 896 bytes of status and counters plus, each rounded up to 256:
+ *     M > 8:  M*K/2 + ceil(K/256)*2048          (quantised activation)
+ *     r > 0:  (ceil(K/256) + 1) * M * rpad * 4  (z partials and z; rpad = 16*ceil(r/16))
+ *     always: 2 * G * BN * 512                  (split-K partials)
+ *   with G = min(#SMs, (N/128)*ceil(K/256)) and BN = 16, 32, 64, 128 for
+ *   M <= 16, 32, 64, 128.  On a 148-SM B200 every M <= 32 shape with
+ *   K <= 13824 and r <= 512 fits; M > 64 fits only tiny weights.
+ * Caveats:
+ *   - There is one array per device, shared by all streams and host threads:
+ *     calls that overlap in time (on different streams, or from several threads
+ *     without ordering) race on it and give wrong results.  Order the calls.
+ *   - The first call on a device looks up the array's address
+ *     (cudaGetSymbolAddress) and clears its status and counters with an
+ *     asynchronous memset; make it before any stream capture begins.
+ *   - Device-side errors (an expired bounded wait) are reported by
+ *     biloco_last_error(stream), which also clears the array's counters.
+ */
+#define BILOCO_NOALLOC_SCRATCH_BYTES (16u << 20)
+#define BILOCO_NOALLOC_MAX_N (1 << 18)
+int biloco_gemm_noalloc(const void *x_bf16, const uint8_t *W_fp4, const uint8_t *W_sf,
+                        const float *gscale, const uint32_t *Ubits, const uint32_t *Vbits,
+                        const float *alpha, void *y_bf16, int M, int N, int K, int r,
+                        biloco_stream_t stream);
+
 /* Select the z schedule for later biloco_gemm calls (process-wide). */
 int biloco_set_mode(int mode);
 /* The schedule biloco_gemm would use for this shape under the current setting. */
@@ -165,7 +202,9 @@ int biloco_resolve_mode(int M, int N, int K, int r);
 /*
  * biloco_last_error - synchronise `stream`, return and clear the first error a
  * kernel on it recorded (BILOCO_ERR_TIMEOUT when a bounded wait expired), or
- * BILOCO_OK.  After an error the stream's scratch counters are reset.
+ * BILOCO_OK.  After an error the stream's scratch counters are reset.  The
+ * static scratch of biloco_gemm_noalloc on the current device is checked and
+ * reset the same way.
  */
 int biloco_last_error(biloco_stream_t stream);
 

@@ -35,6 +35,7 @@ SIGNATURES = {
     "biloco_pack_weight": (_I, [_P, _I, _I, _P, _P, _P, _P]),
     "biloco_weight_sf_bytes": (ctypes.c_size_t, [_I, _I]),
     "biloco_gemm": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
+    "biloco_gemm_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
     "biloco_set_mode": (_I, [_I]),
     "biloco_resolve_mode": (_I, [_I, _I, _I, _I]),
     "biloco_last_error": (_I, [_P]),
@@ -132,10 +133,7 @@ def pack_weight(R: torch.Tensor, stream=None):
     return W, sf, g
 
 
-def gemm(x: torch.Tensor, W_fp4: torch.Tensor, W_sf: torch.Tensor, gscale: torch.Tensor,
-         Ubits: torch.Tensor | None, Vbits: torch.Tensor | None, alpha: torch.Tensor | None,
-         out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
-    """y[M, N] (bfloat16) = FP4(x) FP4(R)^T * g + sum_i alpha_i (x . v_i) u_i."""
+def _gemm_call(fn: str, x, W_fp4, W_sf, gscale, Ubits, Vbits, alpha, out, stream):
     _need_cuda(x, "x", torch.bfloat16)
     _need_cuda(W_fp4, "W_fp4", torch.uint8)
     _need_cuda(W_sf, "W_sf", torch.uint8)
@@ -153,11 +151,29 @@ def gemm(x: torch.Tensor, W_fp4: torch.Tensor, W_sf: torch.Tensor, gscale: torch
         out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
     else:
         _need_cuda(out, "out", torch.bfloat16)
-    _check("biloco_gemm", load().biloco_gemm(
+    _check(fn, getattr(load(), fn)(
         _ptr(x), _ptr(W_fp4), _ptr(W_sf), _ptr(gscale), _ptr(Ubits if r else None),
         _ptr(Vbits if r else None), _ptr(alpha if r else None), _ptr(out), M, N, K, r,
         _stream(stream)))
     return out
+
+
+def gemm(x: torch.Tensor, W_fp4: torch.Tensor, W_sf: torch.Tensor, gscale: torch.Tensor,
+         Ubits: torch.Tensor | None, Vbits: torch.Tensor | None, alpha: torch.Tensor | None,
+         out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """y[M, N] (bfloat16) = FP4(x) FP4(R)^T * g + sum_i alpha_i (x . v_i) u_i."""
+    return _gemm_call("biloco_gemm", x, W_fp4, W_sf, gscale, Ubits, Vbits, alpha, out, stream)
+
+
+def gemm_noalloc(x: torch.Tensor, W_fp4: torch.Tensor, W_sf: torch.Tensor, gscale: torch.Tensor,
+                 Ubits: torch.Tensor | None, Vbits: torch.Tensor | None,
+                 alpha: torch.Tensor | None, out: torch.Tensor | None = None,
+                 stream=None) -> torch.Tensor:
+    """gemm() whose library scratch is a fixed static device array: no device
+    allocation inside the call (only `out`, when not given, is allocated here by
+    PyTorch).  Overlapping calls race on that array; order them."""
+    return _gemm_call("biloco_gemm_noalloc", x, W_fp4, W_sf, gscale, Ubits, Vbits, alpha, out,
+                      stream)
 
 
 def set_mode(mode: int):

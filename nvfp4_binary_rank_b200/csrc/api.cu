@@ -1,5 +1,6 @@
 // C ABI of libbiloco.so: argument checking, per-(device, stream) scratch and the
-// device status word.  The compute lives in quant.cu and gemm.cu.
+// device status word.  The compute lives in quant.cu, gemm_host.cu and the
+// fused_*.cu kernel instances; noalloc.cu holds the static-scratch variant.
 #include <algorithm>
 #include <atomic>
 #include <cstdint>
@@ -145,6 +146,37 @@ Scratch* get_scratch(cudaStream_t stream, const ScratchNeed& need) {
   return &e->s;
 }
 
+int check_gemm_args(const void* x_bf16, const uint8_t* W_fp4, const uint8_t* W_sf, const float* gscale,
+                    const uint32_t* Ubits, const uint32_t* Vbits, const float* alpha, void* y_bf16,
+                    int M, int N, int K, int r, GemmArgs* a) {
+  if (!x_bf16 || !W_fp4 || !W_sf || !gscale || !y_bf16) return BILOCO_ERR_ARG;
+  if (r > 0 && (!Ubits || !Vbits || !alpha)) return BILOCO_ERR_ARG;
+  if (M < 1 || M > BILOCO_MAX_M || N < 128 || N % 128 || K < 64 || K % 64 || r < 0 ||
+      r > BILOCO_MAX_R || N > BILOCO_MAX_N ||
+      static_cast<long long>(N / 128) * ((K + 255) / 256) > BILOCO_MAX_UNITS)
+    return BILOCO_ERR_SHAPE;
+  if (!aligned16(x_bf16) || !aligned16(W_fp4) || !aligned16(W_sf) || !aligned16(y_bf16) ||
+      (reinterpret_cast<uintptr_t>(gscale) & 3u) || (r > 0 && (!aligned16(Ubits) || !aligned16(Vbits) ||
+                                                               (reinterpret_cast<uintptr_t>(alpha) & 3u))))
+    return BILOCO_ERR_ALIGN;
+  int d = check_device();
+  if (d) return d;
+  a->x = static_cast<const uint16_t*>(x_bf16);
+  a->W_fp4 = W_fp4;
+  a->W_sf = W_sf;
+  a->gscale = gscale;
+  a->Ubits = Ubits;
+  a->Vbits = Vbits;
+  a->alpha = alpha;
+  a->y = static_cast<uint16_t*>(y_bf16);
+  a->M = M;
+  a->N = N;
+  a->K = K;
+  a->r = r;
+  a->mode = resolve_mode(M, N, K, r, g_mode.load());
+  return BILOCO_OK;
+}
+
 }  // namespace biloco
 
 using namespace biloco;
@@ -197,32 +229,9 @@ int biloco_pack_weight(const float* R, int N, int K, uint8_t* W_fp4, uint8_t* W_
 int biloco_gemm(const void* x_bf16, const uint8_t* W_fp4, const uint8_t* W_sf, const float* gscale,
                 const uint32_t* Ubits, const uint32_t* Vbits, const float* alpha, void* y_bf16, int M,
                 int N, int K, int r, biloco_stream_t stream) {
-  if (!x_bf16 || !W_fp4 || !W_sf || !gscale || !y_bf16) return BILOCO_ERR_ARG;
-  if (r > 0 && (!Ubits || !Vbits || !alpha)) return BILOCO_ERR_ARG;
-  if (M < 1 || M > BILOCO_MAX_M || N < 128 || N % 128 || K < 64 || K % 64 || r < 0 ||
-      r > BILOCO_MAX_R || N > BILOCO_MAX_N ||
-      static_cast<long long>(N / 128) * ((K + 255) / 256) > BILOCO_MAX_UNITS)
-    return BILOCO_ERR_SHAPE;
-  if (!aligned16(x_bf16) || !aligned16(W_fp4) || !aligned16(W_sf) || !aligned16(y_bf16) ||
-      (reinterpret_cast<uintptr_t>(gscale) & 3u) || (r > 0 && (!aligned16(Ubits) || !aligned16(Vbits) ||
-                                                               (reinterpret_cast<uintptr_t>(alpha) & 3u))))
-    return BILOCO_ERR_ALIGN;
-  int d = check_device();
-  if (d) return d;
   GemmArgs a;
-  a.x = static_cast<const uint16_t*>(x_bf16);
-  a.W_fp4 = W_fp4;
-  a.W_sf = W_sf;
-  a.gscale = gscale;
-  a.Ubits = Ubits;
-  a.Vbits = Vbits;
-  a.alpha = alpha;
-  a.y = static_cast<uint16_t*>(y_bf16);
-  a.M = M;
-  a.N = N;
-  a.K = K;
-  a.r = r;
-  a.mode = resolve_mode(M, N, K, r, g_mode.load());
+  const int st = check_gemm_args(x_bf16, W_fp4, W_sf, gscale, Ubits, Vbits, alpha, y_bf16, M, N, K, r, &a);
+  if (st) return st;
   return run_gemm(a, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -246,17 +255,19 @@ int biloco_last_error(biloco_stream_t stream) {
     for (ScratchEntry* e : g_entries)
       if (e->s.device == dev && e->s.stream == s && e->s.base) sc = &e->s;
   }
-  if (!sc) return BILOCO_OK;
   int status = 0;
-  if (cudaMemcpy(&status, sc->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
-    return BILOCO_ERR_CUDA;
-  if (status != 0) {
-    // a kernel gave up part-way: clear the status and every cross-CTA counter
-    cudaMemset(sc->status, 0, sizeof(int));
-    cudaMemset(sc->counters, 0, sc->counter_words * 4);
-    cudaDeviceSynchronize();
+  if (sc) {
+    if (cudaMemcpy(&status, sc->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+      return BILOCO_ERR_CUDA;
+    if (status != 0) {
+      // a kernel gave up part-way: clear the status and every cross-CTA counter
+      cudaMemset(sc->status, 0, sizeof(int));
+      cudaMemset(sc->counters, 0, sc->counter_words * 4);
+      cudaDeviceSynchronize();
+    }
   }
-  return status;
+  const int static_status = noalloc_take_status();
+  return status != 0 ? status : static_status;
 }
 
 const char* biloco_status_string(int status) {

@@ -101,31 +101,47 @@ int resolve_mode(int M, int N, int K, int r, int requested) {
 
 int gemm_kernel_count_for(int M) { return M <= kInKernelQuantMaxM ? 1 : 2; }
 
-int run_gemm(const GemmArgs& a, cudaStream_t s) {
+GemmPlan plan_gemm(const GemmArgs& a) {
   const int M = a.M, N = a.N, K = a.K, r = a.r;
-  const int KC = (K + kUnitK - 1) / kUnitK;
-  const int T = N / kTileRows;
-  const int U = T * KC;
-  const int G = std::min(num_sms(), U);
-  const int KW = K / 32;
-  const int rpad = std::max((r + kRB - 1) / kRB, 1) * kRB;
-  const int BN = pick_bn(M);
-  const bool inq = M <= kInKernelQuantMaxM;
-  const bool zdirect = (M <= 2) || (M * KC <= 64);
-  const bool shared_z = r > 0 && a.mode == BILOCO_MODE_SHARED_Z;
-  const bool unit_alu = inq || shared_z;
-  const int ranks_per_tile = (r + T - 1) / T;
-  const bool fast = unit_alu && BN <= 32 && K % 128 == 0 && (!shared_z || ranks_per_tile <= kVStageRanks);
+  GemmPlan p;
+  p.KC = (K + kUnitK - 1) / kUnitK;
+  p.T = N / kTileRows;
+  p.U = p.T * p.KC;
+  p.G = std::min(num_sms(), p.U);
+  p.KW = K / 32;
+  p.rpad = std::max((r + kRB - 1) / kRB, 1) * kRB;
+  p.BN = pick_bn(M);
+  p.bxr = p.BN <= 16 ? 16 : 32;
+  p.inq = M <= kInKernelQuantMaxM;
+  p.zdirect = (M <= 2) || (M * p.KC <= 64);
+  p.shared_z = r > 0 && a.mode == BILOCO_MODE_SHARED_Z;
+  p.unit_alu = p.inq || p.shared_z;
+  const int ranks_per_tile = (r + p.T - 1) / p.T;
+  p.fast = p.unit_alu && p.BN <= 32 && K % 128 == 0 && (!p.shared_z || ranks_per_tile <= kVStageRanks);
 
-  ScratchNeed need;
-  need.act_fp4 = inq ? 16 : static_cast<size_t>(M) * K / 2;
-  need.act_sf = inq ? 16 : static_cast<size_t>(KC) * kSfBytes;
-  need.zpart = r ? static_cast<size_t>(KC) * M * rpad * 4 : 16;
-  need.zfin = r ? static_cast<size_t>(M) * rpad * 4 : 16;
-  need.slots = static_cast<size_t>(2 * G) * BN * kTileRows * 4;
-  need.counter_words = 2 + 2 * static_cast<size_t>(T);
-  Scratch* sc = get_scratch(s, need);
+  ScratchNeed& need = p.need;
+  need.act_fp4 = p.inq ? 16 : static_cast<size_t>(M) * K / 2;
+  need.act_sf = p.inq ? 16 : static_cast<size_t>(p.KC) * kSfBytes;
+  need.zpart = r ? static_cast<size_t>(p.KC) * M * p.rpad * 4 : 16;
+  need.zfin = r ? static_cast<size_t>(M) * p.rpad * 4 : 16;
+  need.slots = static_cast<size_t>(2 * p.G) * p.BN * kTileRows * 4;
+  need.counter_words = 2 + 2 * static_cast<size_t>(p.T);
+  return p;
+}
+
+int run_gemm(const GemmArgs& a, cudaStream_t s) {
+  const GemmPlan p = plan_gemm(a);
+  Scratch* sc = get_scratch(s, p.need);
   if (!sc) return BILOCO_ERR_NOMEM;
+  return launch_gemm(a, p, *sc, s);
+}
+
+int launch_gemm(const GemmArgs& a, const GemmPlan& p, const Scratch& scr, cudaStream_t s) {
+  const int M = a.M, N = a.N, K = a.K, r = a.r;
+  const int KC = p.KC, T = p.T, U = p.U, G = p.G, KW = p.KW, rpad = p.rpad, BN = p.BN;
+  const bool inq = p.inq, zdirect = p.zdirect, shared_z = p.shared_z, unit_alu = p.unit_alu;
+  const bool fast = p.fast;
+  const Scratch* sc = &scr;
 
   cudaError_t e = cudaSuccess;
   if (!inq) {
@@ -141,7 +157,7 @@ int run_gemm(const GemmArgs& a, cudaStream_t s) {
   } else if (!make_tmap(&tx, sc->act_fp4, static_cast<uint64_t>(K) / 2, static_cast<uint64_t>(M), BN)) {
     return BILOCO_ERR_CUDA;
   }
-  const int bxr = BN <= 16 ? 16 : 32;
+  const int bxr = p.bxr;
   txs = tw;
   tv = tw;
   if (fast) {

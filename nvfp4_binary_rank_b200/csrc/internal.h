@@ -56,9 +56,32 @@ struct GemmArgs {
   int mode;   // resolved: 1 shared z, 2 local z
 };
 
-// Validated arguments; launches prep + fused kernels.  Returns a BILOCO_* status.
+// Host checks of biloco_gemm's arguments (include/biloco.h); fills `a` with the
+// resolved z schedule.  Returns BILOCO_OK or the error code, launching nothing.
+int check_gemm_args(const void* x_bf16, const uint8_t* W_fp4, const uint8_t* W_sf, const float* gscale,
+                    const uint32_t* Ubits, const uint32_t* Vbits, const float* alpha, void* y_bf16,
+                    int M, int N, int K, int r, GemmArgs* a);
+
+// Shape decomposition of one call: tiles, chunks, grid, kernel options and the
+// scratch the call needs.
+struct GemmPlan {
+  int KC, T, U, G, KW, rpad, BN, bxr;
+  bool inq, zdirect, shared_z, unit_alu, fast;
+  ScratchNeed need;
+};
+GemmPlan plan_gemm(const GemmArgs& a);
+
+// Launches the call's kernels on `s`; `sc` holds at least `p.need`, with its
+// status word and counters zero.  Returns a BILOCO_* status.
+int launch_gemm(const GemmArgs& a, const GemmPlan& p, const Scratch& sc, cudaStream_t s);
+
+// Validated arguments; per-stream scratch, then launch_gemm.  Returns a BILOCO_* status.
 int run_gemm(const GemmArgs& a, cudaStream_t s);
 int resolve_mode(int M, int N, int K, int r, int requested);
+
+// Status word of biloco_gemm_noalloc's static scratch on the current device:
+// returned and, if non-zero, cleared together with its counters (synchronous).
+int noalloc_take_status();
 int gemm_kernel_count_for(int M);
 
 }  // namespace biloco

@@ -68,6 +68,8 @@ def test_host_validation_rejects_bad_arguments_without_a_gpu(lib):
     assert lib.biloco_pack_weight(fake, 100, 64, fake, fake, fake, None) == -2
     assert lib.biloco_quant_act(fake, 1, 24, fake, fake, None) == -2
     assert lib.biloco_pack_signs(None, 1, 1, fake, None) == -1
+    assert lib.biloco_gemm_noalloc(None, fake, fake, fake, None, None, None, fake, 1, 128, 64, 0, None) == -1
+    assert lib.biloco_gemm_noalloc(fake, fake, fake, fake, None, None, None, fake, 1, 100, 64, 0, None) == -2
 
 
 def test_mode_setting(lib):
