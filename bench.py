@@ -56,6 +56,42 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+# ----------------------------------------------------------------------------- ncu traffic
+
+KERNEL_SOURCES = os.path.join(ROOT, "nvfp4_binary_rank_b200", "csrc")
+
+
+def kernel_source_digest() -> str:
+    """sha256 over the library's CUDA/C++ sources (names and contents, sorted)."""
+    import hashlib
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(KERNEL_SOURCES)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            h.update(name.encode())
+            with open(os.path.join(KERNEL_SOURCES, name), "rb") as f:
+                h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(workload: str):
+    """DRAM bytes (read + write) per launch of the fused kernel from the committed
+    ncu summary of this workload, or None when there is none or the kernel
+    sources changed since it was captured."""
+    path = os.path.join(ROOT, "profiles", f"fused_kernel_{workload}.md")
+    try:
+        fields = {}
+        with open(path) as f:
+            for line in f:
+                if ":" in line and line.startswith("- "):
+                    k, v = line[2:].split(":", 1)
+                    fields[k.strip()] = v.strip().strip("`")
+        if fields.get("source_digest") != kernel_source_digest():
+            return None
+        return int(fields["dram_bytes_per_launch"])
+    except (OSError, KeyError, ValueError):
+        return None
+
+
 # ----------------------------------------------------------------------------- clocks
 
 class ClockSampler:
@@ -333,7 +369,8 @@ def run_ours(args):
                    "l2": f"{n_copies_for(w, l2)} weight copies rotated (> L2 {l2 >> 20} MiB)",
                    "launch": f"CUDA graph replay, {nb.gemm_kernel_count(w.M)} kernel(s) per step"},
         "roofline": {"bound": "hbm", "achieved": round(gbs_rank, 1), "peak": peak,
-                     "unit": "GB/s", "frac": round(gbs_rank / peak, 4), "traffic": None,
+                     "unit": "GB/s", "frac": round(gbs_rank / peak, 4),
+                     "traffic": ncu_traffic(w.name),
                      "peak_kind": peak_kind, "per": "step (all kernels of one call)"},
         "e2e": {"value": round(e2e_val, 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "us_per_step": round(e2e_ms * 1e3, 3),

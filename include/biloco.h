@@ -149,8 +149,13 @@ size_t biloco_weight_sf_bytes(int N, int K);
  *           (N/128) * ceil(K/256) <= 2^24
  * Accumulation is FP32 in an unspecified order; results are deterministic for a
  * fixed shape, mode and GPU.  For M <= 8 one kernel is launched (it quantises
- * the activation itself); for larger M an activation quantiser runs first and
- * the fused kernel follows through programmatic dependent launch.
+ * the activation itself); for larger M an activation quantiser runs first.
+ * The fused kernel is launched with programmatic dependent launch: it may start
+ * while the kernel before it on the stream finishes, and it reads W_fp4 and
+ * W_sf before waiting for that kernel (everything else after).  So the weight
+ * operand must not be written by a preceding kernel that triggers early launch
+ * of its dependents (griddepcontrol.launch_dependents); kernels without that
+ * trigger, biloco_pack_weight's included, are fully ordered before the call.
  */
 int biloco_gemm(const void *x_bf16, const uint8_t *W_fp4, const uint8_t *W_sf,
                 const float *gscale, const uint32_t *Ubits, const uint32_t *Vbits,

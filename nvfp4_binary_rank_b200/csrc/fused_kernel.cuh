@@ -856,6 +856,15 @@ fused_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
+  // Programmatic dependent launch.  The next kernel on the stream may start
+  // taking SMs as soon as this one's CTAs leave them.  This kernel, in turn,
+  // waits for the kernel before it only where that kernel's results or this
+  // call's scratch are touched: every warp but the producer waits here, and the
+  // producer first requests the weight bytes of its first stages (no kernel of
+  // this library writes the weight operand).
+  if (threadIdx.x == 0) griddep_launch_dependents();
+  if (warp >= 2) griddep_wait();
+
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
     if (lane == 0) {
@@ -874,10 +883,8 @@ fused_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
                       c * kXWords, i_lo);
         }
       };
-      // the CUDA cores' inputs first, then the weight bytes (they do not depend on
-      // the activation)
-      if (p.fast)
-        for (int k = 0; k < pre; ++k) issue_x(k, k);
+      // the weight bytes of the first stages before waiting for the previous
+      // kernel, then the activation (and V rows) those stages need
       for (int k = 0; k < pre; ++k) {
         const int u = u0 + k, t = u / p.KC, c = u % p.KC;
         mbar_arrive_expect_tx(full_bar(k), stage_bytes);
@@ -886,8 +893,10 @@ fused_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
         bulk_load(smem_u32(smem + L::kSFA + k * kSfBytes),
                   p.w_sf + (static_cast<size_t>(t) * p.KC + c) * kSfBytes, kSfBytes, full_bar(k));
       }
+      griddep_wait();
+      if (p.fast)
+        for (int k = 0; k < pre; ++k) issue_x(k, k);
       if (!p.inq) {
-        griddep_wait();
         for (int k = 0; k < pre; ++k) {
           const int c = (u0 + k) % p.KC;
           tma_load_2d(smem_u32(smem + L::kB + k * BN * 128), &tmap_x, full_bar(k), c * 128, 0);

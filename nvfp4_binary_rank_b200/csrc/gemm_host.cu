@@ -198,8 +198,9 @@ int launch_gemm(const GemmArgs& a, const GemmPlan& p, const Scratch& scr, cudaSt
   fp.unit_alu = unit_alu ? 1 : 0;
   fp.bxr = bxr;
 
-  const bool pdl = !inq;
-  e = launch_for(M, tw, tx, txs, tv, fp, s, pdl);
+  // always launched for programmatic overlap with the kernel before it (the
+  // activation quantiser, or the previous call)
+  e = launch_for(M, tw, tx, txs, tv, fp, s, true);
   return e == cudaSuccess ? BILOCO_OK : BILOCO_ERR_CUDA;
 }
 
