@@ -1,0 +1,602 @@
+// Fused NVFP4 GEMM + binary-sign low-rank correction for decode batches
+// (M <= 8 activation rows) on one B200 (sm_100a).
+//
+//   y[m, n] = g * sum_k FP4(x)[m, k] FP4(R)[n, k]  +  sum_i U[n, i] z[m, i],
+//   z[m, i] = alpha_i * sum_k V[k, i] x[m, k]
+//
+// (BiLoCo README, section "Kernel": FP4 GEMM on the tensor cores, z = alpha.(V x)
+// on the CUDA cores from bit-packed V, U z expanded before the BF16 store, one
+// launch.)
+//
+// The weight is cut into units of 128 rows x 256 K elements, split over G <= #SMs
+// CTAs in contiguous ranges (stream-K), exactly like the general kernel.  What
+// differs is the order of the work after the wait on the previous kernel of the
+// stream, which is what bounds a decode call:
+//   * Weight stages are requested before that wait: no kernel of this library
+//     writes the weight operand.
+//   * The CUDA-core warps quantise the activation chunks of all the CTA's units
+//     at once into an operand cache in shared memory.  The MMAs read the
+//     activation from there, so the stage ring carries weight bytes only.
+//   * z is computed in rank slices: CTA g computes z for the ranks
+//     [g r / G, (g + 1) r / G) over the whole of K and publishes them behind one
+//     arrival counter.  This is the "side CTAs + arrival flag" schedule of the
+//     README's mode table, with every CTA taking a slice.
+//   * Only the CTA that completes a weight tile (its sole owner, or the last
+//     split-K contributor to arrive) expands U z for that tile, in parallel with
+//     summing the split-K partials.  So publishing a partial never waits for z.
+//
+// Warp roles (14 warps): warp 0 TMA producer; warp 1 TMEM allocator and MMA
+// issuer (tcgen05 kind::mxf4nvf4, block16); warps 2-5 epilogue (one weight row
+// per thread); warps 6-13 CUDA cores (activation quantisation, V side, U side).
+//
+// Every wait is bounded.  On expiry the kernel records BILOCO_ERR_TIMEOUT in
+// the status word, and the warps that share barriers leave together.
+#pragma once
+
+#include <cstdint>
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "../../include/biloco.h"
+#include "decode_params.h"
+#include "nvfp4_dev.cuh"
+#include "ptx.cuh"
+#include "sched.cuh"
+
+namespace biloco {
+namespace decode {
+
+constexpr int kWarps = 14;
+constexpr int kThreads = kWarps * 32;
+constexpr int kEpiWarp0 = 2;
+constexpr int kEpiThreads = 128;
+constexpr int kAluWarp0 = 6;
+constexpr int kAluWarps = 8;
+constexpr int kAluThreads = kAluWarps * 32;
+constexpr int kFinThreads = kEpiThreads + kAluThreads;
+constexpr int kBN = 16;                   // MMA N (activation rows, padded)
+constexpr int kRowsMax = 8;               // activation rows handled
+constexpr int kTileRows = 128;            // weight rows per tile = MMA M
+constexpr int kUnitK = 256;               // K elements per unit
+constexpr int kUnitBytesA = kTileRows * 128;
+constexpr int kSfBytes = 2048;            // 4 scale atoms of 512 B per unit
+constexpr int kStages = 6;                // weight stage ring
+constexpr int kMaxUnits = 16;             // units per CTA (operand cache entries)
+constexpr int kMaxRanks = 1024;
+constexpr int kRankGroup = 8;             // V-side ranks per pass
+constexpr int kTmemCols = 512;
+constexpr int kSfTmemBase = 256;
+constexpr uint32_t kStageTx = kUnitBytesA + kSfBytes;
+
+// named barriers (0 is __syncthreads)
+constexpr int kBarAlu = 1;
+constexpr int kBarEpi = 2;
+constexpr int kBarFin = 3;                // epilogue + CUDA cores: finisher decision
+constexpr int kBarFin2 = 4;               // epilogue + CUDA cores: correction ready
+
+template <int MC>
+struct Layout {
+  static constexpr int kA = 0;                                        // [ST][128][128 B]
+  static constexpr int kSFA = kA + kStages * kUnitBytesA;              // [ST][2 KB]
+  static constexpr int kB = kSFA + kStages * kSfBytes;                 // [NU][16][128 B]
+  static constexpr int kSFB = kB + kMaxUnits * kBN * 128;              // [NU][2 KB]
+  static constexpr int kZ = kSFB + kMaxUnits * kSfBytes;               // [MC][1024] floats
+  static constexpr int kCorr = kZ + MC * kMaxRanks * 4;                // [2][MC][128] floats
+  static constexpr int kVRed = kCorr + 2 * MC * kTileRows * 4;         // [8][MC * 8] floats
+  static constexpr int kBar = kVRed + kAluWarps * MC * kRankGroup * 4;
+  static constexpr int kNumBars = 2 * kStages + 7;
+  static constexpr int kMisc = kBar + kNumBars * 8;
+  static constexpr int kFinFlags = kMisc + 32;                         // [kMaxUnits + 1] ints
+  static constexpr int kTotal = kFinFlags + (kMaxUnits + 1) * 4;
+  static constexpr int kAlloc = kTotal + 1024;
+  static_assert(kSFA % 1024 == 0 && kB % 1024 == 0, "swizzled tiles need 1 KB alignment");
+  static_assert(kAlloc <= 232448, "shared memory budget");
+};
+
+// V-side word loop of one rank group: lane l takes element 32 w + l of every
+// word w this warp handles; acc[m][i] collects sum_k s_ik x[m][k].  Inputs that
+// the previous kernel of the stream may have written are read through L2
+// (ld.global.cg), never through a possibly stale L1 line.
+template <int MC>
+__device__ __forceinline__ void vside_group(const DecodeParams& p, int ig, int nr, int a, int lane,
+                                            float (&acc)[MC][kRankGroup]) {
+#pragma unroll
+  for (int m = 0; m < MC; ++m)
+#pragma unroll
+    for (int i = 0; i < kRankGroup; ++i) acc[m][i] = 0.0f;
+  const uint32_t lane_shift = 31u - static_cast<uint32_t>(lane);
+  const uint32_t* vrow = p.Vbits + static_cast<size_t>(ig) * p.KW;
+  constexpr int kUnroll = (MC >= 8) ? 2 : 4;
+  for (int w0 = a; w0 < p.KW; w0 += kAluWarps * kUnroll) {
+    uint32_t xs[kUnroll][MC];
+    uint32_t vw[kUnroll][kRankGroup];
+#pragma unroll
+    for (int q = 0; q < kUnroll; ++q) {
+      const int w = w0 + q * kAluWarps;
+      const bool in = w < p.KW;
+#pragma unroll
+      for (int m = 0; m < MC; ++m)
+        xs[q][m] = (in && m < p.M) ? static_cast<uint32_t>(__ldcg(p.x + static_cast<size_t>(m) * p.K +
+                                                                   static_cast<size_t>(w) * 32 + lane))
+                                   : 0u;
+#pragma unroll
+      for (int i = 0; i < kRankGroup; ++i)
+        vw[q][i] = (in && i < nr) ? __ldcg(vrow + static_cast<size_t>(i) * p.KW + w) : 0u;
+    }
+#pragma unroll
+    for (int q = 0; q < kUnroll; ++q) {
+#pragma unroll
+      for (int i = 0; i < kRankGroup; ++i) {
+        const uint32_t sgn = (vw[q][i] << lane_shift) & 0x80000000u;
+#pragma unroll
+        for (int m = 0; m < MC; ++m)
+          acc[m][i] += __uint_as_float((xs[q][m] << 16) ^ sgn);
+      }
+    }
+  }
+}
+
+template <int MC>
+__global__ void __launch_bounds__(kThreads, 1)
+decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ DecodeParams p) {
+  using L = Layout<MC>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
+  auto full_bar = [&](int s) { return smem_u32(&bars[s]); };
+  auto empty_bar = [&](int s) { return smem_u32(&bars[kStages + s]); };
+  const uint32_t actr_bar = smem_u32(&bars[2 * kStages]);
+  auto accf_bar = [&](int b) { return smem_u32(&bars[2 * kStages + 1 + b]); };
+  auto acce_bar = [&](int b) { return smem_u32(&bars[2 * kStages + 3 + b]); };
+  const uint32_t drain_bar = smem_u32(&bars[2 * kStages + 5]);
+  const uint32_t done_bar = smem_u32(&bars[2 * kStages + 6]);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+  volatile int* epi_last = reinterpret_cast<volatile int*>(smem + L::kMisc + 8);
+  volatile int* fin_flag = reinterpret_cast<volatile int*>(smem + L::kFinFlags);
+  const Ctl ctl{abort_flag, p.status};
+
+  const int g = blockIdx.x;
+  const int u0 = first_unit(g, p.G, p.U), u1 = first_unit(g + 1, p.G, p.U);
+  const int t_first = u0 / p.KC, t_last = (u1 - 1) / p.KC;
+  const int nseg = t_last - t_first + 1;
+  const int nunits = u1 - u0;
+
+  if (threadIdx.x == 0) {
+    prefetch_tmap(&tmap_w);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    mbar_init(actr_bar, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(accf_bar(b), 1);
+      mbar_init(acce_bar(b), kEpiThreads);
+    }
+    mbar_init(drain_bar, 1);
+    mbar_init(done_bar, kWarps);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_holder), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  // Programmatic dependent launch: the next kernel may take this CTA's SM as
+  // soon as it leaves.  The producer streams only the weight operand and never
+  // waits for the previous kernel; the epilogue and CUDA-core warps wait below.
+  if (threadIdx.x == 0) griddep_launch_dependents();
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      int issued = 0;
+      for (int k = 0; k < nunits; ++k) {
+        const int s = k % kStages;
+        if (k >= kStages && !mbar_wait(empty_bar(s), ((k / kStages) - 1) & 1, abort_flag)) {
+          fail(ctl);
+          break;
+        }
+        const int u = u0 + k, t = u / p.KC, c = u % p.KC;
+        mbar_arrive_expect_tx(full_bar(s), kStageTx);
+        tma_load_2d(smem_u32(smem + L::kA + s * kUnitBytesA), &tmap_w, full_bar(s), c * 128,
+                    t * kTileRows);
+        bulk_load(smem_u32(smem + L::kSFA + s * kSfBytes),
+                  p.w_sf + (static_cast<size_t>(t) * p.KC + c) * kSfBytes, kSfBytes, full_bar(s));
+        ++issued;
+      }
+      // never leave the CTA with copies in flight
+      for (int k = max(0, issued - kStages); k < issued; ++k) {
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait(full_bar(k % kStages), (k / kStages) & 1)) {
+          if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            record_error(p.status, kDevErrTimeout);
+            break;
+          }
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = (1u << 7) | (1u << 10) | (static_cast<uint32_t>(kBN >> 3) << 17) |
+                             (static_cast<uint32_t>(kTileRows >> 4) << 24);
+      bool ok = mbar_wait(actr_bar, 0, abort_flag);
+      if (!ok) fail(ctl);
+      tc_fence_after();
+      int k = 0;
+      for (int seg = 0; seg < nseg && ok; ++seg) {
+        const int t = t_first + seg;
+        const int ua = max(u0, t * p.KC), ub = min(u1, (t + 1) * p.KC);
+        const int b = seg & 1;
+        if (seg >= 2 && !mbar_wait(acce_bar(b), ((seg >> 1) - 1) & 1, abort_flag)) {
+          fail(ctl);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + static_cast<uint32_t>(b * kBN);
+        for (int u = ua; u < ub; ++u, ++k) {
+          const int s = k % kStages;
+          if (!mbar_wait(full_bar(s), (k / kStages) & 1, abort_flag)) {
+            fail(ctl);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sfa_t = tmem + kSfTmemBase + s * 32, sfb_t = sfa_t + 16;
+          const uint32_t sfa_s = smem_u32(smem + L::kSFA + s * kSfBytes);
+          const uint32_t sfb_s = smem_u32(smem + L::kSFB + k * kSfBytes);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            tc_cp_32x128b_warpx4(sfa_t + 4 * j, smem_desc(sfa_s + 512 * j, 0, 128, 0));
+            tc_cp_32x128b_warpx4(sfb_t + 4 * j, smem_desc(sfb_s + 512 * j, 0, 128, 0));
+          }
+          const uint64_t adesc = smem_desc(smem_u32(smem + L::kA + s * kUnitBytesA), 16, 1024, 2);
+          const uint64_t bdesc = smem_desc(smem_u32(smem + L::kB + k * kBN * 128), 16, 1024, 2);
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            tc_mma_nvf4(d_tmem, adesc + 2 * j, bdesc + 2 * j, idesc, sfa_t + 4 * j, sfb_t + 4 * j,
+                        (u > ua || j > 0) ? 1u : 0u);
+          tc_commit(empty_bar(s));
+        }
+        if (ok) tc_commit(accf_bar(b));
+      }
+      // every MMA and scale copy issued so far must finish before TMEM is freed
+      tc_commit(drain_bar);
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(drain_bar, 0)) {
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+          record_error(p.status, kDevErrTimeout);
+          break;
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + 4) {
+    // ---------------------------------------------------------------- epilogue
+    griddep_wait();
+    const int q = warp & 3;                            // TMEM lane quarter of this warp
+    const int row = q * 32 + lane;                     // weight row within the tile
+    const int etid = threadIdx.x - kEpiWarp0 * 32;
+    const float gs = __ldcg(p.gscale);
+    constexpr int kHB = (MC <= 2) ? 16 : (MC <= 4 ? 8 : 4);   // partials loaded per batch
+    bool ok = true;
+    for (int seg = 0; seg < nseg; ++seg) {
+      const int t = t_first + seg;
+      const int b = seg & 1;
+      const int hf = owner_cta(static_cast<uint32_t>(t * p.KC), p.G, p.U);
+      const int hl = owner_cta(static_cast<uint32_t>((t + 1) * p.KC - 1), p.G, p.U);
+      const bool sole = hf == hl;
+      const int which = (t == t_first) ? 0 : 1;
+      float v[MC];
+      bool fin = false;
+      if (ok) ok = group_wait(accf_bar(b), (seg >> 1) & 1, kBarEpi, kEpiThreads, ctl);
+      if (ok) {
+        tc_fence_after();
+        uint32_t raw[16];
+        tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(b * kBN), raw);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < MC; ++j) v[j] = __fmul_rn(gs, __uint_as_float(raw[j]));
+        tc_fence_before();
+        mbar_arrive(acce_bar(b));
+        if (sole) {
+          fin = true;
+        } else {
+          // publish this partial; the last contributor of the tile completes it
+          float* my_slot = p.slots + static_cast<size_t>(2 * g + which) * kRowsMax * kTileRows;
+#pragma unroll
+          for (int j = 0; j < MC; ++j)
+            if (j < p.M) my_slot[j * kTileRows + row] = v[j];
+          __threadfence();
+          named_barrier(kBarEpi, kEpiThreads);
+          if (etid == 0) {
+            const uint32_t nh = static_cast<uint32_t>(hl - hf + 1);
+            const uint32_t old = atomicAdd(p.tickets + t, 1u);
+            const bool last = old == nh - 1;
+            if (last) atomicExch(p.tickets + t, 0u);
+            __threadfence();
+            *epi_last = last ? 1 : 0;
+          }
+          named_barrier(kBarEpi, kEpiThreads);
+          fin = *epi_last != 0;
+          named_barrier(kBarEpi, kEpiThreads);
+        }
+      }
+      if (p.r > 0) {
+        // tell the CUDA-core warps whether this tile's correction is needed here
+        if (etid == 0) fin_flag[seg] = fin ? 1 : 0;
+        if (named_barrier_or(kBarFin, kFinThreads, !ok)) {
+          if (ok) fail(ctl);
+          ok = false;
+        }
+      }
+      if (!ok) break;
+      if (!fin) continue;
+      float acc[MC];
+      if (sole) {
+#pragma unroll
+        for (int j = 0; j < MC; ++j) acc[j] = v[j];
+      } else {
+        // every contributor's partial, summed in contributor order
+#pragma unroll
+        for (int j = 0; j < MC; ++j) acc[j] = 0.0f;
+        const int wh_first = (t == first_unit(hf, p.G, p.U) / p.KC) ? 0 : 1;
+        for (int h0 = hf; h0 <= hl; h0 += kHB) {
+          float part[kHB][MC];
+#pragma unroll
+          for (int e = 0; e < kHB; ++e) {
+            const int h = h0 + e;
+            const float* sl = p.slots + static_cast<size_t>(2 * h + ((h == hf) ? wh_first : 0)) *
+                                            kRowsMax * kTileRows;
+#pragma unroll
+            for (int j = 0; j < MC; ++j)
+              part[e][j] = (h <= hl && h != g && j < p.M) ? __ldcg(sl + j * kTileRows + row) : 0.0f;
+          }
+#pragma unroll
+          for (int e = 0; e < kHB; ++e) {
+            const int h = h0 + e;
+            if (h <= hl) {
+#pragma unroll
+              for (int j = 0; j < MC; ++j) acc[j] += (h == g) ? v[j] : part[e][j];
+            }
+          }
+        }
+      }
+      if (p.r > 0) {
+        if (named_barrier_or(kBarFin2, kFinThreads, !ok)) {
+          ok = false;
+          break;
+        }
+        const float* corr = reinterpret_cast<const float*>(smem + L::kCorr);
+#pragma unroll
+        for (int j = 0; j < MC; ++j)
+          acc[j] = (acc[j] + corr[j * kTileRows + row]) + corr[(MC + j) * kTileRows + row];
+      }
+      uint16_t* yb = p.y + static_cast<size_t>(t) * kTileRows + row;
+#pragma unroll
+      for (int j = 0; j < MC; ++j)
+        if (j < p.M) yb[static_cast<size_t>(j) * p.N] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[j]));
+    }
+  } else {
+    // ---------------------------------------------------------------- CUDA cores
+    const int tid = threadIdx.x - kAluWarp0 * 32;      // 0..255
+    const int a = warp - kAluWarp0;                     // warp slot 0..7
+    // The operand cache starts zero: rows >= M and blocks past K stay zero.
+    for (int idx = tid; idx < nunits * 256; idx += kAluThreads) {
+      const int k = idx >> 8, o = idx & 255;
+      uint4* dst = (o < 128) ? reinterpret_cast<uint4*>(smem + L::kB + k * kBN * 128) + o
+                             : reinterpret_cast<uint4*>(smem + L::kSFB + k * kSfBytes) + (o - 128);
+      *dst = make_uint4(0u, 0u, 0u, 0u);
+    }
+    const int i0 = static_cast<int>(static_cast<uint32_t>(g) * static_cast<uint32_t>(p.r) /
+                                    static_cast<uint32_t>(p.G));
+    const int i1 = static_cast<int>(static_cast<uint32_t>(g + 1) * static_cast<uint32_t>(p.r) /
+                                    static_cast<uint32_t>(p.G));
+    if (p.r > 0) {
+      // warm L2 with the sign words this CTA reads later (a hint only)
+      const char* vb = reinterpret_cast<const char*>(p.Vbits + static_cast<size_t>(i0) * p.KW);
+      const int vlines = ((i1 - i0) * p.KW * 4 + 127) / 128;
+      for (int l = tid; l < vlines; l += kAluThreads) prefetch_l2(vb + static_cast<size_t>(l) * 128);
+      const int ulines = (kTileRows * p.RW * 4 + 127) / 128;
+      for (int seg = 0; seg < nseg; ++seg) {
+        const char* ub = reinterpret_cast<const char*>(p.Ubits + static_cast<size_t>(t_first + seg) *
+                                                                     kTileRows * p.RW);
+        for (int l = tid; l < ulines; l += kAluThreads) prefetch_l2(ub + static_cast<size_t>(l) * 128);
+      }
+    }
+    griddep_wait();
+    named_barrier(kBarAlu, kAluThreads);               // cache zeroed before any code lands
+
+    // ---- 1. quantise the activation chunks of every unit of this CTA
+    {
+      constexpr int kQB = 4;                            // blocks per thread per round
+      const int per_unit = p.M * 16;
+      const int items = nunits * per_unit;
+      for (int base = 0; base < items; base += kAluThreads * kQB) {
+        uint4 lo[kQB], hi[kQB];
+#pragma unroll
+        for (int e = 0; e < kQB; ++e) {
+          const int idx = base + e * kAluThreads + tid;
+          lo[e] = hi[e] = make_uint4(0u, 0u, 0u, 0u);
+          if (idx < items) {
+            const int k = idx / per_unit, rem = idx - k * per_unit, m = rem >> 4, blk = rem & 15;
+            const int kk = ((u0 + k) % p.KC) * kUnitK + blk * 16;
+            if (kk < p.K) {
+              const uint4* src = reinterpret_cast<const uint4*>(p.x + static_cast<size_t>(m) * p.K + kk);
+              lo[e] = __ldcg(src);
+              hi[e] = __ldcg(src + 1);
+            }
+          }
+        }
+#pragma unroll
+        for (int e = 0; e < kQB; ++e) {
+          const int idx = base + e * kAluThreads + tid;
+          if (idx < items) {
+            const int k = idx / per_unit, rem = idx - k * per_unit, m = rem >> 4, blk = rem & 15;
+            const int kk = ((u0 + k) % p.KC) * kUnitK + blk * 16;
+            if (kk < p.K) {
+              float v[16];
+              bf16x16_to_f32(lo[e], hi[e], v);
+              uint2 codes;
+              const uint32_t s = quant_act_block(v, codes);
+              const int j = blk * 8;
+              *reinterpret_cast<uint2*>(smem + L::kB + k * kBN * 128 + m * 128 +
+                                        ((((j >> 4) ^ (m & 7)) << 4) | (j & 15))) = codes;
+              smem[L::kSFB + k * kSfBytes + (blk >> 2) * 512 + (m & 31) * 16 + ((m >> 5) & 3) * 4 +
+                   (blk & 3)] = static_cast<uint8_t>(s);
+            }
+          }
+        }
+      }
+      fence_proxy_async_smem();
+      named_barrier(kBarAlu, kAluThreads);
+      if (tid == 0) mbar_arrive(actr_bar);
+    }
+
+    if (p.r > 0) {
+      // ---- 2. V side: z for this CTA's rank slice over the whole of K
+      constexpr int kV = MC * kRankGroup;
+      float* vred = reinterpret_cast<float*>(smem + L::kVRed);
+      for (int ig = i0; ig < i1; ig += kRankGroup) {
+        const int nr = min(kRankGroup, i1 - ig);
+        float acc[MC][kRankGroup];
+        vside_group<MC>(p, ig, nr, a, lane, acc);
+        float flat[kV];
+#pragma unroll
+        for (int m = 0; m < MC; ++m)
+#pragma unroll
+          for (int i = 0; i < kRankGroup; ++i) flat[m * kRankGroup + i] = acc[m][i];
+        warp_reduce_scatter<kV>(flat, lane);
+        if constexpr (kV >= 32) {
+#pragma unroll
+          for (int j = 0; j < kV / 32; ++j) vred[a * kV + reduce_out_index<kV>(lane, j)] = flat[j];
+        } else {
+          if ((lane & (32 / kV - 1)) == 0) vred[a * kV + reduce_out_index<kV>(lane, 0)] = flat[0];
+        }
+        named_barrier(kBarAlu, kAluThreads);
+        if (tid < p.M * nr) {
+          const int m = tid / nr, i = tid - m * nr;
+          float sum = 0.0f;
+#pragma unroll
+          for (int w = 0; w < kAluWarps; ++w) sum += vred[w * kV + m * kRankGroup + i];
+          p.z[static_cast<size_t>(m) * p.rpad + ig + i] = __fmul_rn(__ldcg(p.alpha + ig + i), sum);
+        }
+        named_barrier(kBarAlu, kAluThreads);
+      }
+      __threadfence();
+      named_barrier(kBarAlu, kAluThreads);
+      if (tid == 0) atomicAdd(p.z_ready, 1u);
+
+      // ---- 3. U side of every tile this CTA completes
+      float* zs = reinterpret_cast<float*>(smem + L::kZ);
+      float* corr = reinterpret_cast<float*>(smem + L::kCorr);
+      bool ok = true, staged = false;
+      for (int seg = 0; seg < nseg; ++seg) {
+        if (named_barrier_or(kBarFin, kFinThreads, !ok)) {
+          ok = false;
+          break;
+        }
+        if (!fin_flag[seg]) continue;
+        const int t = t_first + seg;
+        if (!staged) {
+          bool okw = true;
+          if (tid == 0) okw = spin_until_geq(p.z_ready, static_cast<uint32_t>(p.G), ctl);
+          if (named_barrier_or(kBarAlu, kAluThreads, !okw)) {
+            fail(ctl);
+            ok = false;
+          } else {
+            const int span = 32 * p.RW;
+            for (int idx = tid; idx < p.M * span; idx += kAluThreads) {
+              const int m = idx / span, i = idx - m * span;
+              zs[m * kMaxRanks + i] = (i < p.r) ? __ldcg(p.z + static_cast<size_t>(m) * p.rpad + i) : 0.0f;
+            }
+            named_barrier(kBarAlu, kAluThreads);
+            staged = true;
+          }
+        }
+        if (ok) {
+          const int row = tid & (kTileRows - 1), half = tid >> 7;
+          const int wsplit = (p.RW + 1) >> 1;
+          const int wa = half ? wsplit : 0, wb = half ? p.RW : wsplit;
+          const uint32_t* ur = p.Ubits + (static_cast<size_t>(t) * kTileRows + row) * p.RW;
+          uint32_t uw[16];
+#pragma unroll
+          for (int w = 0; w < 16; ++w) uw[w] = (wa + w < wb) ? __ldcg(ur + wa + w) : 0u;
+          float acc[MC];
+#pragma unroll
+          for (int m = 0; m < MC; ++m) acc[m] = 0.0f;
+          for (int w = 0; w < wb - wa; ++w) {
+            uint32_t word = 0;
+#pragma unroll
+            for (int e = 0; e < 16; ++e) word = (e == w) ? uw[e] : word;
+            const float* zw = zs + (wa + w) * 32;
+#pragma unroll
+            for (int j4 = 0; j4 < 8; ++j4) {
+#pragma unroll
+              for (int m = 0; m < MC; ++m) {
+                if (m < p.M) {
+                  const float4 z4 = *reinterpret_cast<const float4*>(zw + m * kMaxRanks + 4 * j4);
+                  const float zz[4] = {z4.x, z4.y, z4.z, z4.w};
+#pragma unroll
+                  for (int jj = 0; jj < 4; ++jj) {
+                    const uint32_t sgn = (word << (31 - (4 * j4 + jj))) & 0x80000000u;
+                    acc[m] += __uint_as_float(__float_as_uint(zz[jj]) ^ sgn);
+                  }
+                }
+              }
+            }
+          }
+#pragma unroll
+          for (int m = 0; m < MC; ++m) corr[(half * MC + m) * kTileRows + row] = acc[m];
+        }
+        if (named_barrier_or(kBarFin2, kFinThreads, !ok)) {
+          ok = false;
+          break;
+        }
+      }
+      // this CTA is done with z_ready; the last CTA to get here resets both counters
+      if (tid == 0 && ok) {
+        const uint32_t old = atomicAdd(p.z_seen, 1u);
+        if (old == static_cast<uint32_t>(p.G - 1)) {
+          atomicExch(p.z_ready, 0u);
+          atomicExch(p.z_seen, 0u);
+        }
+      }
+    }
+  }
+
+  // ------------------------------------------------------------------ teardown
+  // Each warp reports once it no longer touches TMEM or shared memory; warp 1
+  // frees TMEM after all of them (bounded wait).
+  __syncwarp();
+  tc_fence_before();
+  if (lane == 0) mbar_arrive(done_bar);
+  if (warp == 1) {
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(done_bar, 0)) {
+      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        record_error(p.status, kDevErrTimeout);
+        break;
+      }
+    }
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace decode
+}  // namespace biloco

@@ -1,0 +1,27 @@
+// Parameters of the decode-batch kernel (M <= 8), shared by its host launcher
+// and the kernel.
+#pragma once
+
+#include <cstdint>
+
+namespace biloco {
+
+struct DecodeParams {
+  const uint8_t* w_sf;     // weight scales, tile layout
+  const float* gscale;     // weight tensor scale g
+  const uint32_t* Ubits;   // [N][RW]
+  const uint32_t* Vbits;   // [r][KW]
+  const float* alpha;      // [r]
+  const uint16_t* x;       // [M][K] BF16
+  uint16_t* y;             // [M][N] BF16
+  float* z;                // [M][rpad] scratch: z = alpha . (V^T x)
+  float* slots;            // [2 G][8][128] scratch: split-K partials
+  uint32_t* z_ready;       // CTAs that published their z slice
+  uint32_t* z_seen;        // CTAs done with z_ready (the last one resets both)
+  uint32_t* tickets;       // [T] split-K arrivals per weight tile
+  int* status;             // first device-side error
+  int M, N, K, r;
+  int KC, T, U, G, KW, RW, rpad;
+};
+
+}  // namespace biloco

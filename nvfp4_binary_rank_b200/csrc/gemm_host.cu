@@ -8,6 +8,7 @@
 #include <cuda_runtime.h>
 
 #include "../../include/biloco.h"
+#include "decode_launch.h"
 #include "fused_launch.h"
 #include "fused_params.h"
 #include "internal.h"
@@ -119,7 +120,20 @@ GemmPlan plan_gemm(const GemmArgs& a) {
   const int ranks_per_tile = (r + p.T - 1) / p.T;
   p.fast = p.unit_alu && p.BN <= 32 && K % 128 == 0 && (!p.shared_z || ranks_per_tile <= kVStageRanks);
 
+  // decode batches take the decode kernel when its operand cache holds every
+  // unit of a CTA (ceil(U / G) units)
+  p.decode = M <= kDecodeMaxRows && (r == 0 || p.shared_z) && (p.U + p.G - 1) / p.G <= kDecodeMaxUnits;
+
   ScratchNeed& need = p.need;
+  if (p.decode) {
+    need.act_fp4 = 16;
+    need.act_sf = 16;
+    need.zpart = 16;
+    need.zfin = r ? static_cast<size_t>(M) * p.rpad * 4 : 16;
+    need.slots = static_cast<size_t>(2 * p.G) * kDecodeMaxRows * kTileRows * 4;
+    need.counter_words = 2 + 2 * static_cast<size_t>(p.T);
+    return p;
+  }
   need.act_fp4 = p.inq ? 16 : static_cast<size_t>(M) * K / 2;
   need.act_sf = p.inq ? 16 : static_cast<size_t>(p.KC) * kSfBytes;
   need.zpart = r ? static_cast<size_t>(p.KC) * M * p.rpad * 4 : 16;
@@ -144,6 +158,34 @@ int launch_gemm(const GemmArgs& a, const GemmPlan& p, const Scratch& scr, cudaSt
   const Scratch* sc = &scr;
 
   cudaError_t e = cudaSuccess;
+  if (p.decode) {
+    CUtensorMap tw;
+    if (!make_tmap(&tw, a.W_fp4, static_cast<uint64_t>(K) / 2, static_cast<uint64_t>(N), kTileRows))
+      return BILOCO_ERR_CUDA;
+    DecodeParams dp = {};
+    dp.w_sf = a.W_sf;
+    dp.gscale = a.gscale;
+    dp.Ubits = a.Ubits;
+    dp.Vbits = a.Vbits;
+    dp.alpha = a.alpha;
+    dp.x = a.x;
+    dp.y = a.y;
+    dp.z = sc->zfin;
+    dp.slots = sc->slots;
+    dp.z_ready = sc->counters;
+    dp.z_seen = sc->counters + 1;
+    dp.tickets = sc->counters + 2;
+    dp.status = sc->status;
+    dp.M = M; dp.N = N; dp.K = K; dp.r = r;
+    dp.KC = KC; dp.T = T; dp.U = U; dp.G = G; dp.KW = KW;
+    dp.RW = (r + 31) / 32;
+    dp.rpad = rpad;
+    if (M <= 1) e = launch_decode_1(tw, dp, s);
+    else if (M <= 2) e = launch_decode_2(tw, dp, s);
+    else if (M <= 4) e = launch_decode_4(tw, dp, s);
+    else e = launch_decode_8(tw, dp, s);
+    return e == cudaSuccess ? BILOCO_OK : BILOCO_ERR_CUDA;
+  }
   if (!inq) {
     e = launch_prep_act(a.x, M, K, sc->act_fp4, sc->act_sf, s);
     if (e != cudaSuccess) return BILOCO_ERR_CUDA;

@@ -67,6 +67,7 @@ int check_gemm_args(const void* x_bf16, const uint8_t* W_fp4, const uint8_t* W_s
 struct GemmPlan {
   int KC, T, U, G, KW, rpad, BN, bxr;
   bool inq, zdirect, shared_z, unit_alu, fast;
+  bool decode;   // the decode-batch kernel (M <= 8, shared z) runs the call
   ScratchNeed need;
 };
 GemmPlan plan_gemm(const GemmArgs& a);
