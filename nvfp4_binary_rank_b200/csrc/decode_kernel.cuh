@@ -66,8 +66,11 @@ constexpr int kStages = 6;                // weight stage ring
 constexpr int kMaxUnits = 16;             // units per CTA (operand cache entries)
 constexpr int kMaxRanks = 1024;
 constexpr int kRankGroup = 8;             // V-side ranks per pass
+// TMEM columns: accumulators [0, 32); activation scales per unit [32, 288);
+// weight scales per stage [288, 384)
 constexpr int kTmemCols = 512;
-constexpr int kSfTmemBase = 256;
+constexpr int kSfbTmemBase = 32;
+constexpr int kSfaTmemBase = kSfbTmemBase + 16 * 16;
 constexpr uint32_t kStageTx = kUnitBytesA + kSfBytes;
 
 // named barriers (0 is __syncthreads)
@@ -81,8 +84,8 @@ struct Layout {
   static constexpr int kA = 0;                                        // [ST][128][128 B]
   static constexpr int kSFA = kA + kStages * kUnitBytesA;              // [ST][2 KB]
   static constexpr int kB = kSFA + kStages * kSfBytes;                 // [NU][16][128 B]
-  static constexpr int kSFB = kB + kMaxUnits * kBN * 128;              // [NU][2 KB]
-  static constexpr int kZ = kSFB + kMaxUnits * kSfBytes;               // [MC][1024] floats
+  static constexpr int kSFB = kB + kMaxUnits * kBN * 128;              // [NU][4 steps][32 rows] u32
+  static constexpr int kZ = kSFB + kMaxUnits * 512;                    // [MC][1024] floats
   static constexpr int kCorr = kZ + MC * kMaxRanks * 4;                // [2][MC][128] floats
   static constexpr int kVRed = kCorr + 2 * MC * kTileRows * 4;         // [8][MC * 8] floats
   static constexpr int kBar = kVRed + kAluWarps * MC * kRankGroup * 4;
@@ -199,21 +202,25 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
+    // (one thread; the unit's tile and chunk advance incrementally: no divisions)
     if (lane == 0) {
       int issued = 0;
+      int t = u0 / p.KC, c = u0 - t * p.KC;
+      int s = 0;
+      uint32_t ph = 0;                                   // parity of the stage's current use
+      const uint8_t* sf = p.w_sf + static_cast<size_t>(u0) * kSfBytes;
       for (int k = 0; k < nunits; ++k) {
-        const int s = k % kStages;
-        if (k >= kStages && !mbar_wait(empty_bar(s), ((k / kStages) - 1) & 1, abort_flag)) {
+        if (k >= kStages && !mbar_wait(empty_bar(s), ph ^ 1u, abort_flag)) {
           fail(ctl);
           break;
         }
-        const int u = u0 + k, t = u / p.KC, c = u % p.KC;
         mbar_arrive_expect_tx(full_bar(s), kStageTx);
-        tma_load_2d(smem_u32(smem + L::kA + s * kUnitBytesA), &tmap_w, full_bar(s), c * 128,
-                    t * kTileRows);
-        bulk_load(smem_u32(smem + L::kSFA + s * kSfBytes),
-                  p.w_sf + (static_cast<size_t>(t) * p.KC + c) * kSfBytes, kSfBytes, full_bar(s));
+        tma_load_2d(smem_u32(smem + L::kA + s * kUnitBytesA), &tmap_w, full_bar(s), c * 128, t * kTileRows);
+        bulk_load(smem_u32(smem + L::kSFA + s * kSfBytes), sf, kSfBytes, full_bar(s));
         ++issued;
+        sf += kSfBytes;
+        if (++c == p.KC) { c = 0; ++t; }
+        if (++s == kStages) { s = 0; ph ^= 1u; }
       }
       // never leave the CTA with copies in flight
       for (int k = max(0, issued - kStages); k < issued; ++k) {
@@ -229,13 +236,41 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
     __syncwarp();
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
+    // One thread issues every tcgen05 instruction; descriptors are built once and
+    // offset per unit (the 14-bit address field counts 16-byte units and never
+    // carries here).
     if (lane == 0) {
       const uint32_t idesc = (1u << 7) | (1u << 10) | (static_cast<uint32_t>(kBN >> 3) << 17) |
                              (static_cast<uint32_t>(kTileRows >> 4) << 24);
-      bool ok = mbar_wait(actr_bar, 0, abort_flag);
-      if (!ok) fail(ctl);
+      const uint64_t a_desc0 = smem_desc(smem_u32(smem + L::kA), 16, 1024, 2);
+      const uint64_t b_desc0 = smem_desc(smem_u32(smem + L::kB), 16, 1024, 2);
+      const uint64_t sfa_desc0 = smem_desc(smem_u32(smem + L::kSFA), 0, 128, 0);
+      constexpr uint64_t kAtom = 512 >> 4, kUnitSf = kSfBytes >> 4;
+      constexpr uint64_t kUnitA = kUnitBytesA >> 4, kUnitB = (kBN * 128) >> 4;
+      // weight scales of the stages already requested go to TMEM while the
+      // activation is still being quantised
+      const int pre = min(nunits, kStages);
+      bool ok = true;
+      for (int j = 0; j < pre && ok; ++j) {
+        if (!mbar_wait(full_bar(j), 0, abort_flag)) {
+          fail(ctl);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint64_t sfa_d = sfa_desc0 + static_cast<uint64_t>(j) * kUnitSf;
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          tc_cp_32x128b_warpx4(tmem + kSfaTmemBase + j * 16 + 4 * q, sfa_d + kAtom * q);
+      }
+      // the activation codes (shared memory) and scales (TMEM) are in place
+      if (ok && !mbar_wait(actr_bar, 0, abort_flag)) {
+        fail(ctl);
+        ok = false;
+      }
       tc_fence_after();
-      int k = 0;
+      int k = 0, s = 0;
+      uint32_t ph = 0;
       for (int seg = 0; seg < nseg && ok; ++seg) {
         const int t = t_first + seg;
         const int ua = max(u0, t * p.KC), ub = min(u1, (t + 1) * p.KC);
@@ -248,28 +283,27 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
         tc_fence_after();
         const uint32_t d_tmem = tmem + static_cast<uint32_t>(b * kBN);
         for (int u = ua; u < ub; ++u, ++k) {
-          const int s = k % kStages;
-          if (!mbar_wait(full_bar(s), (k / kStages) & 1, abort_flag)) {
-            fail(ctl);
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t sfa_t = tmem + kSfTmemBase + s * 32, sfb_t = sfa_t + 16;
-          const uint32_t sfa_s = smem_u32(smem + L::kSFA + s * kSfBytes);
-          const uint32_t sfb_s = smem_u32(smem + L::kSFB + k * kSfBytes);
+          const uint32_t sfa_t = tmem + kSfaTmemBase + s * 16;
+          const uint32_t sfb_t = tmem + kSfbTmemBase + k * 16;
+          if (k >= pre) {
+            if (!mbar_wait(full_bar(s), ph, abort_flag)) {
+              fail(ctl);
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint64_t sfa_d = sfa_desc0 + static_cast<uint64_t>(s) * kUnitSf;
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            tc_cp_32x128b_warpx4(sfa_t + 4 * j, smem_desc(sfa_s + 512 * j, 0, 128, 0));
-            tc_cp_32x128b_warpx4(sfb_t + 4 * j, smem_desc(sfb_s + 512 * j, 0, 128, 0));
+            for (int q = 0; q < 4; ++q) tc_cp_32x128b_warpx4(sfa_t + 4 * q, sfa_d + kAtom * q);
           }
-          const uint64_t adesc = smem_desc(smem_u32(smem + L::kA + s * kUnitBytesA), 16, 1024, 2);
-          const uint64_t bdesc = smem_desc(smem_u32(smem + L::kB + k * kBN * 128), 16, 1024, 2);
+          const uint64_t a_d = a_desc0 + static_cast<uint64_t>(s) * kUnitA;
+          const uint64_t b_d = b_desc0 + static_cast<uint64_t>(k) * kUnitB;
 #pragma unroll
           for (int j = 0; j < 4; ++j)
-            tc_mma_nvf4(d_tmem, adesc + 2 * j, bdesc + 2 * j, idesc, sfa_t + 4 * j, sfb_t + 4 * j,
+            tc_mma_nvf4(d_tmem, a_d + 2 * j, b_d + 2 * j, idesc, sfa_t + 4 * j, sfb_t + 4 * j,
                         (u > ua || j > 0) ? 1u : 0u);
           tc_commit(empty_bar(s));
+          if (++s == kStages) { s = 0; ph ^= 1u; }
         }
         if (ok) tc_commit(accf_bar(b));
       }
@@ -320,14 +354,13 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
 #pragma unroll
           for (int j = 0; j < MC; ++j)
             if (j < p.M) my_slot[j * kTileRows + row] = v[j];
-          __threadfence();
           named_barrier(kBarEpi, kEpiThreads);
           if (etid == 0) {
+            // release: this CTA's partial; acquire: every earlier contributor's
             const uint32_t nh = static_cast<uint32_t>(hl - hf + 1);
-            const uint32_t old = atomicAdd(p.tickets + t, 1u);
+            const uint32_t old = atom_add_acq_rel_gpu(p.tickets + t, 1u);
             const bool last = old == nh - 1;
             if (last) atomicExch(p.tickets + t, 0u);
-            __threadfence();
             *epi_last = last ? 1 : 0;
           }
           named_barrier(kBarEpi, kEpiThreads);
@@ -395,10 +428,10 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
     const int tid = threadIdx.x - kAluWarp0 * 32;      // 0..255
     const int a = warp - kAluWarp0;                     // warp slot 0..7
     // The operand cache starts zero: rows >= M and blocks past K stay zero.
-    for (int idx = tid; idx < nunits * 256; idx += kAluThreads) {
-      const int k = idx >> 8, o = idx & 255;
+    for (int idx = tid; idx < nunits * 160; idx += kAluThreads) {
+      const int k = idx / 160, o = idx - k * 160;
       uint4* dst = (o < 128) ? reinterpret_cast<uint4*>(smem + L::kB + k * kBN * 128) + o
-                             : reinterpret_cast<uint4*>(smem + L::kSFB + k * kSfBytes) + (o - 128);
+                             : reinterpret_cast<uint4*>(smem + L::kSFB + k * 512) + (o - 128);
       *dst = make_uint4(0u, 0u, 0u, 0u);
     }
     const int i0 = static_cast<int>(static_cast<uint32_t>(g) * static_cast<uint32_t>(p.r) /
@@ -455,13 +488,33 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
               const int j = blk * 8;
               *reinterpret_cast<uint2*>(smem + L::kB + k * kBN * 128 + m * 128 +
                                         ((((j >> 4) ^ (m & 7)) << 4) | (j & 15))) = codes;
-              smem[L::kSFB + k * kSfBytes + (blk >> 2) * 512 + (m & 31) * 16 + ((m >> 5) & 3) * 4 +
-                   (blk & 3)] = static_cast<uint8_t>(s);
+              smem[L::kSFB + k * 512 + (blk >> 2) * 128 + m * 4 + (blk & 3)] = static_cast<uint8_t>(s);
             }
           }
         }
       }
       fence_proxy_async_smem();
+      named_barrier(kBarAlu, kAluThreads);
+      // Activation scales to TMEM, in the layout a 32x128b.warpx4 copy of scale
+      // atoms would give: lane i of every lane quarter holds, in column 16 k + 4 j,
+      // the four block scales of row i for K step j of unit k (rows >= 16 and the
+      // other three columns of a step are zero).  Warps 6..9 cover the four lane
+      // quarters.
+      if (a < 4) {
+        const uint32_t quarter = static_cast<uint32_t>(warp & 3);
+        for (int k = 0; k < nunits; ++k) {
+          const uint32_t* sfb = reinterpret_cast<const uint32_t*>(smem + L::kSFB + k * 512) + lane;
+          uint32_t v[16];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            v[4 * j] = sfb[j * 32];
+            v[4 * j + 1] = v[4 * j + 2] = v[4 * j + 3] = 0u;
+          }
+          tmem_st16(tmem + ((quarter * 32) << 16) + kSfbTmemBase + k * 16, v);
+        }
+        tmem_wait_st();
+      }
+      tc_fence_before();
       named_barrier(kBarAlu, kAluThreads);
       if (tid == 0) mbar_arrive(actr_bar);
     }
@@ -496,9 +549,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
         }
         named_barrier(kBarAlu, kAluThreads);
       }
-      __threadfence();
       named_barrier(kBarAlu, kAluThreads);
-      if (tid == 0) atomicAdd(p.z_ready, 1u);
+      if (tid == 0) red_add_release_gpu(p.z_ready, 1u);   // covers the slice the CTA wrote
 
       // ---- 3. U side of every tile this CTA completes
       float* zs = reinterpret_cast<float*>(smem + L::kZ);
