@@ -73,11 +73,13 @@ def kernel_source_digest() -> str:
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(workload: str):
-    """DRAM bytes (read + write) per launch of the fused kernel from the committed
-    ncu summary of this workload, or None when there is none or the kernel
-    sources changed since it was captured."""
-    path = os.path.join(ROOT, "profiles", f"fused_kernel_{workload}.md")
+def ncu_traffic(workload: str, M: int):
+    """DRAM bytes (read + write) per launch of the GEMM kernel that serves this
+    workload (decode_kernel for M <= 8, fused_kernel above), from the committed
+    ncu summary, or None when there is none or the kernel sources changed since
+    it was captured."""
+    kernel = "decode_kernel" if M <= 8 else "fused_kernel"
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
     try:
         fields = {}
         with open(path) as f:
@@ -267,10 +269,14 @@ def time_e2e(prob, steps, stream):
 
 
 class DistCtx:
-    def __init__(self):
+    """One process per GPU (torchrun env vars).  NCCL on the GPU machine; `gloo`
+    serves the CPU tests of the rank logic."""
+
+    def __init__(self, backend: str = "nccl"):
         self.world = int(os.environ.get("WORLD_SIZE", "1"))
         self.rank = int(os.environ.get("RANK", "0"))
         self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.backend = backend
         self.pg = False
 
     def init(self):
@@ -279,8 +285,10 @@ class DistCtx:
         import torch.distributed as dist
         if self.world > 1:
             os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
-            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                    device_id=torch.device("cuda", self.local))
+            kw = {"timeout": datetime.timedelta(seconds=120)}
+            if self.backend == "nccl":
+                kw["device_id"] = torch.device("cuda", self.local)
+            dist.init_process_group(self.backend, **kw)
             self.pg = True
 
     def barrier(self):
@@ -293,7 +301,8 @@ class DistCtx:
             return v
         import torch
         import torch.distributed as dist
-        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        dev = "cuda" if self.backend == "nccl" else "cpu"
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         return float(t.item())
 
@@ -301,6 +310,14 @@ class DistCtx:
         if self.pg:
             import torch.distributed as dist
             dist.destroy_process_group()
+
+
+def step_metrics(bytes_per_step: int, ms_max: float, steps: int, world: int):
+    """(us per step, GB/s of one rank, whole-job GB/s): every rank moves the same
+    bytes; the slowest rank's time (ms for `steps` steps) bounds the job."""
+    us = ms_max * 1e3 / steps
+    gbs_rank = bytes_per_step / (us * 1e-6) / 1e9
+    return us, gbs_rank, gbs_rank * world
 
 
 def measure_config(w, steps, warmup, stream, dist_ctx, l2):
@@ -337,10 +354,8 @@ def run_ours(args):
     with ClockSampler(ctx.local) as clk:
         ms_local = time_graph(prob, args.steps, args.warmup, stream, ctx)
     ms = ctx.max(ms_local)
-    us = ms * 1e3 / args.steps
     b = algo_bytes(w.M, w.N, w.K, w.r)
-    gbs_rank = b / (us * 1e-6) / 1e9
-    value = gbs_rank * ctx.world
+    us, gbs_rank, value = step_metrics(b, ms, args.steps, ctx.world)
 
     e2e_steps = min(args.steps, 2000)
     e2e_ms, h2d, d2h = time_e2e(prob, e2e_steps, stream)
@@ -370,7 +385,7 @@ def run_ours(args):
                    "launch": f"CUDA graph replay, {nb.gemm_kernel_count(w.M)} kernel(s) per step"},
         "roofline": {"bound": "hbm", "achieved": round(gbs_rank, 1), "peak": peak,
                      "unit": "GB/s", "frac": round(gbs_rank / peak, 4),
-                     "traffic": ncu_traffic(w.name),
+                     "traffic": ncu_traffic(w.name, w.M),
                      "peak_kind": peak_kind, "per": "step (all kernels of one call)"},
         "e2e": {"value": round(e2e_val, 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "us_per_step": round(e2e_ms * 1e3, 3),
