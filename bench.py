@@ -382,7 +382,7 @@ def run_ours(args):
         "config": {"workload": w.name, "M": w.M, "N": w.N, "K": w.K, "r": w.r,
                    "seed": w.seed, "parallelism": f"replicas x{ctx.world}",
                    "l2": f"{n_copies_for(w, l2)} weight copies rotated (> L2 {l2 >> 20} MiB)",
-                   "launch": f"CUDA graph replay, {nb.gemm_kernel_count(w.M)} kernel(s) per step"},
+                   "launch": f"CUDA graph replay, {nb.gemm_kernel_count(w.M, w.N, w.K, w.r)} kernel(s) per step"},
         "roofline": {"bound": "hbm", "achieved": round(gbs_rank, 1), "peak": peak,
                      "unit": "GB/s", "frac": round(gbs_rank / peak, 4),
                      "traffic": ncu_traffic(w.name, w.M),
@@ -390,7 +390,7 @@ def run_ours(args):
         "e2e": {"value": round(e2e_val, 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "us_per_step": round(e2e_ms * 1e3, 3),
                 "api": "nvfp4_binary_rank_b200.gemm, eager, pinned host x/y"},
-        "gpu_launches": nb.gemm_kernel_count(w.M) * args.steps,
+        "gpu_launches": nb.gemm_kernel_count(w.M, w.N, w.K, w.r) * args.steps,
         "clocks": clk.summary(),
         "extra_configs": extra,
     }

@@ -148,8 +148,9 @@ size_t biloco_weight_sf_bytes(int N, int K);
  *   limits  1 <= M <= 128, N % 128 == 0, N <= 2^24, K % 64 == 0, 0 <= r <= 1024,
  *           (N/128) * ceil(K/256) <= 2^24
  * Accumulation is FP32 in an unspecified order; results are deterministic for a
- * fixed shape, mode and GPU.  For M <= 8 one kernel is launched (it quantises
- * the activation itself); for larger M an activation quantiser runs first.
+ * fixed shape, mode and GPU.  Decode batches (M <= 16, shared-z schedule) run
+ * one kernel that quantises the activation itself; otherwise an activation
+ * quantiser runs first for M > 8 (biloco_gemm_kernel_count).
  * The fused kernel is launched with programmatic dependent launch: it may start
  * while the kernel before it on the stream finishes, and it reads W_fp4 and
  * W_sf before waiting for that kernel (everything else after).  So the weight
@@ -216,9 +217,12 @@ int biloco_last_error(biloco_stream_t stream);
 /* Human-readable name of a status code (static storage). */
 const char *biloco_status_string(int status);
 
-/* Number of kernels biloco_gemm launches per call for a batch of M rows:
- * 1 when the activation is quantised inside the fused kernel (M <= 8), else 2. */
-int biloco_gemm_kernel_count(int M);
+/* Number of kernels biloco_gemm would launch per call for this shape under the
+ * current schedule setting: 1 when the GEMM kernel quantises the activation
+ * itself (the decode-batch kernel, M <= 16, or the general kernel at M <= 8),
+ * else 2 (quantiser + GEMM).  BILOCO_ERR_SHAPE for shapes biloco_gemm rejects.
+ * Uses the device's SM count (the current device must be set). */
+int biloco_gemm_kernel_count(int M, int N, int K, int r);
 
 /* Free every stream's scratch.  Safe to call more than once. */
 void biloco_shutdown(void);

@@ -40,7 +40,7 @@ SIGNATURES = {
     "biloco_resolve_mode": (_I, [_I, _I, _I, _I]),
     "biloco_last_error": (_I, [_P]),
     "biloco_status_string": (ctypes.c_char_p, [_I]),
-    "biloco_gemm_kernel_count": (_I, [_I]),
+    "biloco_gemm_kernel_count": (_I, [_I, _I, _I, _I]),
     "biloco_shutdown": (None, []),
 }
 
@@ -188,8 +188,10 @@ def last_error(stream=None) -> int:
     return int(load().biloco_last_error(_stream(stream)))
 
 
-def gemm_kernel_count(M: int) -> int:
-    return int(load().biloco_gemm_kernel_count(M))
+def gemm_kernel_count(M: int, N: int, K: int, r: int) -> int:
+    n = int(load().biloco_gemm_kernel_count(M, N, K, r))
+    _check("biloco_gemm_kernel_count", min(n, 0))
+    return n
 
 
 def shutdown():

@@ -284,7 +284,17 @@ const char* biloco_status_string(int status) {
   }
 }
 
-int biloco_gemm_kernel_count(int M) { return gemm_kernel_count_for(M); }
+int biloco_gemm_kernel_count(int M, int N, int K, int r) {
+  if (M < 1 || M > BILOCO_MAX_M || N < 128 || N % 128 || K < 64 || K % 64 || r < 0 || r > BILOCO_MAX_R)
+    return BILOCO_ERR_SHAPE;
+  GemmArgs a = {};
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.r = r;
+  a.mode = resolve_mode(M, N, K, r, g_mode.load());
+  return gemm_kernel_count_for(a);
+}
 
 void biloco_shutdown(void) {
   std::lock_guard<std::mutex> lk(g_mu);

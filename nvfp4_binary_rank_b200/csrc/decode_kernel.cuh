@@ -57,15 +57,13 @@ constexpr int kAluWarps = 8;
 constexpr int kAluThreads = kAluWarps * 32;
 constexpr int kFinThreads = kEpiThreads + kAluThreads;
 constexpr int kBN = 16;                   // MMA N (activation rows, padded)
-constexpr int kRowsMax = 8;               // activation rows handled
+constexpr int kRowsMax = 16;              // activation rows handled
 constexpr int kTileRows = 128;            // weight rows per tile = MMA M
 constexpr int kUnitK = 256;               // K elements per unit
 constexpr int kUnitBytesA = kTileRows * 128;
 constexpr int kSfBytes = 2048;            // 4 scale atoms of 512 B per unit
-constexpr int kStages = 6;                // weight stage ring
 constexpr int kMaxUnits = 16;             // units per CTA (operand cache entries)
 constexpr int kMaxRanks = 1024;
-constexpr int kRankGroup = 8;             // V-side ranks per pass
 // TMEM columns: accumulators [0, 32); activation scales per unit [32, 288);
 // weight scales per stage [288, 384)
 constexpr int kTmemCols = 512;
@@ -79,8 +77,19 @@ constexpr int kBarEpi = 2;
 constexpr int kBarFin = 3;                // epilogue + CUDA cores: finisher decision
 constexpr int kBarFin2 = 4;               // epilogue + CUDA cores: correction ready
 
+// Per batch class (MC = most activation rows): weight stages and V-side ranks
+// per pass (the largest class trades stages and ranks for its z and register
+// footprint).
+template <int MC>
+struct Cfg {
+  static constexpr int kStages = (MC >= 16) ? 4 : 6;
+  static constexpr int kRankGroup = (MC >= 16) ? 4 : 8;
+};
+
 template <int MC>
 struct Layout {
+  static constexpr int kStages = Cfg<MC>::kStages;
+  static constexpr int kRankGroup = Cfg<MC>::kRankGroup;
   static constexpr int kA = 0;                                        // [ST][128][128 B]
   static constexpr int kSFA = kA + kStages * kUnitBytesA;              // [ST][2 KB]
   static constexpr int kB = kSFA + kStages * kSfBytes;                 // [NU][16][128 B]
@@ -102,7 +111,7 @@ struct Layout {
 // word w this warp handles; acc[m][i] collects sum_k s_ik x[m][k].  Inputs that
 // the previous kernel of the stream may have written are read through L2
 // (ld.global.cg), never through a possibly stale L1 line.
-template <int MC>
+template <int MC, int kRankGroup = Cfg<MC>::kRankGroup>
 __device__ __forceinline__ void vside_group(const DecodeParams& p, int ig, int nr, int a, int lane,
                                             float (&acc)[MC][kRankGroup]) {
 #pragma unroll
@@ -111,7 +120,7 @@ __device__ __forceinline__ void vside_group(const DecodeParams& p, int ig, int n
     for (int i = 0; i < kRankGroup; ++i) acc[m][i] = 0.0f;
   const uint32_t lane_shift = 31u - static_cast<uint32_t>(lane);
   const uint32_t* vrow = p.Vbits + static_cast<size_t>(ig) * p.KW;
-  constexpr int kUnroll = (MC >= 8) ? 2 : 4;
+  constexpr int kUnroll = (MC >= 16) ? 1 : ((MC >= 8) ? 2 : 4);   // words per warp per load round
   for (int w0 = a; w0 < p.KW; w0 += kAluWarps * kUnroll) {
     uint32_t xs[kUnroll][MC];
     uint32_t vw[kUnroll][kRankGroup];
@@ -145,6 +154,7 @@ template <int MC>
 __global__ void __launch_bounds__(kThreads, 1)
 decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ DecodeParams p) {
   using L = Layout<MC>;
+  constexpr int kStages = Cfg<MC>::kStages, kRankGroup = Cfg<MC>::kRankGroup;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -325,7 +335,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
     const int row = q * 32 + lane;                     // weight row within the tile
     const int etid = threadIdx.x - kEpiWarp0 * 32;
     const float gs = __ldcg(p.gscale);
-    constexpr int kHB = (MC <= 2) ? 16 : (MC <= 4 ? 8 : 4);   // partials loaded per batch
+    constexpr int kHB = (MC <= 2) ? 16 : (MC <= 4 ? 8 : (MC <= 8 ? 4 : 2));   // partials loaded per batch
     bool ok = true;
     for (int seg = 0; seg < nseg; ++seg) {
       const int t = t_first + seg;

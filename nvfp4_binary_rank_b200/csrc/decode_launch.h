@@ -1,5 +1,5 @@
-// Launchers of the decode-batch kernel instances (batch classes 1, 2, 4 and 8
-// activation rows; each in its own translation unit).
+// Launchers of the decode-batch kernel instances (batch classes 1, 2, 4, 8 and
+// 16 activation rows; each in its own translation unit).
 #pragma once
 
 #include <cuda.h>
@@ -11,11 +11,12 @@ namespace biloco {
 
 // Units of 128 weight rows x 256 K elements one CTA of the decode kernel can hold.
 constexpr int kDecodeMaxUnits = 16;
-constexpr int kDecodeMaxRows = 8;
+constexpr int kDecodeMaxRows = 16;
 
 cudaError_t launch_decode_1(const CUtensorMap& tw, const DecodeParams& dp, cudaStream_t s);
 cudaError_t launch_decode_2(const CUtensorMap& tw, const DecodeParams& dp, cudaStream_t s);
 cudaError_t launch_decode_4(const CUtensorMap& tw, const DecodeParams& dp, cudaStream_t s);
 cudaError_t launch_decode_8(const CUtensorMap& tw, const DecodeParams& dp, cudaStream_t s);
+cudaError_t launch_decode_16(const CUtensorMap& tw, const DecodeParams& dp, cudaStream_t s);
 
 }  // namespace biloco

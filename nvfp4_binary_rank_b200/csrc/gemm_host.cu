@@ -105,7 +105,10 @@ int resolve_mode(int M, int N, int K, int r, int requested) {
   return BILOCO_MODE_SHARED_Z;
 }
 
-int gemm_kernel_count_for(int M) { return M <= kInKernelQuantMaxM ? 1 : 2; }
+int gemm_kernel_count_for(const GemmArgs& a) {
+  const GemmPlan p = plan_gemm(a);
+  return (p.decode || p.inq) ? 1 : 2;
+}
 
 GemmPlan plan_gemm(const GemmArgs& a) {
   const int M = a.M, N = a.N, K = a.K, r = a.r;
@@ -188,7 +191,8 @@ int launch_gemm(const GemmArgs& a, const GemmPlan& p, const Scratch& scr, cudaSt
     if (M <= 1) e = launch_decode_1(tw, dp, s);
     else if (M <= 2) e = launch_decode_2(tw, dp, s);
     else if (M <= 4) e = launch_decode_4(tw, dp, s);
-    else e = launch_decode_8(tw, dp, s);
+    else if (M <= 8) e = launch_decode_8(tw, dp, s);
+    else e = launch_decode_16(tw, dp, s);
     return e == cudaSuccess ? BILOCO_OK : BILOCO_ERR_CUDA;
   }
   if (!inq) {

@@ -83,6 +83,6 @@ int resolve_mode(int M, int N, int K, int r, int requested);
 // Status word of biloco_gemm_noalloc's static scratch on the current device:
 // returned and, if non-zero, cleared together with its counters (synchronous).
 int noalloc_take_status();
-int gemm_kernel_count_for(int M);
+int gemm_kernel_count_for(const GemmArgs& a);
 
 }  // namespace biloco

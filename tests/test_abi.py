@@ -80,3 +80,20 @@ def test_mode_setting(lib):
         assert lib.biloco_resolve_mode(1, 5120, 5120, 512) == m
     assert lib.biloco_set_mode(_lib.MODE_AUTO) == 0
     assert lib.biloco_resolve_mode(1, 5120, 5120, 512) in (_lib.MODE_SHARED_Z, _lib.MODE_LOCAL_Z)
+
+
+def test_kernel_count_follows_the_schedule(lib):
+    from nvfp4_binary_rank_b200 import _lib
+    # decode batches run one kernel (it quantises the activation itself)
+    assert lib.biloco_gemm_kernel_count(1, 5120, 5120, 512) == 1
+    assert lib.biloco_gemm_kernel_count(16, 13824, 5120, 512) == 1
+    # larger batches: quantiser + GEMM
+    assert lib.biloco_gemm_kernel_count(32, 5120, 13824, 512) == 2
+    # the local-z schedule runs the general kernel (in-kernel quantisation up to M = 8)
+    assert lib.biloco_set_mode(_lib.MODE_LOCAL_Z) == 0
+    try:
+        assert lib.biloco_gemm_kernel_count(8, 5120, 5120, 512) == 1
+        assert lib.biloco_gemm_kernel_count(16, 5120, 5120, 512) == 2
+    finally:
+        lib.biloco_set_mode(_lib.MODE_AUTO)
+    assert lib.biloco_gemm_kernel_count(1, 100, 64, 0) == -2
