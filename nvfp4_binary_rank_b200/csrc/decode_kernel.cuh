@@ -65,10 +65,13 @@ constexpr int kSfBytes = 2048;            // 4 scale atoms of 512 B per unit
 constexpr int kMaxUnits = 16;             // units per CTA (operand cache entries)
 constexpr int kMaxRanks = 1024;
 // TMEM columns: accumulators [0, 32); activation scales per unit [32, 288);
-// weight scales per stage [288, 384)
+// weight scales per stage [288, 384); the U-side product [384, 416)
 constexpr int kTmemCols = 512;
 constexpr int kSfbTmemBase = 32;
 constexpr int kSfaTmemBase = kSfbTmemBase + 16 * 16;
+constexpr int kUTmem = 384;
+constexpr int kUChunk = 64;               // ranks per U-side MMA chunk (one 128-byte BF16 row)
+constexpr int kUChunksMax = 16;           // r <= 1024
 constexpr uint32_t kStageTx = kUnitBytesA + kSfBytes;
 
 // named barriers (0 is __syncthreads)
@@ -84,6 +87,9 @@ template <int MC>
 struct Cfg {
   static constexpr int kStages = (MC >= 16) ? 4 : 6;
   static constexpr int kRankGroup = (MC >= 16) ? 4 : 8;
+  // U side on the tensor cores from 4 rows up; below, per-thread sign-adds are
+  // cheaper than the chunked MMA chain (measured on B200)
+  static constexpr bool kTensorU = MC >= 4;
 };
 
 template <int MC>
@@ -94,16 +100,25 @@ struct Layout {
   static constexpr int kSFA = kA + kStages * kUnitBytesA;              // [ST][2 KB]
   static constexpr int kB = kSFA + kStages * kSfBytes;                 // [NU][16][128 B]
   static constexpr int kSFB = kB + kMaxUnits * kBN * 128;              // [NU][4 steps][32 rows] u32
+  // U side on the tensor cores: A = the tile's U signs as +-1 BF16, 64 ranks per
+  // chunk (two buffers); B = z as BF16 high and low parts, kUN rows per chunk
+  static constexpr int kUN = (2 * MC < 16) ? 16 : 2 * MC;               // MMA N of the U side
+  static constexpr int kUA = kSFB + kMaxUnits * 512;                   // [2][128][128 B]
+  static constexpr int kUZ = kUA + 2 * kTileRows * 128;                // [16][kUN][128 B]
+  // without the tensor-core U side: z staged as floats and the two half sums
   static constexpr int kZ = kSFB + kMaxUnits * 512;                    // [MC][1024] floats
   static constexpr int kCorr = kZ + MC * kMaxRanks * 4;                // [2][MC][128] floats
-  static constexpr int kVRed = kCorr + 2 * MC * kTileRows * 4;         // [8][MC * 8] floats
+  static constexpr int kUEnd = Cfg<MC>::kTensorU ? kUZ + kUChunksMax * kUN * 128
+                                                 : kCorr + 2 * MC * kTileRows * 4;
+  static constexpr int kVRed = kUEnd;                                  // [8][MC * ranks] floats
   static constexpr int kBar = kVRed + kAluWarps * MC * kRankGroup * 4;
-  static constexpr int kNumBars = 2 * kStages + 7;
+  static constexpr int kNumBars = 2 * kStages + 10;
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kFinFlags = kMisc + 32;                         // [kMaxUnits + 1] ints
   static constexpr int kTotal = kFinFlags + (kMaxUnits + 1) * 4;
   static constexpr int kAlloc = kTotal + 1024;
-  static_assert(kSFA % 1024 == 0 && kB % 1024 == 0, "swizzled tiles need 1 KB alignment");
+  static_assert(kSFA % 1024 == 0 && kB % 1024 == 0 && kUA % 1024 == 0 && kUZ % 1024 == 0,
+                "swizzled tiles need 1 KB alignment");
   static_assert(kAlloc <= 232448, "shared memory budget");
 };
 
@@ -168,6 +183,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
   auto acce_bar = [&](int b) { return smem_u32(&bars[2 * kStages + 3 + b]); };
   const uint32_t drain_bar = smem_u32(&bars[2 * kStages + 5]);
   const uint32_t done_bar = smem_u32(&bars[2 * kStages + 6]);
+  auto ubuf_bar = [&](int b) { return smem_u32(&bars[2 * kStages + 7 + b]); };
+  const uint32_t ud_bar = smem_u32(&bars[2 * kStages + 9]);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
   volatile int* epi_last = reinterpret_cast<volatile int*>(smem + L::kMisc + 8);
@@ -193,6 +210,9 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
     }
     mbar_init(drain_bar, 1);
     mbar_init(done_bar, kWarps);
+    mbar_init(ubuf_bar(0), 1);
+    mbar_init(ubuf_bar(1), 1);
+    mbar_init(ud_bar, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -337,6 +357,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
     const float gs = __ldcg(p.gscale);
     constexpr int kHB = (MC <= 2) ? 16 : (MC <= 4 ? 8 : (MC <= 8 ? 4 : 2));   // partials loaded per batch
     bool ok = true;
+    int nfin = 0;                                      // tiles completed here (U-side results read)
     for (int seg = 0; seg < nseg; ++seg) {
       const int t = t_first + seg;
       const int b = seg & 1;
@@ -423,10 +444,31 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
           ok = false;
           break;
         }
-        const float* corr = reinterpret_cast<const float*>(smem + L::kCorr);
+        if constexpr (Cfg<MC>::kTensorU) {
+          // the correction: the U-side MMAs left sum_i U[n][i] zhi[m][i] in column m
+          // and sum_i U[n][i] zlo[m][i] in column MC + m of lane n
+          const bool got = group_wait(ud_bar, nfin & 1, kBarEpi, kEpiThreads, ctl);
+          ++nfin;
+          if (!got) {
+            ok = false;
+            continue;                                    // the next vote tells the CUDA-core warps
+          }
+          tc_fence_after();
+          uint32_t du[L::kUN];
+          tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + kUTmem, *reinterpret_cast<uint32_t(*)[16]>(du));
+          if constexpr (L::kUN > 16)
+            tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + kUTmem + 16,
+                      *reinterpret_cast<uint32_t(*)[16]>(du + 16));
+          tmem_wait_ld();
+          tc_fence_before();
+  #pragma unroll
+          for (int j = 0; j < MC; ++j) acc[j] += __uint_as_float(du[j]) + __uint_as_float(du[MC + j]);
+        } else {
+          const float* corr = reinterpret_cast<const float*>(smem + L::kCorr);
 #pragma unroll
-        for (int j = 0; j < MC; ++j)
-          acc[j] = (acc[j] + corr[j * kTileRows + row]) + corr[(MC + j) * kTileRows + row];
+          for (int j = 0; j < MC; ++j)
+            acc[j] = (acc[j] + corr[j * kTileRows + row]) + corr[(MC + j) * kTileRows + row];
+        }
       }
       uint16_t* yb = p.y + static_cast<size_t>(t) * kTileRows + row;
 #pragma unroll
@@ -562,79 +604,232 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
       named_barrier(kBarAlu, kAluThreads);
       if (tid == 0) red_add_release_gpu(p.z_ready, 1u);   // covers the slice the CTA wrote
 
-      // ---- 3. U side of every tile this CTA completes
-      float* zs = reinterpret_cast<float*>(smem + L::kZ);
-      float* corr = reinterpret_cast<float*>(smem + L::kCorr);
-      bool ok = true, staged = false;
-      for (int seg = 0; seg < nseg; ++seg) {
-        if (named_barrier_or(kBarFin, kFinThreads, !ok)) {
-          ok = false;
-          break;
-        }
-        if (!fin_flag[seg]) continue;
-        const int t = t_first + seg;
-        if (!staged) {
-          bool okw = true;
-          if (tid == 0) okw = spin_until_geq(p.z_ready, static_cast<uint32_t>(p.G), ctl);
-          if (named_barrier_or(kBarAlu, kAluThreads, !okw)) {
-            fail(ctl);
+      if constexpr (Cfg<MC>::kTensorU) {
+        // ---- 3. U side of every tile this CTA completes, on the tensor cores:
+        // corr[n][m] = sum_i U[n][i] z[m][i] as one BF16 MMA chain per tile, 64 ranks
+        // per chunk.  A = the tile's sign bits expanded to +-1 BF16 (exact); B = z split
+        // into a BF16 high part and the BF16 rounding of the rest (rows m and MC + m),
+        // so the product keeps about 16 bits of z.  The epilogue adds both columns.
+        const int nuc = (p.r + kUChunk - 1) / kUChunk;
+        const int row = tid & (kTileRows - 1), half = tid >> 7;
+        const uint32_t idesc_u = (1u << 4) | (1u << 7) | (1u << 10) |
+                                 (static_cast<uint32_t>(L::kUN >> 3) << 17) |
+                                 (static_cast<uint32_t>(kTileRows >> 4) << 24);
+        // this thread expands word 2 c + half of row `row` for chunk c
+        auto load_words = [&](int t, uint32_t (&uw)[kUChunksMax]) {
+          const uint32_t* ur = p.Ubits + (static_cast<size_t>(t) * kTileRows + row) * p.RW;
+  #pragma unroll
+          for (int c = 0; c < kUChunksMax; ++c) {
+            const int w = 2 * c + half;
+            uw[c] = (w < p.RW) ? __ldcg(ur + w) : 0u;
+          }
+        };
+        uint32_t uw0[kUChunksMax], uw1[kUChunksMax];
+        load_words(t_first, uw0);
+        if (nseg > 1) load_words(t_first + 1, uw1);
+        bool ok = true, ztiles = false;
+        int uses0 = 0, uses1 = 0;                        // MMA rounds issued on each A buffer
+        for (int seg = 0; seg < nseg; ++seg) {
+          if (named_barrier_or(kBarFin, kFinThreads, !ok)) {
             ok = false;
-          } else {
-            const int span = 32 * p.RW;
-            for (int idx = tid; idx < p.M * span; idx += kAluThreads) {
-              const int m = idx / span, i = idx - m * span;
-              zs[m * kMaxRanks + i] = (i < p.r) ? __ldcg(p.z + static_cast<size_t>(m) * p.rpad + i) : 0.0f;
+            break;
+          }
+          if (!fin_flag[seg]) continue;
+          if (!ztiles) {
+            // first tile this CTA completes: wait for every slice of z, then the B tiles
+            bool okw = true;
+            if (tid == 0) okw = spin_until_geq(p.z_ready, static_cast<uint32_t>(p.G), ctl);
+            if (named_barrier_or(kBarAlu, kAluThreads, !okw)) {
+              fail(ctl);
+              ok = false;
             }
+            uint4* zt4 = reinterpret_cast<uint4*>(smem + L::kUZ);
+            for (int idx = tid; idx < nuc * L::kUN * 8; idx += kAluThreads) zt4[idx] = make_uint4(0u, 0u, 0u, 0u);
             named_barrier(kBarAlu, kAluThreads);
-            staged = true;
+            const int items = nuc * p.M * 32;             // (chunk, row, rank pair)
+            constexpr int kZB = 4;
+            for (int base = 0; base < items; base += kAluThreads * kZB) {
+              float2 zv[kZB];
+  #pragma unroll
+              for (int e = 0; e < kZB; ++e) {
+                const int idx = base + e * kAluThreads + tid;
+                zv[e] = make_float2(0.0f, 0.0f);
+                if (idx < items) {
+                  const int c = idx / (p.M * 32), rem = idx - c * p.M * 32, m = rem >> 5, qq = rem & 31;
+                  const int i = c * kUChunk + 2 * qq;
+                  if (i < p.r) {                           // i even and rpad even: i + 1 < rpad
+                    const float2 v = __ldcg(reinterpret_cast<const float2*>(p.z + static_cast<size_t>(m) * p.rpad + i));
+                    zv[e].x = v.x;
+                    zv[e].y = (i + 1 < p.r) ? v.y : 0.0f;
+                  }
+                }
+              }
+  #pragma unroll
+              for (int e = 0; e < kZB; ++e) {
+                const int idx = base + e * kAluThreads + tid;
+                if (idx < items) {
+                  const int c = idx / (p.M * 32), rem = idx - c * p.M * 32, m = rem >> 5, qq = rem & 31;
+                  const __nv_bfloat16 h0 = __float2bfloat16_rn(zv[e].x), h1 = __float2bfloat16_rn(zv[e].y);
+                  const __nv_bfloat16 l0 = __float2bfloat16_rn(zv[e].x - __bfloat162float(h0));
+                  const __nv_bfloat16 l1 = __float2bfloat16_rn(zv[e].y - __bfloat162float(h1));
+                  const uint32_t hi = static_cast<uint32_t>(__bfloat16_as_ushort(h0)) |
+                                      (static_cast<uint32_t>(__bfloat16_as_ushort(h1)) << 16);
+                  const uint32_t lo = static_cast<uint32_t>(__bfloat16_as_ushort(l0)) |
+                                      (static_cast<uint32_t>(__bfloat16_as_ushort(l1)) << 16);
+                  const int byte = 4 * qq;
+                  uint8_t* tile = smem + L::kUZ + c * L::kUN * 128;
+                  *reinterpret_cast<uint32_t*>(tile + m * 128 + ((((byte >> 4) ^ (m & 7)) << 4) | (byte & 15))) = hi;
+                  const int ml = MC + m;
+                  *reinterpret_cast<uint32_t*>(tile + ml * 128 + ((((byte >> 4) ^ (ml & 7)) << 4) | (byte & 15))) = lo;
+                }
+              }
+            }
+            fence_proxy_async_smem();
+            named_barrier(kBarAlu, kAluThreads);
+            ztiles = true;
+          }
+          if (seg >= 2) load_words(t_first + seg, uw1);    // segments past the second: load now
+  #pragma unroll
+          for (int c = 0; c < kUChunksMax; ++c) {
+            if (c < nuc) {
+              const int buf = c & 1;
+              int& uses = buf ? uses1 : uses0;
+              if (uses > 0) {
+                // the MMAs that read this buffer last are done
+                bool okb = true;
+                if (tid == 0) okb = mbar_wait(ubuf_bar(buf), (uses - 1) & 1, abort_flag);
+                if (named_barrier_or(kBarAlu, kAluThreads, !okb)) {
+                  fail(ctl);
+                  ok = false;
+                }
+              }
+              const uint32_t word = (seg == 0) ? uw0[c] : uw1[c];
+              uint8_t* arow = smem + L::kUA + buf * (kTileRows * 128) + row * 128;
+  #pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                uint32_t pk[4];
+  #pragma unroll
+                for (int t2 = 0; t2 < 4; ++t2) {
+                  const int j = 8 * k + 2 * t2;
+                  pk[t2] = 0x3F803F80u | (((word >> j) & 1u) << 15) | (((word >> (j + 1)) & 1u) << 31);
+                }
+                const int piece = 4 * half + k;
+                *reinterpret_cast<uint4*>(arow + ((piece ^ (row & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+              }
+              fence_proxy_async_smem();
+              named_barrier(kBarAlu, kAluThreads);
+              if (tid == 0) {
+                tc_fence_after();
+                const uint64_t a_d = smem_desc(smem_u32(smem + L::kUA + buf * (kTileRows * 128)), 16, 1024, 2);
+                const uint64_t b_d = smem_desc(smem_u32(smem + L::kUZ + c * L::kUN * 128), 16, 1024, 2);
+  #pragma unroll
+                for (int j = 0; j < 4; ++j)
+                  tc_mma_bf16(tmem + kUTmem, a_d + 2 * j, b_d + 2 * j, idesc_u, (c > 0 || j > 0) ? 1u : 0u);
+                tc_commit(ubuf_bar(buf));
+              }
+              ++uses;
+            }
+          }
+          if (tid == 0) tc_commit(ud_bar);
+          if (named_barrier_or(kBarFin2, kFinThreads, !ok)) {
+            ok = false;
+            break;
           }
         }
-        if (ok) {
-          const int row = tid & (kTileRows - 1), half = tid >> 7;
-          const int wsplit = (p.RW + 1) >> 1;
-          const int wa = half ? wsplit : 0, wb = half ? p.RW : wsplit;
-          const uint32_t* ur = p.Ubits + (static_cast<size_t>(t) * kTileRows + row) * p.RW;
-          uint32_t uw[16];
-#pragma unroll
-          for (int w = 0; w < 16; ++w) uw[w] = (wa + w < wb) ? __ldcg(ur + wa + w) : 0u;
-          float acc[MC];
-#pragma unroll
-          for (int m = 0; m < MC; ++m) acc[m] = 0.0f;
-          for (int w = 0; w < wb - wa; ++w) {
-            uint32_t word = 0;
-#pragma unroll
-            for (int e = 0; e < 16; ++e) word = (e == w) ? uw[e] : word;
-            const float* zw = zs + (wa + w) * 32;
-#pragma unroll
-            for (int j4 = 0; j4 < 8; ++j4) {
-#pragma unroll
-              for (int m = 0; m < MC; ++m) {
-                if (m < p.M) {
-                  const float4 z4 = *reinterpret_cast<const float4*>(zw + m * kMaxRanks + 4 * j4);
-                  const float zz[4] = {z4.x, z4.y, z4.z, z4.w};
-#pragma unroll
-                  for (int jj = 0; jj < 4; ++jj) {
-                    const uint32_t sgn = (word << (31 - (4 * j4 + jj))) & 0x80000000u;
-                    acc[m] += __uint_as_float(__float_as_uint(zz[jj]) ^ sgn);
+        // the U-side MMAs must be finished before TMEM is freed (bounded wait)
+        if (tid == 0 && uses0 + uses1 > 0) {
+          tc_commit(ubuf_bar(0));
+          const uint64_t t0 = globaltimer_ns();
+          while (!mbar_try_wait(ubuf_bar(0), uses0 & 1)) {
+            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+              record_error(p.status, kDevErrTimeout);
+              break;
+            }
+          }
+        }
+        // this CTA is done with z_ready; the last CTA to get here resets both counters
+        if (tid == 0 && ok) {
+          const uint32_t old = atomicAdd(p.z_seen, 1u);
+          if (old == static_cast<uint32_t>(p.G - 1)) {
+            atomicExch(p.z_ready, 0u);
+            atomicExch(p.z_seen, 0u);
+          }
+        }
+      } else {
+        // ---- 3. U side of every tile this CTA completes
+        float* zs = reinterpret_cast<float*>(smem + L::kZ);
+        float* corr = reinterpret_cast<float*>(smem + L::kCorr);
+        bool ok = true, staged = false;
+        for (int seg = 0; seg < nseg; ++seg) {
+          if (named_barrier_or(kBarFin, kFinThreads, !ok)) {
+            ok = false;
+            break;
+          }
+          if (!fin_flag[seg]) continue;
+          const int t = t_first + seg;
+          if (!staged) {
+            bool okw = true;
+            if (tid == 0) okw = spin_until_geq(p.z_ready, static_cast<uint32_t>(p.G), ctl);
+            if (named_barrier_or(kBarAlu, kAluThreads, !okw)) {
+              fail(ctl);
+              ok = false;
+            } else {
+              const int span = 32 * p.RW;
+              for (int idx = tid; idx < p.M * span; idx += kAluThreads) {
+                const int m = idx / span, i = idx - m * span;
+                zs[m * kMaxRanks + i] = (i < p.r) ? __ldcg(p.z + static_cast<size_t>(m) * p.rpad + i) : 0.0f;
+              }
+              named_barrier(kBarAlu, kAluThreads);
+              staged = true;
+            }
+          }
+          if (ok) {
+            const int row = tid & (kTileRows - 1), half = tid >> 7;
+            const int wsplit = (p.RW + 1) >> 1;
+            const int wa = half ? wsplit : 0, wb = half ? p.RW : wsplit;
+            const uint32_t* ur = p.Ubits + (static_cast<size_t>(t) * kTileRows + row) * p.RW;
+            uint32_t uw[16];
+  #pragma unroll
+            for (int w = 0; w < 16; ++w) uw[w] = (wa + w < wb) ? __ldcg(ur + wa + w) : 0u;
+            float acc[MC];
+  #pragma unroll
+            for (int m = 0; m < MC; ++m) acc[m] = 0.0f;
+            for (int w = 0; w < wb - wa; ++w) {
+              uint32_t word = 0;
+  #pragma unroll
+              for (int e = 0; e < 16; ++e) word = (e == w) ? uw[e] : word;
+              const float* zw = zs + (wa + w) * 32;
+  #pragma unroll
+              for (int j4 = 0; j4 < 8; ++j4) {
+  #pragma unroll
+                for (int m = 0; m < MC; ++m) {
+                  if (m < p.M) {
+                    const float4 z4 = *reinterpret_cast<const float4*>(zw + m * kMaxRanks + 4 * j4);
+                    const float zz[4] = {z4.x, z4.y, z4.z, z4.w};
+  #pragma unroll
+                    for (int jj = 0; jj < 4; ++jj) {
+                      const uint32_t sgn = (word << (31 - (4 * j4 + jj))) & 0x80000000u;
+                      acc[m] += __uint_as_float(__float_as_uint(zz[jj]) ^ sgn);
+                    }
                   }
                 }
               }
             }
+  #pragma unroll
+            for (int m = 0; m < MC; ++m) corr[(half * MC + m) * kTileRows + row] = acc[m];
           }
-#pragma unroll
-          for (int m = 0; m < MC; ++m) corr[(half * MC + m) * kTileRows + row] = acc[m];
+          if (named_barrier_or(kBarFin2, kFinThreads, !ok)) {
+            ok = false;
+            break;
+          }
         }
-        if (named_barrier_or(kBarFin2, kFinThreads, !ok)) {
-          ok = false;
-          break;
-        }
-      }
-      // this CTA is done with z_ready; the last CTA to get here resets both counters
-      if (tid == 0 && ok) {
-        const uint32_t old = atomicAdd(p.z_seen, 1u);
-        if (old == static_cast<uint32_t>(p.G - 1)) {
-          atomicExch(p.z_ready, 0u);
-          atomicExch(p.z_seen, 0u);
+        // this CTA is done with z_ready; the last CTA to get here resets both counters
+        if (tid == 0 && ok) {
+          const uint32_t old = atomicAdd(p.z_seen, 1u);
+          if (old == static_cast<uint32_t>(p.G - 1)) {
+            atomicExch(p.z_ready, 0u);
+            atomicExch(p.z_seen, 0u);
+          }
         }
       }
     }
