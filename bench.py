@@ -75,10 +75,10 @@ def kernel_source_digest() -> str:
 
 def ncu_traffic(workload: str, M: int):
     """DRAM bytes (read + write) per launch of the GEMM kernel that serves this
-    workload (decode_kernel for M <= 8, fused_kernel above), from the committed
+    workload (decode_kernel for M <= 16, fused_kernel above), from the committed
     ncu summary, or None when there is none or the kernel sources changed since
     it was captured."""
-    kernel = "decode_kernel" if M <= 8 else "fused_kernel"
+    kernel = "decode_kernel" if M <= 16 else "fused_kernel"
     path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
     try:
         fields = {}

@@ -214,6 +214,17 @@ int biloco_resolve_mode(int M, int N, int K, int r);
  */
 int biloco_last_error(biloco_stream_t stream);
 
+/*
+ * biloco_selftest_wait_timeout - exercise the failure path on the GPU without a
+ * fault.  Launches one warp that waits, through the same bounded mbarrier wait
+ * the GEMM kernels use, on a phase nothing completes.  After the wait's
+ * wall-clock limit (about 1 s) the kernel records BILOCO_ERR_TIMEOUT in
+ * `stream`'s status word and returns, leaving the context usable; a following
+ * biloco_last_error(stream) reports it.  The BiLoCo pages have no counterpart
+ * of this call.
+ */
+int biloco_selftest_wait_timeout(biloco_stream_t stream);
+
 /* Human-readable name of a status code (static storage). */
 const char *biloco_status_string(int status);
 

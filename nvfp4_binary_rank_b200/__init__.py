@@ -9,7 +9,7 @@ is its thin ctypes binding.  Build the library with
 
 from ._lib import (  # noqa: F401
     BilocoError, MODE_AUTO, MODE_LOCAL_Z, MODE_SHARED_Z, MAX_M, MAX_R, gemm, gemm_kernel_count,
-    gemm_noalloc,
+    gemm_noalloc, selftest_wait_timeout,
     last_error, load, pack_signs, pack_weight, quant_act, resolve_mode, set_mode, shutdown,
     status_string, weight_sf_bytes,
 )

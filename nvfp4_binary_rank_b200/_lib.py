@@ -39,6 +39,7 @@ SIGNATURES = {
     "biloco_set_mode": (_I, [_I]),
     "biloco_resolve_mode": (_I, [_I, _I, _I, _I]),
     "biloco_last_error": (_I, [_P]),
+    "biloco_selftest_wait_timeout": (_I, [_P]),
     "biloco_status_string": (ctypes.c_char_p, [_I]),
     "biloco_gemm_kernel_count": (_I, [_I, _I, _I, _I]),
     "biloco_shutdown": (None, []),
@@ -182,6 +183,12 @@ def set_mode(mode: int):
 
 def resolve_mode(M: int, N: int, K: int, r: int) -> int:
     return int(load().biloco_resolve_mode(M, N, K, r))
+
+
+def selftest_wait_timeout(stream=None):
+    """Launch the bounded-wait self test (about 1 s on the GPU); biloco_last_error
+    on the same stream then reports BILOCO_ERR_TIMEOUT."""
+    _check("biloco_selftest_wait_timeout", load().biloco_selftest_wait_timeout(_stream(stream)))
 
 
 def last_error(stream=None) -> int:

@@ -235,6 +235,16 @@ int biloco_gemm(const void* x_bf16, const uint8_t* W_fp4, const uint8_t* W_sf, c
   return run_gemm(a, reinterpret_cast<cudaStream_t>(stream));
 }
 
+int biloco_selftest_wait_timeout(biloco_stream_t stream) {
+  int d = check_device();
+  if (d) return d;
+  ScratchNeed need = {16, 16, 16, 16, 16, 2};
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  Scratch* sc = get_scratch(s, need);
+  if (!sc) return BILOCO_ERR_NOMEM;
+  return launch_wait_timeout(sc->status, s) == cudaSuccess ? BILOCO_OK : BILOCO_ERR_CUDA;
+}
+
 int biloco_set_mode(int mode) {
   if (mode != BILOCO_MODE_AUTO && mode != BILOCO_MODE_SHARED_Z && mode != BILOCO_MODE_LOCAL_Z)
     return BILOCO_ERR_ARG;

@@ -536,7 +536,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
               float v[16];
               bf16x16_to_f32(lo[e], hi[e], v);
               uint2 codes;
-              const uint32_t s = quant_act_block(v, codes);
+              const uint32_t s = quant_act_block_fast(v, codes);
               const int j = blk * 8;
               *reinterpret_cast<uint2*>(smem + L::kB + k * kBN * 128 + m * 128 +
                                         ((((j >> 4) ^ (m & 7)) << 4) | (j & 15))) = codes;

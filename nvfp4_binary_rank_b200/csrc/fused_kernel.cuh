@@ -324,7 +324,7 @@ __device__ __forceinline__ void quant_chunk(const uint16_t* xb, int mcnt, int nw
     float v[16];
     bf16x16_to_f32(src[0], src[1], v);
     uint2 codes;
-    const uint32_t s = quant_act_block(v, codes);
+    const uint32_t s = quant_act_block_fast(v, codes);
     const int j = blk * 8;
     *reinterpret_cast<uint2*>(btile + m * 128 + ((((j >> 4) ^ (m & 7)) << 4) | (j & 15))) = codes;
     sfb[(blk >> 2) * 512 + (m & 31) * 16 + ((m >> 5) & 3) * 4 + (blk & 3)] = static_cast<uint8_t>(s);

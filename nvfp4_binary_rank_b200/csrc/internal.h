@@ -42,6 +42,7 @@ cudaError_t launch_prep_act(const uint16_t* x, int M, int K, uint8_t* codes, uin
 cudaError_t launch_pack_weight(const float* R, int N, int K, uint8_t* W_fp4, uint8_t* W_sf,
                                float* gscale, cudaStream_t s);
 cudaError_t launch_pack_signs(const float* S, int rows, int cols, uint32_t* bits, cudaStream_t s);
+cudaError_t launch_wait_timeout(int* status, cudaStream_t s);
 
 struct GemmArgs {
   const uint16_t* x;

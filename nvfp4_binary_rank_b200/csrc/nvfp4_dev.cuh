@@ -89,21 +89,33 @@ __device__ __forceinline__ uint32_t e2m1_code_bf16(float v, const E2M1Thresholds
   return (c != 0 && v < 0.0f) ? (c | 8u) : c;
 }
 
-// Activation block (no tensor scale): s = E4M3(amax / 6), codes = E2M1(x / s).
-// Inputs are BF16 values, so the division-free rounding above applies.
-__device__ __forceinline__ uint32_t quant_act_block(const float (&v)[16], uint2& codes) {
+// RN_FP32(v / S) without a division instruction, by Markstein's correction of a
+// reciprocal-based quotient (P. Markstein, "Computation of elementary functions
+// on the IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1), 1990, Thm. 8):
+// with y = RN(1/S), q0 = RN(v y) and the exact remainder r = v - S q0 (one FMA),
+// RN(q0 + r y) equals RN(v / S) in round-to-nearest when y is correctly rounded
+// and nothing overflows or underflows.  Here |v| < 2^16 and S >= 2^-9.
+__device__ __forceinline__ float div_rn_by(float v, float S, float y) {
+  const float q0 = __fmul_rn(v, y);
+  const float r = __fmaf_rn(-S, q0, v);
+  return __fmaf_rn(r, y, q0);
+}
+
+// Activation block (no tensor scale), quotient by Markstein's correction and the
+// hardware E2M1 conversion (nearest, ties to even, saturating): the same codes as
+// the definition E2M1(RN(x / s)).
+__device__ __forceinline__ uint32_t quant_act_block_fast(const float (&v)[16], uint2& codes) {
   const float t = __fdiv_rn(amax16(v), 6.0f);
   const uint32_t s = e4m3_from_f32(t);
   const float S = e4m3_to_f32(s);
-  const E2M1Thresholds th = e2m1_thresholds(S);
   codes = make_uint2(0u, 0u);
+  if (S != 0.0f) {
+    const float y = __frcp_rn(S);
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    codes.x |= (e2m1_code_bf16(v[2 * j], th, S == 0.0f) | (e2m1_code_bf16(v[2 * j + 1], th, S == 0.0f) << 4))
-               << (8 * j);
-    codes.y |= (e2m1_code_bf16(v[8 + 2 * j], th, S == 0.0f) |
-                (e2m1_code_bf16(v[8 + 2 * j + 1], th, S == 0.0f) << 4))
-               << (8 * j);
+    for (int j = 0; j < 4; ++j) {
+      codes.x |= e2m1x2(div_rn_by(v[2 * j], S, y), div_rn_by(v[2 * j + 1], S, y)) << (8 * j);
+      codes.y |= e2m1x2(div_rn_by(v[8 + 2 * j], S, y), div_rn_by(v[8 + 2 * j + 1], S, y)) << (8 * j);
+    }
   }
   return s;
 }

@@ -33,7 +33,7 @@ quant_act_rowmajor_kernel(const uint16_t* __restrict__ x, int M, int K, uint8_t*
   float v[16];
   load_bf16_block(x, K, m, b, v);
   uint2 c;
-  const uint32_t s = quant_act_block(v, c);
+  const uint32_t s = quant_act_block_fast(v, c);
   *reinterpret_cast<uint2*>(codes + static_cast<size_t>(m) * (K / 2) + b * 8) = c;
   sf[static_cast<size_t>(m) * nb + b] = static_cast<uint8_t>(s);
 }
@@ -51,7 +51,7 @@ prep_act_kernel(const uint16_t* __restrict__ x, int M, int K, uint8_t* __restric
   float v[16];
   load_bf16_block(x, K, m, b, v);
   uint2 c;
-  const uint32_t s = quant_act_block(v, c);
+  const uint32_t s = quant_act_block_fast(v, c);
   *reinterpret_cast<uint2*>(codes + static_cast<size_t>(m) * (K / 2) + b * 8) = c;
   sf_atoms[sf_atom_offset(static_cast<uint32_t>(m), static_cast<uint32_t>(b))] = static_cast<uint8_t>(s);
 }
@@ -153,6 +153,26 @@ cudaError_t launch_pack_weight(const float* R, int N, int K, uint8_t* W_fp4, uin
   gscale_kernel<<<1, 1, 0, s>>>(gscale);
   const long long nblk = static_cast<long long>(N) * ((K + 255) / 256) * 16;
   quant_weight_kernel<<<grid_for(nblk), kQuantThreads, 0, s>>>(R, N, K, gscale, W_fp4, W_sf);
+  return cudaGetLastError();
+}
+
+// Failure-path self test: one warp waits, through the same bounded mbarrier wait
+// the GEMM kernels use, on a phase nothing will complete.  The wait gives up after
+// its wall-clock limit, and the kernel records the timeout in `status` and returns.
+__global__ void wait_timeout_kernel(int* status) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && !mbar_wait(smem_u32(&bar), 0, &abort_flag)) record_error(status, kDevErrTimeout);
+}
+
+cudaError_t launch_wait_timeout(int* status, cudaStream_t s) {
+  wait_timeout_kernel<<<1, 32, 0, s>>>(status);
   return cudaGetLastError();
 }
 
