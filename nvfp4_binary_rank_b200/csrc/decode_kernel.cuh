@@ -122,6 +122,20 @@ struct Layout {
   static_assert(kAlloc <= 232448, "shared memory budget");
 };
 
+// One z value's two BF16 parts into the global tile image of the U side's B
+// operand: chunk i / 64 of kUN rows x 128 bytes, element i % 64 of row m (high)
+// and row MC + m (low), 128-byte swizzle (16-byte piece j of row q at j ^ (q & 7)).
+__device__ __forceinline__ void store_ztile(uint8_t* tiles, int kUN, int MC, int m, int i, __nv_bfloat16 hi,
+                                            __nv_bfloat16 lo) {
+  const int c = i >> 6, byte = (i & 63) * 2;
+  uint8_t* tile = tiles + static_cast<size_t>(c) * kUN * 128;
+  const int rl = MC + m;
+  *reinterpret_cast<uint16_t*>(tile + m * 128 + ((((byte >> 4) ^ (m & 7)) << 4) | (byte & 15))) =
+      __bfloat16_as_ushort(hi);
+  *reinterpret_cast<uint16_t*>(tile + rl * 128 + ((((byte >> 4) ^ (rl & 7)) << 4) | (byte & 15))) =
+      __bfloat16_as_ushort(lo);
+}
+
 // V-side word loop of one rank group: lane l takes element 32 w + l of every
 // word w this warp handles; acc[m][i] collects sum_k s_ik x[m][k].  Inputs that
 // the previous kernel of the stream may have written are read through L2
@@ -507,7 +521,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
 
     // ---- 1. quantise the activation chunks of every unit of this CTA
     {
-      constexpr int kQB = 4;                            // blocks per thread per round
+      constexpr int kQB = (MC <= 2) ? 4 : 8;            // blocks per thread per round
       const int per_unit = p.M * 16;
       const int items = nunits * per_unit;
       for (int base = 0; base < items; base += kAluThreads * kQB) {
@@ -597,9 +611,28 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
           float sum = 0.0f;
 #pragma unroll
           for (int w = 0; w < kAluWarps; ++w) sum += vred[w * kV + m * kRankGroup + i];
-          p.z[static_cast<size_t>(m) * p.rpad + ig + i] = __fmul_rn(__ldcg(p.alpha + ig + i), sum);
+          const float zv = __fmul_rn(__ldcg(p.alpha + ig + i), sum);
+          if constexpr (Cfg<MC>::kTensorU) {
+            // straight into the U side's B tiles: BF16 high part in row m, the BF16
+            // rounding of the rest in row MC + m (128-byte swizzled rows)
+            const __nv_bfloat16 hi = __float2bfloat16_rn(zv);
+            const __nv_bfloat16 lo = __float2bfloat16_rn(zv - __bfloat162float(hi));
+            store_ztile(p.ztiles, Layout<MC>::kUN, MC, m, ig + i, hi, lo);
+          } else {
+            p.z[static_cast<size_t>(m) * p.rpad + ig + i] = zv;
+          }
         }
         named_barrier(kBarAlu, kAluThreads);
+      }
+      if constexpr (Cfg<MC>::kTensorU) {
+        // the CTA holding the last ranks clears the tiles' tail past r
+        if (i1 == p.r) {
+          const int tail = ((p.r + kUChunk - 1) / kUChunk) * kUChunk;
+          for (int idx = tid; idx < p.M * (tail - p.r); idx += kAluThreads) {
+            const int m = idx / (tail - p.r), i = p.r + idx - m * (tail - p.r);
+            store_ztile(p.ztiles, Layout<MC>::kUN, MC, m, i, __float2bfloat16_rn(0.0f), __float2bfloat16_rn(0.0f));
+          }
+        }
       }
       named_barrier(kBarAlu, kAluThreads);
       if (tid == 0) red_add_release_gpu(p.z_ready, 1u);   // covers the slice the CTA wrote
@@ -643,44 +676,24 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
               fail(ctl);
               ok = false;
             }
-            uint4* zt4 = reinterpret_cast<uint4*>(smem + L::kUZ);
-            for (int idx = tid; idx < nuc * L::kUN * 8; idx += kAluThreads) zt4[idx] = make_uint4(0u, 0u, 0u, 0u);
-            named_barrier(kBarAlu, kAluThreads);
-            const int items = nuc * p.M * 32;             // (chunk, row, rank pair)
-            constexpr int kZB = 4;
-            for (int base = 0; base < items; base += kAluThreads * kZB) {
-              float2 zv[kZB];
-  #pragma unroll
-              for (int e = 0; e < kZB; ++e) {
-                const int idx = base + e * kAluThreads + tid;
-                zv[e] = make_float2(0.0f, 0.0f);
-                if (idx < items) {
-                  const int c = idx / (p.M * 32), rem = idx - c * p.M * 32, m = rem >> 5, qq = rem & 31;
-                  const int i = c * kUChunk + 2 * qq;
-                  if (i < p.r) {                           // i even and rpad even: i + 1 < rpad
-                    const float2 v = __ldcg(reinterpret_cast<const float2*>(p.z + static_cast<size_t>(m) * p.rpad + i));
-                    zv[e].x = v.x;
-                    zv[e].y = (i + 1 < p.r) ? v.y : 0.0f;
-                  }
+            // the B tiles were written in their final layout by the CTAs that computed
+            // z: copy them (rows past 2 M only feed output columns nobody reads)
+            {
+              uint4* zt4 = reinterpret_cast<uint4*>(smem + L::kUZ);
+              const uint4* src = reinterpret_cast<const uint4*>(p.ztiles);
+              constexpr int kZR = 8;
+              const int n16 = nuc * L::kUN * 8;
+              for (int base = 0; base < n16; base += kAluThreads * kZR) {
+                uint4 t4[kZR];
+#pragma unroll
+                for (int e = 0; e < kZR; ++e) {
+                  const int idx = base + e * kAluThreads + tid;
+                  t4[e] = (idx < n16) ? __ldcg(src + idx) : make_uint4(0u, 0u, 0u, 0u);
                 }
-              }
-  #pragma unroll
-              for (int e = 0; e < kZB; ++e) {
-                const int idx = base + e * kAluThreads + tid;
-                if (idx < items) {
-                  const int c = idx / (p.M * 32), rem = idx - c * p.M * 32, m = rem >> 5, qq = rem & 31;
-                  const __nv_bfloat16 h0 = __float2bfloat16_rn(zv[e].x), h1 = __float2bfloat16_rn(zv[e].y);
-                  const __nv_bfloat16 l0 = __float2bfloat16_rn(zv[e].x - __bfloat162float(h0));
-                  const __nv_bfloat16 l1 = __float2bfloat16_rn(zv[e].y - __bfloat162float(h1));
-                  const uint32_t hi = static_cast<uint32_t>(__bfloat16_as_ushort(h0)) |
-                                      (static_cast<uint32_t>(__bfloat16_as_ushort(h1)) << 16);
-                  const uint32_t lo = static_cast<uint32_t>(__bfloat16_as_ushort(l0)) |
-                                      (static_cast<uint32_t>(__bfloat16_as_ushort(l1)) << 16);
-                  const int byte = 4 * qq;
-                  uint8_t* tile = smem + L::kUZ + c * L::kUN * 128;
-                  *reinterpret_cast<uint32_t*>(tile + m * 128 + ((((byte >> 4) ^ (m & 7)) << 4) | (byte & 15))) = hi;
-                  const int ml = MC + m;
-                  *reinterpret_cast<uint32_t*>(tile + ml * 128 + ((((byte >> 4) ^ (ml & 7)) << 4) | (byte & 15))) = lo;
+#pragma unroll
+                for (int e = 0; e < kZR; ++e) {
+                  const int idx = base + e * kAluThreads + tid;
+                  if (idx < n16) zt4[idx] = t4[e];
                 }
               }
             }

@@ -15,7 +15,8 @@ struct DecodeParams {
   const uint16_t* x;       // [M][K] BF16
   uint16_t* y;             // [M][N] BF16
   float* z;                // [M][rpad] scratch: z = alpha . (V^T x)
-  float* slots;            // [2 G][8][128] scratch: split-K partials
+  uint8_t* ztiles;         // [16][32][128 B] scratch: z as BF16 high/low MMA tiles (4+ rows)
+  float* slots;            // [2 G][16][128] scratch: split-K partials
   uint32_t* z_ready;       // CTAs that published their z slice
   uint32_t* z_seen;        // CTAs done with z_ready (the last one resets both)
   uint32_t* tickets;       // [T] split-K arrivals per weight tile

@@ -136,7 +136,7 @@ GemmPlan plan_gemm(const GemmArgs& a) {
   if (p.decode) {
     need.act_fp4 = 16;
     need.act_sf = 16;
-    need.zpart = 16;
+    need.zpart = 16 * 32 * 128;                 // the decode kernel's z tiles
     need.zfin = r ? static_cast<size_t>(M) * p.rpad * 4 : 16;
     need.slots = static_cast<size_t>(2 * p.G) * kDecodeMaxRows * kTileRows * 4;
     need.counter_words = 2 + 2 * static_cast<size_t>(p.T);
@@ -179,6 +179,7 @@ int launch_gemm(const GemmArgs& a, const GemmPlan& p, const Scratch& scr, cudaSt
     dp.x = a.x;
     dp.y = a.y;
     dp.z = sc->zfin;
+    dp.ztiles = reinterpret_cast<uint8_t*>(sc->zpart);
     dp.slots = sc->slots;
     dp.z_ready = sc->counters;
     dp.z_seen = sc->counters + 1;
