@@ -136,6 +136,68 @@ __device__ __forceinline__ void store_ztile(uint8_t* tiles, int kUN, int MC, int
       __bfloat16_as_ushort(lo);
 }
 
+// V side for classes of 8+ rows.  Every warp owns two activation rows, row0 and
+// row0 + MC / 2, and walks the blocks of 256 K elements numbered kb0, kb0 + kbs, ..;
+// lane l takes elements 8 l .. 8 l + 7 of a block with one 16-byte load per row, and
+// the matching byte of the block's sign words (word 8 kb + l / 4, bits 8 (l % 4) ..).
+// Loads run three blocks ahead through a register ring.  Each lane returns its
+// partial sums acc[j][i] for row row0 + j MC / 2 and rank ig + i.
+template <int MC, int kRankGroup = Cfg<MC>::kRankGroup>
+__device__ __forceinline__ void vside_rows(const DecodeParams& p, int ig, int nr, int row0, int kb0, int kbs,
+                                           int lane, float (&acc)[2][kRankGroup]) {
+  constexpr int RPW = 2;
+  const int nkb = (p.K + 255) / 256;
+#pragma unroll
+  for (int j = 0; j < RPW; ++j)
+#pragma unroll
+    for (int i = 0; i < kRankGroup; ++i) acc[j][i] = 0.0f;
+  struct Stage {
+    uint4 x[RPW];
+    uint32_t v[kRankGroup];
+  };
+  auto load = [&](int kb, Stage& st) {
+    const int k0 = kb * 256 + lane * 8;
+    const bool kin = kb < nkb && k0 < p.K;
+#pragma unroll
+    for (int j = 0; j < RPW; ++j) {
+      const int m = row0 + (MC / 2) * j;
+      st.x[j] = (kin && m < p.M) ? __ldcg(reinterpret_cast<const uint4*>(p.x + static_cast<size_t>(m) * p.K + k0))
+                                 : make_uint4(0u, 0u, 0u, 0u);
+    }
+    const int w = kb * 8 + (lane >> 2);
+#pragma unroll
+    for (int i = 0; i < kRankGroup; ++i)
+      st.v[i] = (kin && i < nr) ? __ldcg(p.Vbits + static_cast<size_t>(ig + i) * p.KW + w) : 0u;
+  };
+  Stage s0, s1, s2;
+  load(kb0, s0);
+  load(kb0 + kbs, s1);
+  load(kb0 + 2 * kbs, s2);
+  const uint32_t bshift = 8u * static_cast<uint32_t>(lane & 3);
+#pragma unroll 1
+  for (int kb = kb0; kb < nkb; kb += kbs) {
+    const Stage cur = s0;
+    s0 = s1;
+    s1 = s2;
+    load(kb + 3 * kbs, s2);
+#pragma unroll
+    for (int i = 0; i < kRankGroup; ++i) {
+      const uint32_t bits = cur.v[i] >> bshift;            // this lane's 8 sign bits
+#pragma unroll
+      for (int j = 0; j < RPW; ++j) {
+        const uint32_t w4[4] = {cur.x[j].x, cur.x[j].y, cur.x[j].z, cur.x[j].w};
+        float sum = 0.0f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const uint32_t xb = (e & 1) ? (w4[e >> 1] & 0xFFFF0000u) : (w4[e >> 1] << 16);
+          sum += __uint_as_float(xb ^ ((bits << (31 - e)) & 0x80000000u));
+        }
+        acc[j][i] += sum;
+      }
+    }
+  }
+}
+
 // V-side word loop of one rank group: lane l takes element 32 w + l of every
 // word w this warp handles; acc[m][i] collects sum_k s_ik x[m][k].  Inputs that
 // the previous kernel of the stream may have written are read through L2
@@ -589,40 +651,99 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
       // ---- 2. V side: z for this CTA's rank slice over the whole of K
       constexpr int kV = MC * kRankGroup;
       float* vred = reinterpret_cast<float*>(smem + L::kVRed);
-      for (int ig = i0; ig < i1; ig += kRankGroup) {
-        const int nr = min(kRankGroup, i1 - ig);
-        float acc[MC][kRankGroup];
-        vside_group<MC>(p, ig, nr, a, lane, acc);
-        float flat[kV];
-#pragma unroll
-        for (int m = 0; m < MC; ++m)
-#pragma unroll
-          for (int i = 0; i < kRankGroup; ++i) flat[m * kRankGroup + i] = acc[m][i];
-        warp_reduce_scatter<kV>(flat, lane);
-        if constexpr (kV >= 32) {
-#pragma unroll
-          for (int j = 0; j < kV / 32; ++j) vred[a * kV + reduce_out_index<kV>(lane, j)] = flat[j];
-        } else {
-          if ((lane & (32 / kV - 1)) == 0) vred[a * kV + reduce_out_index<kV>(lane, 0)] = flat[0];
-        }
-        named_barrier(kBarAlu, kAluThreads);
-        if (tid < p.M * nr) {
-          const int m = tid / nr, i = tid - m * nr;
-          float sum = 0.0f;
-#pragma unroll
-          for (int w = 0; w < kAluWarps; ++w) sum += vred[w * kV + m * kRankGroup + i];
-          const float zv = __fmul_rn(__ldcg(p.alpha + ig + i), sum);
-          if constexpr (Cfg<MC>::kTensorU) {
-            // straight into the U side's B tiles: BF16 high part in row m, the BF16
-            // rounding of the rest in row MC + m (128-byte swizzled rows)
-            const __nv_bfloat16 hi = __float2bfloat16_rn(zv);
-            const __nv_bfloat16 lo = __float2bfloat16_rn(zv - __bfloat162float(hi));
-            store_ztile(p.ztiles, Layout<MC>::kUN, MC, m, ig + i, hi, lo);
+      if constexpr (MC >= 8) {
+        // two rows per warp: with 16 rows warp a owns rows a and a + 8 over all of K;
+        // with 8, warps a and a + 4 share rows a and a + 4 (even and odd K blocks) and
+        // the second hands its sums to the first through shared memory
+        constexpr int KS = 16 / MC, RH = MC / 2;
+        const int row0 = a % RH, kb0 = a / RH;
+        for (int ig = i0; ig < i1; ig += kRankGroup) {
+          const int nr = min(kRankGroup, i1 - ig);
+          float acc[2][kRankGroup];
+          if (row0 < p.M) {
+            vside_rows<MC>(p, ig, nr, row0, kb0, KS, lane, acc);
           } else {
-            p.z[static_cast<size_t>(m) * p.rpad + ig + i] = zv;
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+#pragma unroll
+              for (int i = 0; i < kRankGroup; ++i) acc[j][i] = 0.0f;
           }
+#pragma unroll
+          for (int j = 0; j < 2; ++j)
+#pragma unroll
+            for (int i = 0; i < kRankGroup; ++i)
+#pragma unroll
+              for (int o = 16; o >= 1; o >>= 1) acc[j][i] += __shfl_xor_sync(0xffffffffu, acc[j][i], o);
+          if constexpr (KS == 2) {
+            if (kb0 == 1 && lane == 0) {
+#pragma unroll
+              for (int j = 0; j < 2; ++j)
+#pragma unroll
+                for (int i = 0; i < kRankGroup; ++i) vred[(row0 * 2 + j) * kRankGroup + i] = acc[j][i];
+            }
+            named_barrier(kBarAlu, kAluThreads);
+            if (kb0 == 0) {
+#pragma unroll
+              for (int j = 0; j < 2; ++j)
+#pragma unroll
+                for (int i = 0; i < kRankGroup; ++i) acc[j][i] += vred[(row0 * 2 + j) * kRankGroup + i];
+            }
+          }
+          if (kb0 == 0 && lane == 0) {
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              const int m = row0 + RH * j;
+              if (m < p.M) {
+#pragma unroll
+                for (int i = 0; i < kRankGroup; ++i) {
+                  if (i < nr) {
+                    const float zv = __fmul_rn(__ldcg(p.alpha + ig + i), acc[j][i]);
+                    const __nv_bfloat16 hi = __float2bfloat16_rn(zv);
+                    const __nv_bfloat16 lo = __float2bfloat16_rn(zv - __bfloat162float(hi));
+                    store_ztile(p.ztiles, Layout<MC>::kUN, MC, m, ig + i, hi, lo);
+                  }
+                }
+              }
+            }
+          }
+          if constexpr (KS == 2) named_barrier(kBarAlu, kAluThreads);   // vred reused next group
         }
-        named_barrier(kBarAlu, kAluThreads);
+      } else {
+        for (int ig = i0; ig < i1; ig += kRankGroup) {
+          const int nr = min(kRankGroup, i1 - ig);
+          float acc[MC][kRankGroup];
+          vside_group<MC>(p, ig, nr, a, lane, acc);
+          float flat[kV];
+  #pragma unroll
+          for (int m = 0; m < MC; ++m)
+  #pragma unroll
+            for (int i = 0; i < kRankGroup; ++i) flat[m * kRankGroup + i] = acc[m][i];
+          warp_reduce_scatter<kV>(flat, lane);
+          if constexpr (kV >= 32) {
+  #pragma unroll
+            for (int j = 0; j < kV / 32; ++j) vred[a * kV + reduce_out_index<kV>(lane, j)] = flat[j];
+          } else {
+            if ((lane & (32 / kV - 1)) == 0) vred[a * kV + reduce_out_index<kV>(lane, 0)] = flat[0];
+          }
+          named_barrier(kBarAlu, kAluThreads);
+          if (tid < p.M * nr) {
+            const int m = tid / nr, i = tid - m * nr;
+            float sum = 0.0f;
+  #pragma unroll
+            for (int w = 0; w < kAluWarps; ++w) sum += vred[w * kV + m * kRankGroup + i];
+            const float zv = __fmul_rn(__ldcg(p.alpha + ig + i), sum);
+            if constexpr (Cfg<MC>::kTensorU) {
+              // straight into the U side's B tiles: BF16 high part in row m, the BF16
+              // rounding of the rest in row MC + m (128-byte swizzled rows)
+              const __nv_bfloat16 hi = __float2bfloat16_rn(zv);
+              const __nv_bfloat16 lo = __float2bfloat16_rn(zv - __bfloat162float(hi));
+              store_ztile(p.ztiles, Layout<MC>::kUN, MC, m, ig + i, hi, lo);
+            } else {
+              p.z[static_cast<size_t>(m) * p.rpad + ig + i] = zv;
+            }
+          }
+          named_barrier(kBarAlu, kAluThreads);
+        }
       }
       if constexpr (Cfg<MC>::kTensorU) {
         // the CTA holding the last ranks clears the tiles' tail past r
