@@ -1,5 +1,5 @@
 // Fused NVFP4 GEMM + binary-sign low-rank correction for decode batches
-// (M <= 8 activation rows) on one B200 (sm_100a).
+// (M <= 16 activation rows) on one B200 (sm_100a).
 //
 //   y[m, n] = g * sum_k FP4(x)[m, k] FP4(R)[n, k]  +  sum_i U[n, i] z[m, i],
 //   z[m, i] = alpha_i * sum_k V[k, i] x[m, k]
@@ -40,6 +40,7 @@
 #include <cuda_runtime.h>
 
 #include "../../include/biloco.h"
+#include "decode_launch.h"
 #include "decode_params.h"
 #include "nvfp4_dev.cuh"
 #include "ptx.cuh"
@@ -86,11 +87,23 @@ constexpr int kBarFin2 = 4;               // epilogue + CUDA cores: correction r
 template <int MC>
 struct Cfg {
   static constexpr int kStages = (MC >= 16) ? 4 : 6;
-  static constexpr int kRankGroup = (MC >= 16) ? 4 : 8;
+  static constexpr int kRankGroup = (MC >= 4) ? 4 : 8;     // ranks per V-side pass (register bound)
   // U side on the tensor cores from 4 rows up; below, per-thread sign-adds are
   // cheaper than the chunked MMA chain (measured on B200)
   static constexpr bool kTensorU = MC >= 4;
+  // from 8 rows up the CTAs quantise the activation once between them (a global
+  // image behind an arrival counter) instead of each CTA quantising the chunks of
+  // all its units
+  static constexpr bool kGlobalQ = MC >= 8;
 };
+
+// Global activation image (8+ rows): per 256-element K chunk, the 16 x 128 B code
+// rows exactly as the operand cache holds them (128-byte swizzle), then 256 B of
+// block scales, 64 B per 64-element K step (row m at byte 4 m, block b of the step
+// at byte b).
+constexpr int kQImgCodes = kBN * 128;
+constexpr int kQImgBytes = kQImgCodes + 256;
+static_assert(kQImgBytes == kDecodeQImgBytes, "activation image size differs from the host's");
 
 template <int MC>
 struct Layout {
@@ -136,16 +149,35 @@ __device__ __forceinline__ void store_ztile(uint8_t* tiles, int kUN, int MC, int
       __bfloat16_as_ushort(lo);
 }
 
-// V side for classes of 8+ rows.  Every warp owns two activation rows, row0 and
-// row0 + MC / 2, and walks the blocks of 256 K elements numbered kb0, kb0 + kbs, ..;
-// lane l takes elements 8 l .. 8 l + 7 of a block with one 16-byte load per row, and
-// the matching byte of the block's sign words (word 8 kb + l / 4, bits 8 (l % 4) ..).
-// Loads run three blocks ahead through a register ring.  Each lane returns its
-// partial sums acc[j][i] for row row0 + j MC / 2 and rank ig + i.
+// V side: how the 8 CUDA-core warps share the rows and the K blocks (256
+// elements each).  With 8+ rows a warp owns two rows, row0 and row0 + MC / 2, and
+// 16 / MC warps split K between them; with fewer rows every warp owns all of them
+// and the 8 warps split K.
+template <int MC>
+struct VSplit {
+  static constexpr int kRows = (MC >= 8) ? 2 : MC;          // rows per warp
+  static constexpr int kStep = (MC >= 8) ? MC / 2 : 1;      // row stride within a warp
+  static constexpr int kSplit = (MC >= 8) ? 16 / MC : kAluWarps;   // warps per row (K split)
+  __device__ static int row0(int a) { return (MC >= 8) ? a % (MC / 2) : 0; }
+  __device__ static int kb0(int a) { return (MC >= 8) ? a / (MC / 2) : a; }
+  // warp q (< kSplit) of those holding row m, and the row's slot in that warp
+  __device__ static int warp_of(int m, int q) { return (MC >= 8) ? m % (MC / 2) + (MC / 2) * q : q; }
+  __device__ static int slot_of(int m) { return (MC >= 8) ? m / (MC / 2) : m; }
+};
+
+// V-side partial sums of one warp: rows row0 + j kStep (j < kRows), the K blocks
+// kb0, kb0 + kSplit, ..; lane l takes elements 8 l .. 8 l + 7 of a block with one
+// 16-byte load per row, and the matching byte of the block's sign words (word
+// 8 kb + l / 4, bits 8 (l % 4) ..).  Loads run three blocks ahead.  Each lane
+// returns acc[j][i] for row row0 + j kStep and rank ig + i (ranks i >= nr are
+// left at zero).  Inputs that the previous kernel of the stream may have written
+// are read through L2 (ld.global.cg), never through a possibly stale L1 line.
 template <int MC, int kRankGroup = Cfg<MC>::kRankGroup>
-__device__ __forceinline__ void vside_rows(const DecodeParams& p, int ig, int nr, int row0, int kb0, int kbs,
-                                           int lane, float (&acc)[2][kRankGroup]) {
-  constexpr int RPW = 2;
+__device__ __forceinline__ void vside_rows(const DecodeParams& p, int ig, int nr, int a, int lane,
+                                           float (&acc)[VSplit<MC>::kRows][kRankGroup]) {
+  using VS = VSplit<MC>;
+  constexpr int RPW = VS::kRows, kbs = VS::kSplit;
+  const int row0 = VS::row0(a), kb0 = VS::kb0(a);
   const int nkb = (p.K + 255) / 256;
 #pragma unroll
   for (int j = 0; j < RPW; ++j)
@@ -160,7 +192,7 @@ __device__ __forceinline__ void vside_rows(const DecodeParams& p, int ig, int nr
     const bool kin = kb < nkb && k0 < p.K;
 #pragma unroll
     for (int j = 0; j < RPW; ++j) {
-      const int m = row0 + (MC / 2) * j;
+      const int m = row0 + VS::kStep * j;
       st.x[j] = (kin && m < p.M) ? __ldcg(reinterpret_cast<const uint4*>(p.x + static_cast<size_t>(m) * p.K + k0))
                                  : make_uint4(0u, 0u, 0u, 0u);
     }
@@ -169,74 +201,36 @@ __device__ __forceinline__ void vside_rows(const DecodeParams& p, int ig, int nr
     for (int i = 0; i < kRankGroup; ++i)
       st.v[i] = (kin && i < nr) ? __ldcg(p.Vbits + static_cast<size_t>(ig + i) * p.KW + w) : 0u;
   };
-  Stage s0, s1, s2;
-  load(kb0, s0);
-  load(kb0 + kbs, s1);
-  load(kb0 + 2 * kbs, s2);
+  // a ring of three stages indexed statically (the loop body is unrolled three
+  // times), so that no register copy waits on the load issued last
+  Stage st[3];
+#pragma unroll
+  for (int q = 0; q < 3; ++q) load(kb0 + q * kbs, st[q]);
   const uint32_t bshift = 8u * static_cast<uint32_t>(lane & 3);
 #pragma unroll 1
-  for (int kb = kb0; kb < nkb; kb += kbs) {
-    const Stage cur = s0;
-    s0 = s1;
-    s1 = s2;
-    load(kb + 3 * kbs, s2);
+  for (int t = kb0; t < nkb; t += 3 * kbs) {
 #pragma unroll
-    for (int i = 0; i < kRankGroup; ++i) {
-      const uint32_t bits = cur.v[i] >> bshift;            // this lane's 8 sign bits
+    for (int q = 0; q < 3; ++q) {
+      if (t + q * kbs < nkb) {
 #pragma unroll
-      for (int j = 0; j < RPW; ++j) {
-        const uint32_t w4[4] = {cur.x[j].x, cur.x[j].y, cur.x[j].z, cur.x[j].w};
-        float sum = 0.0f;
+        for (int i = 0; i < kRankGroup; ++i) {
+          if (i < nr) {
+            const uint32_t bits = st[q].v[i] >> bshift;      // this lane's 8 sign bits
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const uint32_t xb = (e & 1) ? (w4[e >> 1] & 0xFFFF0000u) : (w4[e >> 1] << 16);
-          sum += __uint_as_float(xb ^ ((bits << (31 - e)) & 0x80000000u));
+            for (int j = 0; j < RPW; ++j) {
+              const uint32_t w4[4] = {st[q].x[j].x, st[q].x[j].y, st[q].x[j].z, st[q].x[j].w};
+              float sum = 0.0f;
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const uint32_t xb = (e & 1) ? (w4[e >> 1] & 0xFFFF0000u) : (w4[e >> 1] << 16);
+                sum += __uint_as_float(xb ^ ((bits << (31 - e)) & 0x80000000u));
+              }
+              acc[j][i] += sum;
+            }
+          }
         }
-        acc[j][i] += sum;
       }
-    }
-  }
-}
-
-// V-side word loop of one rank group: lane l takes element 32 w + l of every
-// word w this warp handles; acc[m][i] collects sum_k s_ik x[m][k].  Inputs that
-// the previous kernel of the stream may have written are read through L2
-// (ld.global.cg), never through a possibly stale L1 line.
-template <int MC, int kRankGroup = Cfg<MC>::kRankGroup>
-__device__ __forceinline__ void vside_group(const DecodeParams& p, int ig, int nr, int a, int lane,
-                                            float (&acc)[MC][kRankGroup]) {
-#pragma unroll
-  for (int m = 0; m < MC; ++m)
-#pragma unroll
-    for (int i = 0; i < kRankGroup; ++i) acc[m][i] = 0.0f;
-  const uint32_t lane_shift = 31u - static_cast<uint32_t>(lane);
-  const uint32_t* vrow = p.Vbits + static_cast<size_t>(ig) * p.KW;
-  constexpr int kUnroll = (MC >= 16) ? 1 : ((MC >= 8) ? 2 : 4);   // words per warp per load round
-  for (int w0 = a; w0 < p.KW; w0 += kAluWarps * kUnroll) {
-    uint32_t xs[kUnroll][MC];
-    uint32_t vw[kUnroll][kRankGroup];
-#pragma unroll
-    for (int q = 0; q < kUnroll; ++q) {
-      const int w = w0 + q * kAluWarps;
-      const bool in = w < p.KW;
-#pragma unroll
-      for (int m = 0; m < MC; ++m)
-        xs[q][m] = (in && m < p.M) ? static_cast<uint32_t>(__ldcg(p.x + static_cast<size_t>(m) * p.K +
-                                                                   static_cast<size_t>(w) * 32 + lane))
-                                   : 0u;
-#pragma unroll
-      for (int i = 0; i < kRankGroup; ++i)
-        vw[q][i] = (in && i < nr) ? __ldcg(vrow + static_cast<size_t>(i) * p.KW + w) : 0u;
-    }
-#pragma unroll
-    for (int q = 0; q < kUnroll; ++q) {
-#pragma unroll
-      for (int i = 0; i < kRankGroup; ++i) {
-        const uint32_t sgn = (vw[q][i] << lane_shift) & 0x80000000u;
-#pragma unroll
-        for (int m = 0; m < MC; ++m)
-          acc[m][i] += __uint_as_float((xs[q][m] << 16) ^ sgn);
-      }
+      load(t + (q + 3) * kbs, st[q]);
     }
   }
 }
@@ -583,41 +577,106 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
 
     // ---- 1. quantise the activation chunks of every unit of this CTA
     {
-      constexpr int kQB = (MC <= 2) ? 4 : 8;            // blocks per thread per round
-      const int per_unit = p.M * 16;
-      const int items = nunits * per_unit;
-      for (int base = 0; base < items; base += kAluThreads * kQB) {
-        uint4 lo[kQB], hi[kQB];
-#pragma unroll
-        for (int e = 0; e < kQB; ++e) {
-          const int idx = base + e * kAluThreads + tid;
-          lo[e] = hi[e] = make_uint4(0u, 0u, 0u, 0u);
-          if (idx < items) {
-            const int k = idx / per_unit, rem = idx - k * per_unit, m = rem >> 4, blk = rem & 15;
-            const int kk = ((u0 + k) % p.KC) * kUnitK + blk * 16;
-            if (kk < p.K) {
-              const uint4* src = reinterpret_cast<const uint4*>(p.x + static_cast<size_t>(m) * p.K + kk);
-              lo[e] = __ldcg(src);
-              hi[e] = __ldcg(src + 1);
+      if constexpr (!Cfg<MC>::kGlobalQ) {
+        constexpr int kQB = (MC <= 2) ? 4 : 8;            // blocks per thread per round
+        const int per_unit = p.M * 16;
+        const int items = nunits * per_unit;
+        for (int base = 0; base < items; base += kAluThreads * kQB) {
+          uint4 lo[kQB], hi[kQB];
+  #pragma unroll
+          for (int e = 0; e < kQB; ++e) {
+            const int idx = base + e * kAluThreads + tid;
+            lo[e] = hi[e] = make_uint4(0u, 0u, 0u, 0u);
+            if (idx < items) {
+              const int k = idx / per_unit, rem = idx - k * per_unit, m = rem >> 4, blk = rem & 15;
+              const int kk = ((u0 + k) % p.KC) * kUnitK + blk * 16;
+              if (kk < p.K) {
+                const uint4* src = reinterpret_cast<const uint4*>(p.x + static_cast<size_t>(m) * p.K + kk);
+                lo[e] = __ldcg(src);
+                hi[e] = __ldcg(src + 1);
+              }
+            }
+          }
+  #pragma unroll
+          for (int e = 0; e < kQB; ++e) {
+            const int idx = base + e * kAluThreads + tid;
+            if (idx < items) {
+              const int k = idx / per_unit, rem = idx - k * per_unit, m = rem >> 4, blk = rem & 15;
+              const int kk = ((u0 + k) % p.KC) * kUnitK + blk * 16;
+              if (kk < p.K) {
+                float v[16];
+                bf16x16_to_f32(lo[e], hi[e], v);
+                uint2 codes;
+                const uint32_t s = quant_act_block_fast(v, codes);
+                const int j = blk * 8;
+                *reinterpret_cast<uint2*>(smem + L::kB + k * kBN * 128 + m * 128 +
+                                          ((((j >> 4) ^ (m & 7)) << 4) | (j & 15))) = codes;
+                smem[L::kSFB + k * 512 + (blk >> 2) * 128 + m * 4 + (blk & 3)] = static_cast<uint8_t>(s);
+              }
             }
           }
         }
-#pragma unroll
-        for (int e = 0; e < kQB; ++e) {
-          const int idx = base + e * kAluThreads + tid;
-          if (idx < items) {
-            const int k = idx / per_unit, rem = idx - k * per_unit, m = rem >> 4, blk = rem & 15;
-            const int kk = ((u0 + k) % p.KC) * kUnitK + blk * 16;
-            if (kk < p.K) {
-              float v[16];
-              bf16x16_to_f32(lo[e], hi[e], v);
-              uint2 codes;
-              const uint32_t s = quant_act_block_fast(v, codes);
-              const int j = blk * 8;
-              *reinterpret_cast<uint2*>(smem + L::kB + k * kBN * 128 + m * 128 +
-                                        ((((j >> 4) ^ (m & 7)) << 4) | (j & 15))) = codes;
-              smem[L::kSFB + k * 512 + (blk >> 2) * 128 + m * 4 + (blk & 3)] = static_cast<uint8_t>(s);
+      } else {
+        // CTA g quantises items [g I / G, (g + 1) I / G) of the I = 16 KC blocks of
+        // 16 rows x 16 elements (rows >= M and blocks past K as zero codes and scales)
+        // into the global image, publishes them, and after every CTA has done so
+        // copies the chunks of its units into the operand cache
+        const uint32_t items = static_cast<uint32_t>(p.KC) * 256u;
+        const uint32_t q0 = static_cast<uint32_t>(static_cast<uint64_t>(g) * items / static_cast<uint32_t>(p.G));
+        const uint32_t q1 = static_cast<uint32_t>(static_cast<uint64_t>(g + 1) * items / static_cast<uint32_t>(p.G));
+        for (uint32_t it = q0 + static_cast<uint32_t>(tid); it < q1; it += kAluThreads) {
+          const int kc = static_cast<int>(it >> 8), m = static_cast<int>((it >> 4) & 15u), blk = static_cast<int>(it & 15u);
+          const int kk = kc * kUnitK + blk * 16;
+          uint2 codes = make_uint2(0u, 0u);
+          uint32_t sc = 0u;
+          if (m < p.M && kk < p.K) {
+            const uint4* src = reinterpret_cast<const uint4*>(p.x + static_cast<size_t>(m) * p.K + kk);
+            const uint4 lo = __ldcg(src), hi = __ldcg(src + 1);
+            float v[16];
+            bf16x16_to_f32(lo, hi, v);
+            sc = quant_act_block_fast(v, codes);
+          }
+          uint8_t* img = p.xq + static_cast<size_t>(kc) * kQImgBytes;
+          const int j = blk * 8;
+          *reinterpret_cast<uint2*>(img + m * 128 + ((((j >> 4) ^ (m & 7)) << 4) | (j & 15))) = codes;
+          img[kQImgCodes + (blk >> 2) * 64 + m * 4 + (blk & 3)] = static_cast<uint8_t>(sc);
+        }
+        named_barrier(kBarAlu, kAluThreads);
+        bool okq = true;
+        if (tid == 0) {
+          red_add_release_gpu(p.q_ready, 1u);              // covers the items the CTA wrote
+          okq = spin_until_geq(p.q_ready, static_cast<uint32_t>(p.G), ctl);
+          if (okq) {
+            // the last CTA past the wait resets both counters for the next call
+            const uint32_t old = atomicAdd(p.q_seen, 1u);
+            if (old == static_cast<uint32_t>(p.G - 1)) {
+              atomicExch(p.q_ready, 0u);
+              atomicExch(p.q_seen, 0u);
             }
+          }
+        }
+        if (named_barrier_or(kBarAlu, kAluThreads, !okq)) fail(ctl);
+        // one round of 16-byte loads: 144 per unit (128 of codes, 16 of scales)
+        constexpr int kPer = kQImgBytes / 16;
+        constexpr int kLd = (kMaxUnits * kPer + kAluThreads - 1) / kAluThreads;
+        uint4 buf[kLd];
+#pragma unroll
+        for (int e = 0; e < kLd; ++e) {
+          const int idx = e * kAluThreads + tid;
+          if (idx < nunits * kPer) {
+            const int k = idx / kPer, o = idx - k * kPer;
+            const int kc = (u0 + k) % p.KC;
+            buf[e] = __ldcg(reinterpret_cast<const uint4*>(p.xq + static_cast<size_t>(kc) * kQImgBytes) + o);
+          }
+        }
+#pragma unroll
+        for (int e = 0; e < kLd; ++e) {
+          const int idx = e * kAluThreads + tid;
+          if (idx < nunits * kPer) {
+            const int k = idx / kPer, o = idx - k * kPer;
+            uint8_t* dst = (o < 128) ? smem + L::kB + k * kBN * 128 + o * 16
+                                     : smem + L::kSFB + k * 512 + ((o - 128) >> 2) * 128 + ((o - 128) & 3) * 16;
+            *reinterpret_cast<uint4*>(dst) = buf[e];
           }
         }
       }
@@ -649,100 +708,62 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
 
     if (p.r > 0) {
       // ---- 2. V side: z for this CTA's rank slice over the whole of K
-      constexpr int kV = MC * kRankGroup;
       float* vred = reinterpret_cast<float*>(smem + L::kVRed);
-      if constexpr (MC >= 8) {
-        // two rows per warp: with 16 rows warp a owns rows a and a + 8 over all of K;
-        // with 8, warps a and a + 4 share rows a and a + 4 (even and odd K blocks) and
-        // the second hands its sums to the first through shared memory
-        constexpr int KS = 16 / MC, RH = MC / 2;
-        const int row0 = a % RH, kb0 = a / RH;
+      {
+        // every warp sums its rows over its K blocks; the warps that split one row's
+        // K then add their sums through shared memory
+        using VS = VSplit<MC>;
+        constexpr int RPW = VS::kRows;
         for (int ig = i0; ig < i1; ig += kRankGroup) {
           const int nr = min(kRankGroup, i1 - ig);
-          float acc[2][kRankGroup];
-          if (row0 < p.M) {
-            vside_rows<MC>(p, ig, nr, row0, kb0, KS, lane, acc);
-          } else {
+          float acc[RPW][kRankGroup];
+          vside_rows<MC>(p, ig, nr, a, lane, acc);
 #pragma unroll
-            for (int j = 0; j < 2; ++j)
-#pragma unroll
-              for (int i = 0; i < kRankGroup; ++i) acc[j][i] = 0.0f;
-          }
-#pragma unroll
-          for (int j = 0; j < 2; ++j)
+          for (int j = 0; j < RPW; ++j)
 #pragma unroll
             for (int i = 0; i < kRankGroup; ++i)
 #pragma unroll
               for (int o = 16; o >= 1; o >>= 1) acc[j][i] += __shfl_xor_sync(0xffffffffu, acc[j][i], o);
-          if constexpr (KS == 2) {
-            if (kb0 == 1 && lane == 0) {
-#pragma unroll
-              for (int j = 0; j < 2; ++j)
-#pragma unroll
-                for (int i = 0; i < kRankGroup; ++i) vred[(row0 * 2 + j) * kRankGroup + i] = acc[j][i];
-            }
-            named_barrier(kBarAlu, kAluThreads);
-            if (kb0 == 0) {
-#pragma unroll
-              for (int j = 0; j < 2; ++j)
-#pragma unroll
-                for (int i = 0; i < kRankGroup; ++i) acc[j][i] += vred[(row0 * 2 + j) * kRankGroup + i];
-            }
-          }
-          if (kb0 == 0 && lane == 0) {
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-              const int m = row0 + RH * j;
-              if (m < p.M) {
-#pragma unroll
-                for (int i = 0; i < kRankGroup; ++i) {
-                  if (i < nr) {
-                    const float zv = __fmul_rn(__ldcg(p.alpha + ig + i), acc[j][i]);
-                    const __nv_bfloat16 hi = __float2bfloat16_rn(zv);
-                    const __nv_bfloat16 lo = __float2bfloat16_rn(zv - __bfloat162float(hi));
-                    store_ztile(p.ztiles, Layout<MC>::kUN, MC, m, ig + i, hi, lo);
-                  }
-                }
-              }
-            }
-          }
-          if constexpr (KS == 2) named_barrier(kBarAlu, kAluThreads);   // vred reused next group
-        }
-      } else {
-        for (int ig = i0; ig < i1; ig += kRankGroup) {
-          const int nr = min(kRankGroup, i1 - ig);
-          float acc[MC][kRankGroup];
-          vside_group<MC>(p, ig, nr, a, lane, acc);
-          float flat[kV];
-  #pragma unroll
-          for (int m = 0; m < MC; ++m)
-  #pragma unroll
-            for (int i = 0; i < kRankGroup; ++i) flat[m * kRankGroup + i] = acc[m][i];
-          warp_reduce_scatter<kV>(flat, lane);
-          if constexpr (kV >= 32) {
-  #pragma unroll
-            for (int j = 0; j < kV / 32; ++j) vred[a * kV + reduce_out_index<kV>(lane, j)] = flat[j];
-          } else {
-            if ((lane & (32 / kV - 1)) == 0) vred[a * kV + reduce_out_index<kV>(lane, 0)] = flat[0];
-          }
-          named_barrier(kBarAlu, kAluThreads);
-          if (tid < p.M * nr) {
-            const int m = tid / nr, i = tid - m * nr;
-            float sum = 0.0f;
-  #pragma unroll
-            for (int w = 0; w < kAluWarps; ++w) sum += vred[w * kV + m * kRankGroup + i];
+          // z for row m, rank ig + i: straight into the U side's B tiles (BF16 high
+          // part in row m, the BF16 rounding of the rest in row MC + m, 128-byte
+          // swizzled rows) or into the fp32 z scratch
+          auto put = [&](int m, int i, float sum) {
             const float zv = __fmul_rn(__ldcg(p.alpha + ig + i), sum);
             if constexpr (Cfg<MC>::kTensorU) {
-              // straight into the U side's B tiles: BF16 high part in row m, the BF16
-              // rounding of the rest in row MC + m (128-byte swizzled rows)
               const __nv_bfloat16 hi = __float2bfloat16_rn(zv);
               const __nv_bfloat16 lo = __float2bfloat16_rn(zv - __bfloat162float(hi));
               store_ztile(p.ztiles, Layout<MC>::kUN, MC, m, ig + i, hi, lo);
             } else {
               p.z[static_cast<size_t>(m) * p.rpad + ig + i] = zv;
             }
+          };
+          if constexpr (VS::kSplit == 1) {
+            if (lane == 0) {
+#pragma unroll
+              for (int j = 0; j < RPW; ++j) {
+                const int m = VS::row0(a) + VS::kStep * j;
+#pragma unroll
+                for (int i = 0; i < kRankGroup; ++i)
+                  if (m < p.M && i < nr) put(m, i, acc[j][i]);
+              }
+            }
+          } else {
+            if (lane == 0) {
+#pragma unroll
+              for (int j = 0; j < RPW; ++j)
+#pragma unroll
+                for (int i = 0; i < kRankGroup; ++i) vred[(a * RPW + j) * kRankGroup + i] = acc[j][i];
+            }
+            named_barrier(kBarAlu, kAluThreads);
+            if (tid < p.M * nr) {
+              const int m = tid / nr, i = tid - m * nr, j = VS::slot_of(m);
+              float sum = 0.0f;
+#pragma unroll
+              for (int q = 0; q < VS::kSplit; ++q) sum += vred[(VS::warp_of(m, q) * RPW + j) * kRankGroup + i];
+              put(m, i, sum);
+            }
+            named_barrier(kBarAlu, kAluThreads);           // vred is reused by the next group
           }
-          named_barrier(kBarAlu, kAluThreads);
         }
       }
       if constexpr (Cfg<MC>::kTensorU) {

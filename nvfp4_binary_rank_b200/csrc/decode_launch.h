@@ -12,6 +12,9 @@ namespace biloco {
 // Units of 128 weight rows x 256 K elements one CTA of the decode kernel can hold.
 constexpr int kDecodeMaxUnits = 16;
 constexpr int kDecodeMaxRows = 16;
+// Bytes per 256-element K chunk of the kernel's quantised activation image
+// (16 rows x 128 B of codes, 256 B of scales).
+constexpr int kDecodeQImgBytes = 16 * 128 + 256;
 
 cudaError_t launch_decode_1(const CUtensorMap& tw, const DecodeParams& dp, cudaStream_t s);
 cudaError_t launch_decode_2(const CUtensorMap& tw, const DecodeParams& dp, cudaStream_t s);

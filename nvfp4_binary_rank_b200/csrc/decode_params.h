@@ -1,4 +1,4 @@
-// Parameters of the decode-batch kernel (M <= 8), shared by its host launcher
+// Parameters of the decode-batch kernel (M <= 16), shared by its host launcher
 // and the kernel.
 #pragma once
 
@@ -16,10 +16,13 @@ struct DecodeParams {
   uint16_t* y;             // [M][N] BF16
   float* z;                // [M][rpad] scratch: z = alpha . (V^T x)
   uint8_t* ztiles;         // [16][32][128 B] scratch: z as BF16 high/low MMA tiles (4+ rows)
+  uint8_t* xq;             // [KC][2304 B] scratch: quantised activation image (8+ rows)
   float* slots;            // [2 G][16][128] scratch: split-K partials
   uint32_t* z_ready;       // CTAs that published their z slice
   uint32_t* z_seen;        // CTAs done with z_ready (the last one resets both)
   uint32_t* tickets;       // [T] split-K arrivals per weight tile
+  uint32_t* q_ready;       // CTAs that published their part of the activation image
+  uint32_t* q_seen;        // CTAs done with q_ready (the last one resets both)
   int* status;             // first device-side error
   int M, N, K, r;
   int KC, T, U, G, KW, RW, rpad;

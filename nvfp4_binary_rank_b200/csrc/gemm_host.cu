@@ -134,12 +134,12 @@ GemmPlan plan_gemm(const GemmArgs& a) {
 
   ScratchNeed& need = p.need;
   if (p.decode) {
-    need.act_fp4 = 16;
+    need.act_fp4 = static_cast<size_t>(p.KC) * kDecodeQImgBytes;   // the activation image (8+ rows)
     need.act_sf = 16;
     need.zpart = 16 * 32 * 128;                 // the decode kernel's z tiles
     need.zfin = r ? static_cast<size_t>(M) * p.rpad * 4 : 16;
     need.slots = static_cast<size_t>(2 * p.G) * kDecodeMaxRows * kTileRows * 4;
-    need.counter_words = 2 + 2 * static_cast<size_t>(p.T);
+    need.counter_words = 4 + 2 * static_cast<size_t>(p.T);   // z, tickets, q counters
     return p;
   }
   need.act_fp4 = p.inq ? 16 : static_cast<size_t>(M) * K / 2;
@@ -184,6 +184,9 @@ int launch_gemm(const GemmArgs& a, const GemmPlan& p, const Scratch& scr, cudaSt
     dp.z_ready = sc->counters;
     dp.z_seen = sc->counters + 1;
     dp.tickets = sc->counters + 2;
+    dp.q_ready = sc->counters + 2 + T;
+    dp.q_seen = sc->counters + 3 + T;
+    dp.xq = sc->act_fp4;
     dp.status = sc->status;
     dp.M = M; dp.N = N; dp.K = K; dp.r = r;
     dp.KC = KC; dp.T = T; dp.U = U; dp.G = G; dp.KW = KW;

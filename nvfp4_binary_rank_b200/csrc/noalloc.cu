@@ -34,7 +34,7 @@ namespace {
 constexpr size_t kCap = BILOCO_NOALLOC_SCRATCH_BYTES;
 constexpr size_t kStatusOff = 0;
 constexpr size_t kCounterOff = 256;
-constexpr size_t kCounterWordsMax = 2 + 2 * static_cast<size_t>(BILOCO_NOALLOC_MAX_N / 128);
+constexpr size_t kCounterWordsMax = 4 + 2 * static_cast<size_t>(BILOCO_NOALLOC_MAX_N / 128);
 constexpr size_t kDataOff = (kCounterOff + kCounterWordsMax * 4 + 255) / 256 * 256;
 constexpr size_t kSfChunkBytes = 2048;        // scale atoms of one 256-element chunk of K
 
