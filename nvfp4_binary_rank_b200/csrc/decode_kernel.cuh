@@ -87,7 +87,10 @@ constexpr int kBarFin2 = 4;               // epilogue + CUDA cores: correction r
 template <int MC>
 struct Cfg {
   static constexpr int kStages = (MC >= 16) ? 4 : 6;
-  static constexpr int kRankGroup = (MC >= 4) ? 4 : 8;     // ranks per V-side pass (register bound)
+  static constexpr int kRankGroup = 4;                     // ranks per V-side pass
+  // V-side load ring depth (blocks in flight per warp); below 8 rows a warp walks
+  // only two or three K blocks
+  static constexpr int kVStages = (MC >= 8) ? 3 : 2;
   // U side on the tensor cores from 4 rows up; below, per-thread sign-adds are
   // cheaper than the chunked MMA chain (measured on B200)
   static constexpr bool kTensorU = MC >= 4;
@@ -125,7 +128,7 @@ struct Layout {
                                                  : kCorr + 2 * MC * kTileRows * 4;
   static constexpr int kVRed = kUEnd;                                  // [8][MC * ranks] floats
   static constexpr int kBar = kVRed + kAluWarps * MC * kRankGroup * 4;
-  static constexpr int kNumBars = 2 * kStages + 10;
+  static constexpr int kNumBars = 2 * kStages + 12;
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kFinFlags = kMisc + 32;                         // [kMaxUnits + 1] ints
   static constexpr int kTotal = kFinFlags + (kMaxUnits + 1) * 4;
@@ -150,28 +153,31 @@ __device__ __forceinline__ void store_ztile(uint8_t* tiles, int kUN, int MC, int
 }
 
 // V side: how the 8 CUDA-core warps share the rows and the K blocks (256
-// elements each).  With 8+ rows a warp owns two rows, row0 and row0 + MC / 2, and
-// 16 / MC warps split K between them; with fewer rows every warp owns all of them
-// and the 8 warps split K.
+// elements each).  A warp owns kRows = min(MC, 4) rows, row0, row0 + kStep, ..
+// (kStep = MC / kRows row groups), and the kSplit = 8 / kStep warps of one row
+// group split K between them.
 template <int MC>
 struct VSplit {
-  static constexpr int kRows = (MC >= 8) ? 2 : MC;          // rows per warp
-  static constexpr int kStep = (MC >= 8) ? MC / 2 : 1;      // row stride within a warp
-  static constexpr int kSplit = (MC >= 8) ? 16 / MC : kAluWarps;   // warps per row (K split)
-  __device__ static int row0(int a) { return (MC >= 8) ? a % (MC / 2) : 0; }
-  __device__ static int kb0(int a) { return (MC >= 8) ? a / (MC / 2) : a; }
+  static constexpr int kRows = (MC >= 4) ? 4 : MC;          // rows per warp
+  static constexpr int kStep = MC / kRows;                  // row groups
+  static constexpr int kSplit = kAluWarps / kStep;          // warps per row group (K split)
+  __device__ static int row0(int a) { return a % kStep; }
+  __device__ static int kb0(int a) { return a / kStep; }
   // warp q (< kSplit) of those holding row m, and the row's slot in that warp
-  __device__ static int warp_of(int m, int q) { return (MC >= 8) ? m % (MC / 2) + (MC / 2) * q : q; }
-  __device__ static int slot_of(int m) { return (MC >= 8) ? m / (MC / 2) : m; }
+  __device__ static int warp_of(int m, int q) { return m % kStep + kStep * q; }
+  __device__ static int slot_of(int m) { return m / kStep; }
 };
 
 // V-side partial sums of one warp: rows row0 + j kStep (j < kRows), the K blocks
 // kb0, kb0 + kSplit, ..; lane l takes elements 8 l .. 8 l + 7 of a block with one
 // 16-byte load per row, and the matching byte of the block's sign words (word
-// 8 kb + l / 4, bits 8 (l % 4) ..).  Loads run three blocks ahead.  Each lane
-// returns acc[j][i] for row row0 + j kStep and rank ig + i (ranks i >= nr are
-// left at zero).  Inputs that the previous kernel of the stream may have written
-// are read through L2 (ld.global.cg), never through a possibly stale L1 line.
+// 8 kb + l / 4, bits 8 (l % 4) ..).  Loads run kVStages blocks ahead.  The sign-adds
+// are packed FP32 FMAs with +-1.0 multipliers (exact products, one rounding per
+// add, as a plain add or subtract): one instruction covers an element pair, even
+// and odd elements in the two lanes of a pair accumulator.  Each lane returns
+// acc[j][i] for row row0 + j kStep and rank ig + i (ranks i >= nr are left at
+// zero).  Inputs that the previous kernel of the stream may have written are read
+// through L2 (ld.global.cg), never through a possibly stale L1 line.
 template <int MC, int kRankGroup = Cfg<MC>::kRankGroup>
 __device__ __forceinline__ void vside_rows(const DecodeParams& p, int ig, int nr, int a, int lane,
                                            float (&acc)[VSplit<MC>::kRows][kRankGroup]) {
@@ -179,10 +185,11 @@ __device__ __forceinline__ void vside_rows(const DecodeParams& p, int ig, int nr
   constexpr int RPW = VS::kRows, kbs = VS::kSplit;
   const int row0 = VS::row0(a), kb0 = VS::kb0(a);
   const int nkb = (p.K + 255) / 256;
+  uint64_t acc2[RPW][kRankGroup];
 #pragma unroll
   for (int j = 0; j < RPW; ++j)
 #pragma unroll
-    for (int i = 0; i < kRankGroup; ++i) acc[j][i] = 0.0f;
+    for (int i = 0; i < kRankGroup; ++i) acc2[j][i] = 0ull;
   struct Stage {
     uint4 x[RPW];
     uint32_t v[kRankGroup];
@@ -201,38 +208,46 @@ __device__ __forceinline__ void vside_rows(const DecodeParams& p, int ig, int nr
     for (int i = 0; i < kRankGroup; ++i)
       st.v[i] = (kin && i < nr) ? __ldcg(p.Vbits + static_cast<size_t>(ig + i) * p.KW + w) : 0u;
   };
-  // a ring of three stages indexed statically (the loop body is unrolled three
-  // times), so that no register copy waits on the load issued last
-  Stage st[3];
+  // a ring of kVStages stages indexed statically (the loop body is unrolled that
+  // many times), so that no register copy waits on the load issued last
+  constexpr int NS = Cfg<MC>::kVStages;
+  Stage st[NS];
 #pragma unroll
-  for (int q = 0; q < 3; ++q) load(kb0 + q * kbs, st[q]);
+  for (int q = 0; q < NS; ++q) load(kb0 + q * kbs, st[q]);
   const uint32_t bshift = 8u * static_cast<uint32_t>(lane & 3);
 #pragma unroll 1
-  for (int t = kb0; t < nkb; t += 3 * kbs) {
+  for (int t = kb0; t < nkb; t += NS * kbs) {
 #pragma unroll
-    for (int q = 0; q < 3; ++q) {
+    for (int q = 0; q < NS; ++q) {
       if (t + q * kbs < nkb) {
 #pragma unroll
-        for (int i = 0; i < kRankGroup; ++i) {
-          if (i < nr) {
-            const uint32_t bits = st[q].v[i] >> bshift;      // this lane's 8 sign bits
+        for (int pr = 0; pr < 4; ++pr) {               // element pair 2 pr, 2 pr + 1
+          uint64_t x2[RPW];
 #pragma unroll
-            for (int j = 0; j < RPW; ++j) {
-              const uint32_t w4[4] = {st[q].x[j].x, st[q].x[j].y, st[q].x[j].z, st[q].x[j].w};
-              float sum = 0.0f;
+          for (int j = 0; j < RPW; ++j) {
+            const uint32_t w = (pr == 0) ? st[q].x[j].x : (pr == 1) ? st[q].x[j].y : (pr == 2) ? st[q].x[j].z : st[q].x[j].w;
+            x2[j] = f32x2_pack(w << 16, w & 0xFFFF0000u);
+          }
 #pragma unroll
-              for (int e = 0; e < 8; ++e) {
-                const uint32_t xb = (e & 1) ? (w4[e >> 1] & 0xFFFF0000u) : (w4[e >> 1] << 16);
-                sum += __uint_as_float(xb ^ ((bits << (31 - e)) & 0x80000000u));
-              }
-              acc[j][i] += sum;
+          for (int i = 0; i < kRankGroup; ++i) {
+            if (i < nr) {
+              const uint32_t bits = st[q].v[i] >> bshift;    // this lane's 8 sign bits
+              const uint32_t s0 = ((bits << (31 - 2 * pr)) & 0x80000000u) | 0x3F800000u;
+              const uint32_t s1 = ((bits << (30 - 2 * pr)) & 0x80000000u) | 0x3F800000u;
+              const uint64_t s2 = f32x2_pack(s0, s1);
+#pragma unroll
+              for (int j = 0; j < RPW; ++j) acc2[j][i] = f32x2_fma(x2[j], s2, acc2[j][i]);
             }
           }
         }
       }
-      load(t + (q + 3) * kbs, st[q]);
+      load(t + (q + NS) * kbs, st[q]);
     }
   }
+#pragma unroll
+  for (int j = 0; j < RPW; ++j)
+#pragma unroll
+    for (int i = 0; i < kRankGroup; ++i) acc[j][i] = f32x2_sum(acc2[j][i]);
 }
 
 template <int MC>
@@ -255,6 +270,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
   const uint32_t done_bar = smem_u32(&bars[2 * kStages + 6]);
   auto ubuf_bar = [&](int b) { return smem_u32(&bars[2 * kStages + 7 + b]); };
   const uint32_t ud_bar = smem_u32(&bars[2 * kStages + 9]);
+  auto ufull_bar = [&](int b) { return smem_u32(&bars[2 * kStages + 10 + b]); };
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
   volatile int* epi_last = reinterpret_cast<volatile int*>(smem + L::kMisc + 8);
@@ -283,6 +299,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
     mbar_init(ubuf_bar(0), 1);
     mbar_init(ubuf_bar(1), 1);
     mbar_init(ud_bar, 1);
+    mbar_init(ufull_bar(0), kAluThreads);
+    mbar_init(ufull_bar(1), kAluThreads);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -578,12 +596,15 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
     // ---- 1. quantise the activation chunks of every unit of this CTA
     {
       if constexpr (!Cfg<MC>::kGlobalQ) {
-        constexpr int kQB = (MC <= 2) ? 4 : 8;            // blocks per thread per round
+        // two blocks per thread per round, the loop rolled (the quantiser is long
+        // straight-line code; unrolled deeper it would crowd the instruction cache)
+        constexpr int kQB = 2;
         const int per_unit = p.M * 16;
         const int items = nunits * per_unit;
+#pragma unroll 1
         for (int base = 0; base < items; base += kAluThreads * kQB) {
           uint4 lo[kQB], hi[kQB];
-  #pragma unroll
+#pragma unroll
           for (int e = 0; e < kQB; ++e) {
             const int idx = base + e * kAluThreads + tid;
             lo[e] = hi[e] = make_uint4(0u, 0u, 0u, 0u);
@@ -597,7 +618,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
               }
             }
           }
-  #pragma unroll
+#pragma unroll
           for (int e = 0; e < kQB; ++e) {
             const int idx = base + e * kAluThreads + tid;
             if (idx < items) {
@@ -737,33 +758,23 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
               p.z[static_cast<size_t>(m) * p.rpad + ig + i] = zv;
             }
           };
-          if constexpr (VS::kSplit == 1) {
-            if (lane == 0) {
+          // the warps of a row group add their sums through shared memory
+          static_assert(VS::kSplit > 1, "every row group splits K");
+          if (lane == 0) {
 #pragma unroll
-              for (int j = 0; j < RPW; ++j) {
-                const int m = VS::row0(a) + VS::kStep * j;
+            for (int j = 0; j < RPW; ++j)
 #pragma unroll
-                for (int i = 0; i < kRankGroup; ++i)
-                  if (m < p.M && i < nr) put(m, i, acc[j][i]);
-              }
-            }
-          } else {
-            if (lane == 0) {
-#pragma unroll
-              for (int j = 0; j < RPW; ++j)
-#pragma unroll
-                for (int i = 0; i < kRankGroup; ++i) vred[(a * RPW + j) * kRankGroup + i] = acc[j][i];
-            }
-            named_barrier(kBarAlu, kAluThreads);
-            if (tid < p.M * nr) {
-              const int m = tid / nr, i = tid - m * nr, j = VS::slot_of(m);
-              float sum = 0.0f;
-#pragma unroll
-              for (int q = 0; q < VS::kSplit; ++q) sum += vred[(VS::warp_of(m, q) * RPW + j) * kRankGroup + i];
-              put(m, i, sum);
-            }
-            named_barrier(kBarAlu, kAluThreads);           // vred is reused by the next group
+              for (int i = 0; i < kRankGroup; ++i) vred[(a * RPW + j) * kRankGroup + i] = acc[j][i];
           }
+          named_barrier(kBarAlu, kAluThreads);
+          if (tid < p.M * nr) {
+            const int m = tid / nr, i = tid - m * nr, j = VS::slot_of(m);
+            float sum = 0.0f;
+#pragma unroll
+            for (int q = 0; q < VS::kSplit; ++q) sum += vred[(VS::warp_of(m, q) * RPW + j) * kRankGroup + i];
+            put(m, i, sum);
+          }
+          named_barrier(kBarAlu, kAluThreads);             // vred is reused by the next group
         }
       }
       if constexpr (Cfg<MC>::kTensorU) {
@@ -844,21 +855,33 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
             ztiles = true;
           }
           if (seg >= 2) load_words(t_first + seg, uw1);    // segments past the second: load now
-  #pragma unroll
-          for (int c = 0; c < kUChunksMax; ++c) {
+          // chunk pairs in a rolled loop (fully unrolled, the body would make the
+          // kernel's code outgrow the instruction cache; the chunk's word is picked
+          // out of the registers by compare-and-select, so the word arrays stay in
+          // registers), the two A buffers alternating inside a pair.  No
+          // CTA-wide barrier per chunk: every thread arrives on the buffer's fill
+          // barrier after writing its piece; thread 0 alone waits for the fill, issues
+          // the chunk's MMAs and commits them to the buffer's free barrier, which the
+          // threads wait on before they write the buffer again.
+#pragma unroll 1
+          for (int c2 = 0; c2 < kUChunksMax; c2 += 2) {
+#pragma unroll
+          for (int buf = 0; buf < 2; ++buf) {
+            const int c = c2 + buf;
             if (c < nuc) {
-              const int buf = c & 1;
               int& uses = buf ? uses1 : uses0;
               if (uses > 0) {
                 // the MMAs that read this buffer last are done
                 bool okb = true;
-                if (tid == 0) okb = mbar_wait(ubuf_bar(buf), (uses - 1) & 1, abort_flag);
-                if (named_barrier_or(kBarAlu, kAluThreads, !okb)) {
+                if (lane == 0) okb = mbar_wait(ubuf_bar(buf), (uses - 1) & 1, abort_flag);
+                if (__shfl_sync(0xffffffffu, okb ? 1 : 0, 0) == 0) {
                   fail(ctl);
                   ok = false;
                 }
               }
-              const uint32_t word = (seg == 0) ? uw0[c] : uw1[c];
+              uint32_t word = 0u;
+  #pragma unroll
+              for (int e = 0; e < kUChunksMax; ++e) word = (e == c) ? ((seg == 0) ? uw0[e] : uw1[e]) : word;
               uint8_t* arow = smem + L::kUA + buf * (kTileRows * 128) + row * 128;
   #pragma unroll
               for (int k = 0; k < 4; ++k) {
@@ -872,18 +895,24 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
                 *reinterpret_cast<uint4*>(arow + ((piece ^ (row & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
               }
               fence_proxy_async_smem();
-              named_barrier(kBarAlu, kAluThreads);
+              mbar_arrive(ufull_bar(buf));
               if (tid == 0) {
-                tc_fence_after();
-                const uint64_t a_d = smem_desc(smem_u32(smem + L::kUA + buf * (kTileRows * 128)), 16, 1024, 2);
-                const uint64_t b_d = smem_desc(smem_u32(smem + L::kUZ + c * L::kUN * 128), 16, 1024, 2);
+                if (mbar_wait(ufull_bar(buf), uses & 1, abort_flag)) {
+                  tc_fence_after();
+                  const uint64_t a_d = smem_desc(smem_u32(smem + L::kUA + buf * (kTileRows * 128)), 16, 1024, 2);
+                  const uint64_t b_d = smem_desc(smem_u32(smem + L::kUZ + c * L::kUN * 128), 16, 1024, 2);
   #pragma unroll
-                for (int j = 0; j < 4; ++j)
-                  tc_mma_bf16(tmem + kUTmem, a_d + 2 * j, b_d + 2 * j, idesc_u, (c > 0 || j > 0) ? 1u : 0u);
-                tc_commit(ubuf_bar(buf));
+                  for (int j = 0; j < 4; ++j)
+                    tc_mma_bf16(tmem + kUTmem, a_d + 2 * j, b_d + 2 * j, idesc_u, (c > 0 || j > 0) ? 1u : 0u);
+                  tc_commit(ubuf_bar(buf));
+                } else {
+                  fail(ctl);
+                  ok = false;
+                }
               }
               ++uses;
             }
+          }
           }
           if (tid == 0) tc_commit(ud_bar);
           if (named_barrier_or(kBarFin2, kFinThreads, !ok)) {
@@ -915,6 +944,19 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
         float* zs = reinterpret_cast<float*>(smem + L::kZ);
         float* corr = reinterpret_cast<float*>(smem + L::kCorr);
         bool ok = true, staged = false;
+        // thread (row, half) sums ranks [32 wa, 32 wb) of weight row `row`; the sign
+        // words of the first two tiles are requested now, before z is complete
+        const int row = tid & (kTileRows - 1), half = tid >> 7;
+        const int wsplit = (p.RW + 1) >> 1;
+        const int wa = half ? wsplit : 0, wb = half ? p.RW : wsplit;
+        auto load_words = [&](int t, uint32_t (&uw)[16]) {
+          const uint32_t* ur = p.Ubits + (static_cast<size_t>(t) * kTileRows + row) * p.RW;
+  #pragma unroll
+          for (int w = 0; w < 16; ++w) uw[w] = (wa + w < wb) ? __ldcg(ur + wa + w) : 0u;
+        };
+        uint32_t uw0[16], uw1[16];
+        load_words(t_first, uw0);
+        if (nseg > 1) load_words(t_first + 1, uw1);
         for (int seg = 0; seg < nseg; ++seg) {
           if (named_barrier_or(kBarFin, kFinThreads, !ok)) {
             ok = false;
@@ -939,20 +981,14 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
             }
           }
           if (ok) {
-            const int row = tid & (kTileRows - 1), half = tid >> 7;
-            const int wsplit = (p.RW + 1) >> 1;
-            const int wa = half ? wsplit : 0, wb = half ? p.RW : wsplit;
-            const uint32_t* ur = p.Ubits + (static_cast<size_t>(t) * kTileRows + row) * p.RW;
-            uint32_t uw[16];
-  #pragma unroll
-            for (int w = 0; w < 16; ++w) uw[w] = (wa + w < wb) ? __ldcg(ur + wa + w) : 0u;
+            if (seg >= 2) load_words(t, uw1);            // segments past the second: load now
             float acc[MC];
   #pragma unroll
             for (int m = 0; m < MC; ++m) acc[m] = 0.0f;
             for (int w = 0; w < wb - wa; ++w) {
               uint32_t word = 0;
   #pragma unroll
-              for (int e = 0; e < 16; ++e) word = (e == w) ? uw[e] : word;
+              for (int e = 0; e < 16; ++e) word = (e == w) ? ((seg == 0) ? uw0[e] : uw1[e]) : word;
               const float* zw = zs + (wa + w) * 32;
   #pragma unroll
               for (int j4 = 0; j4 < 8; ++j4) {
