@@ -71,6 +71,8 @@ constexpr int kTmemCols = 512;
 constexpr int kSfbTmemBase = 32;
 constexpr int kSfaTmemBase = kSfbTmemBase + 16 * 16;
 constexpr int kUTmem = 384;
+constexpr int kVTmem = 448;               // V side on the tensor cores: 16 columns
+constexpr int kVAtoms = 3;                // K atoms (64 elements) per V-side MMA batch
 constexpr int kUChunk = 64;               // ranks per U-side MMA chunk (one 128-byte BF16 row)
 constexpr int kUChunksMax = 16;           // r <= 1024
 constexpr uint32_t kStageTx = kUnitBytesA + kSfBytes;
@@ -98,6 +100,10 @@ struct Cfg {
   // image behind an arrival counter) instead of each CTA quantising the chunks of
   // all its units
   static constexpr bool kGlobalQ = MC >= 8;
+  // with 16 rows the V side runs on the tensor cores, cut into pieces of 128 ranks
+  // x a slice of K, with the partial sums reduced across CTAs (with 8 the CUDA-core
+  // loop is faster, measured on B200)
+  static constexpr bool kTensorV = MC >= 16;
 };
 
 // Global activation image (8+ rows): per 256-element K chunk, the 16 x 128 B code
@@ -128,7 +134,7 @@ struct Layout {
                                                  : kCorr + 2 * MC * kTileRows * 4;
   static constexpr int kVRed = kUEnd;                                  // [8][MC * ranks] floats
   static constexpr int kBar = kVRed + kAluWarps * MC * kRankGroup * 4;
-  static constexpr int kNumBars = 2 * kStages + 12;
+  static constexpr int kNumBars = 2 * kStages + 13;
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kFinFlags = kMisc + 32;                         // [kMaxUnits + 1] ints
   static constexpr int kTotal = kFinFlags + (kMaxUnits + 1) * 4;
@@ -167,6 +173,24 @@ struct VSplit {
   __device__ static int warp_of(int m, int q) { return m % kStep + kStep * q; }
   __device__ static int slot_of(int m) { return m / kStep; }
 };
+
+// V-side partial sums of one warp: rows row0 + j kStep (j < kRows), the K blocks
+// kb0, kb0 + kSplit, ..; lane l takes elements 8 l .. 8 l + 7 of a block with one
+// 16-byte load per row, and the matching byte of the block's sign words (word
+// 8 kb + l / 4, bits 8 (l % 4) ..).  Loads run kVStages blocks ahead.  The sign-adds
+// are packed FP32 FMAs with +-1.0 multipliers (exact products, one rounding per
+// add, as a plain add or subtract): one instruction covers an element pair, even
+// and odd elements in the two lanes of a pair accumulator.  Each lane returns
+// acc[j][i] for row row0 + j kStep and rank ig + i (ranks i >= nr are left at
+// zero).  Inputs that the previous kernel of the stream may have written are read
+// through L2 (ld.global.cg), never through a possibly stale L1 line.
+// K slices per rank block of the tensor-core V side: one piece per CTA where there
+// are enough CTAs, at most 32 (the cross-CTA sum of a (rank, row) pair takes four
+// lanes x eight partial sums).
+constexpr int kVSliceMax = 32;
+__device__ __forceinline__ int vside_slices(const DecodeParams& p, int RB) {
+  return max(1, min(min(p.G / RB, p.K / 64), kVSliceMax));
+}
 
 // V-side partial sums of one warp: rows row0 + j kStep (j < kRows), the K blocks
 // kb0, kb0 + kSplit, ..; lane l takes elements 8 l .. 8 l + 7 of a block with one
@@ -271,6 +295,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
   auto ubuf_bar = [&](int b) { return smem_u32(&bars[2 * kStages + 7 + b]); };
   const uint32_t ud_bar = smem_u32(&bars[2 * kStages + 9]);
   auto ufull_bar = [&](int b) { return smem_u32(&bars[2 * kStages + 10 + b]); };
+  const uint32_t vmma_bar = smem_u32(&bars[2 * kStages + 12]);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
   volatile int* epi_last = reinterpret_cast<volatile int*>(smem + L::kMisc + 8);
@@ -301,6 +326,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
     mbar_init(ud_bar, 1);
     mbar_init(ufull_bar(0), kAluThreads);
     mbar_init(ufull_bar(1), kAluThreads);
+    mbar_init(vmma_bar, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -662,6 +688,108 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
           *reinterpret_cast<uint2*>(img + m * 128 + ((((j >> 4) ^ (m & 7)) << 4) | (j & 15))) = codes;
           img[kQImgCodes + (blk >> 2) * 64 + m * 4 + (blk & 3)] = static_cast<uint8_t>(sc);
         }
+        if constexpr (Cfg<MC>::kTensorV) {
+          if (p.r > 0) {
+            // ---- V side, part 1, on the tensor cores.  Piece (rb, s) = ranks
+            // [128 rb, 128 rb + 128) x K atoms [s KA / S, (s + 1) KA / S); CTA g takes
+            // pieces g, g + G, ..  For each, the partial sums
+            //   vpart[rb][s][m][i] = sum_{k in the slice} s_ik x[m][k]
+            // come from BF16 MMAs: A = the pieces' sign bits expanded to +-1 (exact,
+            // ranks >= r as zero rows), B = the activation rows (rows >= M zero), D in
+            // TMEM (lane = rank, column = row).  The buffers are the U side's, unused
+            // until z is complete.
+            const int RB = (p.r + kTileRows - 1) / kTileRows, KA = p.K / 64;
+            const int S = vside_slices(p, RB);
+            uint8_t* va = smem + L::kUA;                                  // [kVAtoms][128][128 B]
+            uint8_t* vbt = smem + L::kUA + kVAtoms * kTileRows * 128;     // [kVAtoms][16][128 B]
+            const int row = tid & (kTileRows - 1), half = tid >> 7;
+            const uint32_t idesc_v = (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(kBN >> 3) << 17) |
+                                     (static_cast<uint32_t>(kTileRows >> 4) << 24);
+            int vuses = 0;
+            for (int piece = g; piece < RB * S; piece += p.G) {
+              const int rb = piece / S, sl = piece - rb * S;
+              const int a0 = static_cast<int>(static_cast<int64_t>(sl) * KA / S);
+              const int a1 = static_cast<int>(static_cast<int64_t>(sl + 1) * KA / S);
+              const int rank = rb * kTileRows + row;
+              for (int b0 = a0; b0 < a1; b0 += kVAtoms) {
+                const int nb = min(kVAtoms, a1 - b0);
+                // requests first: this thread's sign words and activation pieces
+                uint32_t vw[kVAtoms];
+#pragma unroll
+                for (int j = 0; j < kVAtoms; ++j)
+                  vw[j] = (j < nb && rank < p.r) ? __ldcg(p.Vbits + static_cast<size_t>(rank) * p.KW + 2 * (b0 + j) + half)
+                                                 : 0u;
+                constexpr int kXL = (kVAtoms * kBN * 8 + kAluThreads - 1) / kAluThreads;
+                uint4 xv[kXL];
+#pragma unroll
+                for (int e = 0; e < kXL; ++e) {
+                  const int idx = e * kAluThreads + tid;
+                  const int j = idx >> 7, m = (idx >> 3) & 15, c = idx & 7;
+                  xv[e] = (j < nb && m < p.M)
+                              ? __ldcg(reinterpret_cast<const uint4*>(p.x + static_cast<size_t>(m) * p.K + 64 * (b0 + j) + 8 * c))
+                              : make_uint4(0u, 0u, 0u, 0u);
+                }
+#pragma unroll
+                for (int j = 0; j < kVAtoms; ++j) {
+                  if (j < nb) {
+                    uint8_t* arow = va + j * (kTileRows * 128) + row * 128;
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                      uint32_t pk[4];
+#pragma unroll
+                      for (int t2 = 0; t2 < 4; ++t2) {
+                        const int jb = 8 * k + 2 * t2;
+                        pk[t2] = (rank < p.r) ? (0x3F803F80u | (((vw[j] >> jb) & 1u) << 15) | (((vw[j] >> (jb + 1)) & 1u) << 31))
+                                              : 0u;
+                      }
+                      const int pc = 4 * half + k;
+                      *reinterpret_cast<uint4*>(arow + ((pc ^ (row & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    }
+                  }
+                }
+#pragma unroll
+                for (int e = 0; e < kXL; ++e) {
+                  const int idx = e * kAluThreads + tid;
+                  const int j = idx >> 7, m = (idx >> 3) & 15, c = idx & 7;
+                  if (j < nb) *reinterpret_cast<uint4*>(vbt + j * (kBN * 128) + m * 128 + ((c ^ (m & 7)) << 4)) = xv[e];
+                }
+                fence_proxy_async_smem();
+                named_barrier(kBarAlu, kAluThreads);
+                bool okv = true;
+                if (tid == 0) {
+                  tc_fence_after();
+                  const uint64_t a_d = smem_desc(smem_u32(va), 16, 1024, 2);
+                  const uint64_t b_d = smem_desc(smem_u32(vbt), 16, 1024, 2);
+                  for (int j = 0; j < nb; ++j)
+#pragma unroll
+                    for (int k4 = 0; k4 < 4; ++k4)
+                      tc_mma_bf16(tmem + kVTmem, a_d + static_cast<uint64_t>(j) * ((kTileRows * 128) >> 4) + 2 * k4,
+                                  b_d + static_cast<uint64_t>(j) * ((kBN * 128) >> 4) + 2 * k4, idesc_v,
+                                  (b0 > a0 || j > 0 || k4 > 0) ? 1u : 0u);
+                  tc_commit(vmma_bar);
+                  okv = mbar_wait(vmma_bar, vuses & 1, abort_flag);
+                }
+                ++vuses;
+                if (named_barrier_or(kBarAlu, kAluThreads, !okv)) fail(ctl);   // buffers free again
+              }
+              // the piece's partial sums: warps 0..3 of this group read the four lane
+              // quarters of the accumulator
+              tc_fence_after();
+              if (a < 4) {
+                const int quarter = warp & 3;
+                uint32_t v[16];
+                tmem_ld16(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + kVTmem, v);
+                tmem_wait_ld();
+                float* dst = p.vpart + static_cast<size_t>(rb * S + sl) * kBN * kTileRows + quarter * 32 + lane;
+#pragma unroll
+                for (int m = 0; m < kBN; ++m)
+                  if (m < p.M) dst[m * kTileRows] = __uint_as_float(v[m]);
+              }
+              tc_fence_before();
+              named_barrier(kBarAlu, kAluThreads);           // TMEM read before the next piece
+            }
+          }
+        }
         named_barrier(kBarAlu, kAluThreads);
         bool okq = true;
         if (tid == 0) {
@@ -730,51 +858,87 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
     if (p.r > 0) {
       // ---- 2. V side: z for this CTA's rank slice over the whole of K
       float* vred = reinterpret_cast<float*>(smem + L::kVRed);
-      {
-        // every warp sums its rows over its K blocks; the warps that split one row's
-        // K then add their sums through shared memory
-        using VS = VSplit<MC>;
-        constexpr int RPW = VS::kRows;
-        for (int ig = i0; ig < i1; ig += kRankGroup) {
-          const int nr = min(kRankGroup, i1 - ig);
-          float acc[RPW][kRankGroup];
-          vside_rows<MC>(p, ig, nr, a, lane, acc);
-#pragma unroll
-          for (int j = 0; j < RPW; ++j)
-#pragma unroll
-            for (int i = 0; i < kRankGroup; ++i)
-#pragma unroll
-              for (int o = 16; o >= 1; o >>= 1) acc[j][i] += __shfl_xor_sync(0xffffffffu, acc[j][i], o);
-          // z for row m, rank ig + i: straight into the U side's B tiles (BF16 high
-          // part in row m, the BF16 rounding of the rest in row MC + m, 128-byte
-          // swizzled rows) or into the fp32 z scratch
-          auto put = [&](int m, int i, float sum) {
-            const float zv = __fmul_rn(__ldcg(p.alpha + ig + i), sum);
-            if constexpr (Cfg<MC>::kTensorU) {
-              const __nv_bfloat16 hi = __float2bfloat16_rn(zv);
-              const __nv_bfloat16 lo = __float2bfloat16_rn(zv - __bfloat162float(hi));
-              store_ztile(p.ztiles, Layout<MC>::kUN, MC, m, ig + i, hi, lo);
-            } else {
-              p.z[static_cast<size_t>(m) * p.rpad + ig + i] = zv;
-            }
-          };
-          // the warps of a row group add their sums through shared memory
-          static_assert(VS::kSplit > 1, "every row group splits K");
-          if (lane == 0) {
-#pragma unroll
+      if constexpr (!Cfg<MC>::kTensorV) {
+        {
+          // every warp sums its rows over its K blocks; the warps that split one row's
+          // K then add their sums through shared memory
+          using VS = VSplit<MC>;
+          constexpr int RPW = VS::kRows;
+          for (int ig = i0; ig < i1; ig += kRankGroup) {
+            const int nr = min(kRankGroup, i1 - ig);
+            float acc[RPW][kRankGroup];
+            vside_rows<MC>(p, ig, nr, a, lane, acc);
+  #pragma unroll
             for (int j = 0; j < RPW; ++j)
-#pragma unroll
-              for (int i = 0; i < kRankGroup; ++i) vred[(a * RPW + j) * kRankGroup + i] = acc[j][i];
+  #pragma unroll
+              for (int i = 0; i < kRankGroup; ++i)
+  #pragma unroll
+                for (int o = 16; o >= 1; o >>= 1) acc[j][i] += __shfl_xor_sync(0xffffffffu, acc[j][i], o);
+            // z for row m, rank ig + i: straight into the U side's B tiles (BF16 high
+            // part in row m, the BF16 rounding of the rest in row MC + m, 128-byte
+            // swizzled rows) or into the fp32 z scratch
+            auto put = [&](int m, int i, float sum) {
+              const float zv = __fmul_rn(__ldcg(p.alpha + ig + i), sum);
+              if constexpr (Cfg<MC>::kTensorU) {
+                const __nv_bfloat16 hi = __float2bfloat16_rn(zv);
+                const __nv_bfloat16 lo = __float2bfloat16_rn(zv - __bfloat162float(hi));
+                store_ztile(p.ztiles, Layout<MC>::kUN, MC, m, ig + i, hi, lo);
+              } else {
+                p.z[static_cast<size_t>(m) * p.rpad + ig + i] = zv;
+              }
+            };
+            // the warps of a row group add their sums through shared memory
+            static_assert(VS::kSplit > 1, "every row group splits K");
+            if (lane == 0) {
+  #pragma unroll
+              for (int j = 0; j < RPW; ++j)
+  #pragma unroll
+                for (int i = 0; i < kRankGroup; ++i) vred[(a * RPW + j) * kRankGroup + i] = acc[j][i];
+            }
+            named_barrier(kBarAlu, kAluThreads);
+            if (tid < p.M * nr) {
+              const int m = tid / nr, i = tid - m * nr, j = VS::slot_of(m);
+              float sum = 0.0f;
+  #pragma unroll
+              for (int q = 0; q < VS::kSplit; ++q) sum += vred[(VS::warp_of(m, q) * RPW + j) * kRankGroup + i];
+              put(m, i, sum);
+            }
+            named_barrier(kBarAlu, kAluThreads);             // vred is reused by the next group
           }
-          named_barrier(kBarAlu, kAluThreads);
-          if (tid < p.M * nr) {
-            const int m = tid / nr, i = tid - m * nr, j = VS::slot_of(m);
-            float sum = 0.0f;
+        }
+      } else {
+        // ---- V side, part 2: z for this CTA's rank slice [i0, i1), the pieces'
+        // partial sums added in a fixed order (four lanes per (rank, row) pair, each
+        // summing every fourth K slice, then an xor-shuffle tree), times alpha
+        const int RB = (p.r + kTileRows - 1) / kTileRows;
+        const int S = vside_slices(p, RB);
+        constexpr int kParts = 4, kPerPart = kVSliceMax / kParts;
+        const int P = (i1 - i0) * p.M;
+        for (int base = 0; base < P * kParts; base += kAluThreads) {
+          const int idx = base + tid, pair = idx >> 2, part = idx & 3;
+          const bool act = pair < P;
+          const int il = act ? pair / p.M : 0;
+          const int i = i0 + il, m = act ? pair - il * p.M : 0;
+          const float* src = p.vpart + (static_cast<size_t>(i / kTileRows) * S * kBN + m) * kTileRows + (i % kTileRows);
+          // every request of the round first: the partial sums and alpha
+          const float al = (act && part == 0) ? __ldcg(p.alpha + i) : 0.0f;
+          float t[kPerPart];
 #pragma unroll
-            for (int q = 0; q < VS::kSplit; ++q) sum += vred[(VS::warp_of(m, q) * RPW + j) * kRankGroup + i];
-            put(m, i, sum);
+          for (int q = 0; q < kPerPart; ++q) {
+            const int sl = part + kParts * q;
+            t[q] = (act && sl < S) ? __ldcg(src + static_cast<size_t>(sl) * kBN * kTileRows) : 0.0f;
           }
-          named_barrier(kBarAlu, kAluThreads);             // vred is reused by the next group
+          float sum = 0.0f;
+#pragma unroll
+          for (int q = 0; q < kPerPart; ++q) sum += t[q];
+          sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+          sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+          if (act && part == 0) {
+            const float zv = __fmul_rn(al, sum);
+            const __nv_bfloat16 hi = __float2bfloat16_rn(zv);
+            const __nv_bfloat16 lo = __float2bfloat16_rn(zv - __bfloat162float(hi));
+            store_ztile(p.ztiles, Layout<MC>::kUN, MC, m, i, hi, lo);
+          }
         }
       }
       if constexpr (Cfg<MC>::kTensorU) {

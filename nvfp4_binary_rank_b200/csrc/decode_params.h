@@ -17,6 +17,7 @@ struct DecodeParams {
   float* z;                // [M][rpad] scratch: z = alpha . (V^T x)
   uint8_t* ztiles;         // [16][32][128 B] scratch: z as BF16 high/low MMA tiles (4+ rows)
   uint8_t* xq;             // [KC][2304 B] scratch: quantised activation image (8+ rows)
+  float* vpart;            // [G][16][128] scratch: V-side partial sums per piece (8+ rows)
   float* slots;            // [2 G][16][128] scratch: split-K partials
   uint32_t* z_ready;       // CTAs that published their z slice
   uint32_t* z_seen;        // CTAs done with z_ready (the last one resets both)

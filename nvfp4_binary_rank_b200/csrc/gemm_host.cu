@@ -136,7 +136,10 @@ GemmPlan plan_gemm(const GemmArgs& a) {
   if (p.decode) {
     need.act_fp4 = static_cast<size_t>(p.KC) * kDecodeQImgBytes;   // the activation image (8+ rows)
     need.act_sf = 16;
-    need.zpart = 16 * 32 * 128;                 // the decode kernel's z tiles
+    // the decode kernel's z tiles, then the V-side partial sums: one 16 x 128 block
+    // per piece, max(G, rank blocks) pieces at most
+    const size_t vpieces = static_cast<size_t>(std::max(p.G, (r + kTileRows - 1) / kTileRows));
+    need.zpart = 16 * 32 * 128 + vpieces * kDecodeMaxRows * kTileRows * 4;
     need.zfin = r ? static_cast<size_t>(M) * p.rpad * 4 : 16;
     need.slots = static_cast<size_t>(2 * p.G) * kDecodeMaxRows * kTileRows * 4;
     need.counter_words = 4 + 2 * static_cast<size_t>(p.T);   // z, tickets, q counters
@@ -180,6 +183,7 @@ int launch_gemm(const GemmArgs& a, const GemmPlan& p, const Scratch& scr, cudaSt
     dp.y = a.y;
     dp.z = sc->zfin;
     dp.ztiles = reinterpret_cast<uint8_t*>(sc->zpart);
+    dp.vpart = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(sc->zpart) + 16 * 32 * 128);
     dp.slots = sc->slots;
     dp.z_ready = sc->counters;
     dp.z_seen = sc->counters + 1;

@@ -106,6 +106,17 @@ def test_ragged_shapes_both_modes(nb, mode, M, N, K, r):
     assert_y_close(y, ref["y"], w.name)
 
 
+@pytest.mark.parametrize("M,N,K,r", [(9, 128, 256, 300), (12, 256, 640, 1024), (13, 384, 5120, 512),
+                                     (16, 1280, 1024, 129)])
+def test_decode_rank_pieces(nb, M, N, K, r):
+    # decode batches of 9-16 rows split V^T x into pieces of 128 ranks x a K slice:
+    # more rank blocks than CTAs, pieces of several MMA batches, a partial rank block
+    w = _small(M, N, K, r, seed=M * 7 + r)
+    d, ref = oracle_for(w)
+    y = _run(nb, device_problem(w, d))
+    assert_y_close(y, ref["y"], w.name)
+
+
 def test_deterministic_and_reusable(nb):
     w = workloads.CONFIGS["decode"]
     d, ref = oracle_for(w)
