@@ -14,13 +14,17 @@
 // stream, which is what bounds a decode call:
 //   * Weight stages are requested before that wait: no kernel of this library
 //     writes the weight operand.
-//   * The CUDA-core warps quantise the activation chunks of all the CTA's units
-//     at once into an operand cache in shared memory.  The MMAs read the
-//     activation from there, so the stage ring carries weight bytes only.
-//   * z is computed in rank slices: CTA g computes z for the ranks
-//     [g r / G, (g + 1) r / G) over the whole of K and publishes them behind one
-//     arrival counter.  This is the "side CTAs + arrival flag" schedule of the
-//     README's mode table, with every CTA taking a slice.
+//   * The activation chunks of all the CTA's units land at once in an operand
+//     cache in shared memory: below 8 rows quantised by the CTA itself, from 8
+//     rows up copied from an image the CTAs quantise once between them.  The MMAs
+//     read the activation from there, so the stage ring carries weight bytes only.
+//   * z is computed in rank slices: CTA g < Z computes z for the ranks
+//     [g r / Z, (g + 1) r / Z) and publishes them behind one arrival counter
+//     (Z = G - 2 on large grids, see shared_work_ctas).  This is the "side CTAs +
+//     arrival flag" schedule of the README's mode table.  Below 16 rows the slice
+//     is summed over the whole of K on the CUDA cores; with 16, V^T x runs on the
+//     tensor cores in pieces of 128 ranks x a K slice whose partial sums the slice
+//     owners add up.
 //   * Only the CTA that completes a weight tile (its sole owner, or the last
 //     split-K contributor to arrive) expands U z for that tile, in parallel with
 //     summing the split-K partials.  So publishing a partial never waits for z.
@@ -184,12 +188,21 @@ struct VSplit {
 // acc[j][i] for row row0 + j kStep and rank ig + i (ranks i >= nr are left at
 // zero).  Inputs that the previous kernel of the stream may have written are read
 // through L2 (ld.global.cg), never through a possibly stale L1 line.
-// K slices per rank block of the tensor-core V side: one piece per CTA where there
-// are enough CTAs, at most 32 (the cross-CTA sum of a (rank, row) pair takes four
-// lanes x eight partial sums).
+// CTAs that share the grid-wide work (z slices, activation image items, V pieces).
+// The last two CTAs of a large grid are left out: they are dispatched last, onto
+// SMs still held by the previous kernel, and pass the dependency wait up to 2 us
+// after the others (measured on B200), so any share of that work would hold up
+// every reader of it.
+__device__ __forceinline__ int shared_work_ctas(const DecodeParams& p) {
+  return p.G > 16 ? p.G - 2 : p.G;
+}
+
+// K slices per rank block of the tensor-core V side: one piece per sharing CTA
+// where there are enough, at most 32 (the cross-CTA sum of a (rank, row) pair takes
+// four lanes x eight partial sums).
 constexpr int kVSliceMax = 32;
 __device__ __forceinline__ int vside_slices(const DecodeParams& p, int RB) {
-  return max(1, min(min(p.G / RB, p.K / 64), kVSliceMax));
+  return max(1, min(min(shared_work_ctas(p) / RB, p.K / 64), kVSliceMax));
 }
 
 // V-side partial sums of one warp: rows row0 + j kStep (j < kRows), the K blocks
@@ -600,10 +613,14 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
                              : reinterpret_cast<uint4*>(smem + L::kSFB + k * 512) + (o - 128);
       *dst = make_uint4(0u, 0u, 0u, 0u);
     }
-    const int i0 = static_cast<int>(static_cast<uint32_t>(g) * static_cast<uint32_t>(p.r) /
-                                    static_cast<uint32_t>(p.G));
-    const int i1 = static_cast<int>(static_cast<uint32_t>(g + 1) * static_cast<uint32_t>(p.r) /
-                                    static_cast<uint32_t>(p.G));
+    // this CTA's slice of the ranks for z (empty for CTAs outside the sharing set)
+    const int zg = shared_work_ctas(p);
+    const int i0 = g < zg ? static_cast<int>(static_cast<uint32_t>(g) * static_cast<uint32_t>(p.r) /
+                                             static_cast<uint32_t>(zg))
+                          : p.r;
+    const int i1 = g < zg ? static_cast<int>(static_cast<uint32_t>(g + 1) * static_cast<uint32_t>(p.r) /
+                                             static_cast<uint32_t>(zg))
+                          : p.r;
     if (p.r > 0) {
       // warm L2 with the sign words this CTA reads later (a hint only)
       const char* vb = reinterpret_cast<const char*>(p.Vbits + static_cast<size_t>(i0) * p.KW);
@@ -664,13 +681,13 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
           }
         }
       } else {
-        // CTA g quantises items [g I / G, (g + 1) I / G) of the I = 16 KC blocks of
+        // CTA g < Z (Z = shared_work_ctas) quantises items [g I / Z, (g + 1) I / Z) of the I = 16 KC blocks of
         // 16 rows x 16 elements (rows >= M and blocks past K as zero codes and scales)
         // into the global image, publishes them, and after every CTA has done so
         // copies the chunks of its units into the operand cache
         const uint32_t items = static_cast<uint32_t>(p.KC) * 256u;
-        const uint32_t q0 = static_cast<uint32_t>(static_cast<uint64_t>(g) * items / static_cast<uint32_t>(p.G));
-        const uint32_t q1 = static_cast<uint32_t>(static_cast<uint64_t>(g + 1) * items / static_cast<uint32_t>(p.G));
+        const uint32_t q0 = g < zg ? static_cast<uint32_t>(static_cast<uint64_t>(g) * items / static_cast<uint32_t>(zg)) : 0u;
+        const uint32_t q1 = g < zg ? static_cast<uint32_t>(static_cast<uint64_t>(g + 1) * items / static_cast<uint32_t>(zg)) : 0u;
         for (uint32_t it = q0 + static_cast<uint32_t>(tid); it < q1; it += kAluThreads) {
           const int kc = static_cast<int>(it >> 8), m = static_cast<int>((it >> 4) & 15u), blk = static_cast<int>(it & 15u);
           const int kk = kc * kUnitK + blk * 16;
@@ -692,7 +709,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
           if (p.r > 0) {
             // ---- V side, part 1, on the tensor cores.  Piece (rb, s) = ranks
             // [128 rb, 128 rb + 128) x K atoms [s KA / S, (s + 1) KA / S); CTA g takes
-            // pieces g, g + G, ..  For each, the partial sums
+            // pieces g, g + Z, .. (Z = shared_work_ctas).  For each, the partial sums
             //   vpart[rb][s][m][i] = sum_{k in the slice} s_ik x[m][k]
             // come from BF16 MMAs: A = the pieces' sign bits expanded to +-1 (exact,
             // ranks >= r as zero rows), B = the activation rows (rows >= M zero), D in
@@ -706,7 +723,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
             const uint32_t idesc_v = (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(kBN >> 3) << 17) |
                                      (static_cast<uint32_t>(kTileRows >> 4) << 24);
             int vuses = 0;
-            for (int piece = g; piece < RB * S; piece += p.G) {
+            for (int piece = g; g < zg && piece < RB * S; piece += zg) {
               const int rb = piece / S, sl = piece - rb * S;
               const int a0 = static_cast<int>(static_cast<int64_t>(sl) * KA / S);
               const int a1 = static_cast<int>(static_cast<int64_t>(sl + 1) * KA / S);
@@ -943,7 +960,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
       }
       if constexpr (Cfg<MC>::kTensorU) {
         // the CTA holding the last ranks clears the tiles' tail past r
-        if (i1 == p.r) {
+        if (i1 == p.r && i0 < i1) {
           const int tail = ((p.r + kUChunk - 1) / kUChunk) * kUChunk;
           for (int idx = tid; idx < p.M * (tail - p.r); idx += kAluThreads) {
             const int m = idx / (tail - p.r), i = p.r + idx - m * (tail - p.r);
