@@ -25,9 +25,13 @@
 //     is summed over the whole of K on the CUDA cores; with 16, V^T x runs on the
 //     tensor cores in pieces of 128 ranks x a K slice whose partial sums the slice
 //     owners add up.
-//   * Only the CTA that completes a weight tile (its sole owner, or the last
-//     split-K contributor to arrive) expands U z for that tile, in parallel with
-//     summing the split-K partials.  So publishing a partial never waits for z.
+//   * U z: from 4 rows up (tensor-core U side) every contributor of a weight tile
+//     expands its share of U z for the tile (the 64-rank chunks in proportion to
+//     its units of the tile) and adds it to the partial it publishes, so the
+//     completing CTA (the sole owner, or the last split-K contributor to arrive)
+//     only sums partials.  Below 4 rows the completing CTA alone expands U z for
+//     the tile, in parallel with summing the partials, so the other CTAs publish
+//     without waiting for z and exit early.
 //
 // Warp roles (14 warps): warp 0 TMA producer; warp 1 TMEM allocator and MMA
 // issuer (tcgen05 kind::mxf4nvf4, block16); warps 2-5 epilogue (one weight row
@@ -100,6 +104,11 @@ struct Cfg {
   // U side on the tensor cores from 4 rows up; below, per-thread sign-adds are
   // cheaper than the chunked MMA chain (measured on B200)
   static constexpr bool kTensorU = MC >= 4;
+  // with the tensor-core U side every contributor of a tile adds its share of U z
+  // to its partial; below, the completing CTA alone expands U z for the tile, so
+  // the other CTAs exit early and free their SMs for the next kernel (each choice
+  // measured faster on B200 for its classes)
+  static constexpr bool kUShares = kTensorU;
   // from 8 rows up the CTAs quantise the activation once between them (a global
   // image behind an arrival counter) instead of each CTA quantising the chunks of
   // all its units
@@ -483,33 +492,77 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
     const int etid = threadIdx.x - kEpiWarp0 * 32;
     const float gs = __ldcg(p.gscale);
     constexpr int kHB = (MC <= 2) ? 16 : (MC <= 4 ? 8 : (MC <= 8 ? 4 : 2));   // partials loaded per batch
-    bool ok = true;
-    int nfin = 0;                                      // tiles completed here (U-side results read)
-    for (int seg = 0; seg < nseg; ++seg) {
-      const int t = t_first + seg;
-      const int b = seg & 1;
-      const int hf = owner_cta(static_cast<uint32_t>(t * p.KC), p.G, p.U);
-      const int hl = owner_cta(static_cast<uint32_t>((t + 1) * p.KC - 1), p.G, p.U);
-      const bool sole = hf == hl;
-      const int which = (t == t_first) ? 0 : 1;
-      float v[MC];
-      bool fin = false;
-      if (ok) ok = group_wait(accf_bar(b), (seg >> 1) & 1, kBarEpi, kEpiThreads, ctl);
-      if (ok) {
-        tc_fence_after();
-        uint32_t raw[16];
-        tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(b * kBN), raw);
-        tmem_wait_ld();
-#pragma unroll
-        for (int j = 0; j < MC; ++j) v[j] = __fmul_rn(gs, __uint_as_float(raw[j]));
-        tc_fence_before();
-        mbar_arrive(acce_bar(b));
+    if constexpr (Cfg<MC>::kUShares) {
+      bool ok = true;
+      for (int seg = 0; seg < nseg; ++seg) {
+        const int t = t_first + seg;
+        const int b = seg & 1;
+        const int hf = owner_cta(static_cast<uint32_t>(t * p.KC), p.G, p.U);
+        const int hl = owner_cta(static_cast<uint32_t>((t + 1) * p.KC - 1), p.G, p.U);
+        const bool sole = hf == hl;
+        const int which = (t == t_first) ? 0 : 1;
+        float v[MC];
+        if (ok) ok = group_wait(accf_bar(b), (seg >> 1) & 1, kBarEpi, kEpiThreads, ctl);
+        if (ok) {
+          tc_fence_after();
+          uint32_t raw[16];
+          tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(b * kBN), raw);
+          tmem_wait_ld();
+  #pragma unroll
+          for (int j = 0; j < MC; ++j) v[j] = __fmul_rn(gs, __uint_as_float(raw[j]));
+          tc_fence_before();
+          mbar_arrive(acce_bar(b));
+        }
+        if (p.r > 0) {
+          // this CTA's share of U z for the tile: the CUDA-core warps compute it once
+          // z is complete (barrier 1: the previous segment's share has been read;
+          // barrier 2: this one is ready)
+          if (named_barrier_or(kBarFin, kFinThreads, !ok)) {
+            if (ok) fail(ctl);
+            ok = false;
+          }
+          if (named_barrier_or(kBarFin2, kFinThreads, !ok)) {
+            if (ok) fail(ctl);
+            ok = false;
+          }
+          if (!ok) break;
+          if constexpr (Cfg<MC>::kTensorU) {
+            // the U-side MMAs left sum_i U[n][i] zhi[m][i] in column m and
+            // sum_i U[n][i] zlo[m][i] in column MC + m of lane n
+            const bool got = group_wait(ud_bar, seg & 1, kBarEpi, kEpiThreads, ctl);
+            if (!got) {
+              ok = false;
+              break;
+            }
+            if (fin_flag[seg]) {
+              tc_fence_after();
+              uint32_t du[L::kUN];
+              tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + kUTmem, *reinterpret_cast<uint32_t(*)[16]>(du));
+              if constexpr (L::kUN > 16)
+                tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + kUTmem + 16,
+                          *reinterpret_cast<uint32_t(*)[16]>(du + 16));
+              tmem_wait_ld();
+              tc_fence_before();
+    #pragma unroll
+              for (int j = 0; j < MC; ++j) v[j] += __uint_as_float(du[j]) + __uint_as_float(du[MC + j]);
+            }
+          } else {
+            const float* corr = reinterpret_cast<const float*>(smem + L::kCorr);
+  #pragma unroll
+            for (int j = 0; j < MC; ++j)
+              v[j] = (v[j] + corr[j * kTileRows + row]) + corr[(MC + j) * kTileRows + row];
+          }
+        }
+        if (!ok) break;
+        float acc[MC];
         if (sole) {
-          fin = true;
+  #pragma unroll
+          for (int j = 0; j < MC; ++j) acc[j] = v[j];
         } else {
-          // publish this partial; the last contributor of the tile completes it
+          // publish this partial (FP4 product and U z share); the last contributor
+          // of the tile completes it
           float* my_slot = p.slots + static_cast<size_t>(2 * g + which) * kRowsMax * kTileRows;
-#pragma unroll
+  #pragma unroll
           for (int j = 0; j < MC; ++j)
             if (j < p.M) my_slot[j * kTileRows + row] = v[j];
           named_barrier(kBarEpi, kEpiThreads);
@@ -522,85 +575,159 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
             *epi_last = last ? 1 : 0;
           }
           named_barrier(kBarEpi, kEpiThreads);
-          fin = *epi_last != 0;
+          const bool fin = *epi_last != 0;
           named_barrier(kBarEpi, kEpiThreads);
-        }
-      }
-      if (p.r > 0) {
-        // tell the CUDA-core warps whether this tile's correction is needed here
-        if (etid == 0) fin_flag[seg] = fin ? 1 : 0;
-        if (named_barrier_or(kBarFin, kFinThreads, !ok)) {
-          if (ok) fail(ctl);
-          ok = false;
-        }
-      }
-      if (!ok) break;
-      if (!fin) continue;
-      float acc[MC];
-      if (sole) {
-#pragma unroll
-        for (int j = 0; j < MC; ++j) acc[j] = v[j];
-      } else {
-        // every contributor's partial, summed in contributor order
-#pragma unroll
-        for (int j = 0; j < MC; ++j) acc[j] = 0.0f;
-        const int wh_first = (t == first_unit(hf, p.G, p.U) / p.KC) ? 0 : 1;
-        for (int h0 = hf; h0 <= hl; h0 += kHB) {
-          float part[kHB][MC];
-#pragma unroll
-          for (int e = 0; e < kHB; ++e) {
-            const int h = h0 + e;
-            const float* sl = p.slots + static_cast<size_t>(2 * h + ((h == hf) ? wh_first : 0)) *
-                                            kRowsMax * kTileRows;
-#pragma unroll
-            for (int j = 0; j < MC; ++j)
-              part[e][j] = (h <= hl && h != g && j < p.M) ? __ldcg(sl + j * kTileRows + row) : 0.0f;
-          }
-#pragma unroll
-          for (int e = 0; e < kHB; ++e) {
-            const int h = h0 + e;
-            if (h <= hl) {
-#pragma unroll
-              for (int j = 0; j < MC; ++j) acc[j] += (h == g) ? v[j] : part[e][j];
+          if (!fin) continue;
+          // every contributor's partial, summed in contributor order
+  #pragma unroll
+          for (int j = 0; j < MC; ++j) acc[j] = 0.0f;
+          const int wh_first = (t == first_unit(hf, p.G, p.U) / p.KC) ? 0 : 1;
+          for (int h0 = hf; h0 <= hl; h0 += kHB) {
+            float part[kHB][MC];
+  #pragma unroll
+            for (int e = 0; e < kHB; ++e) {
+              const int h = h0 + e;
+              const float* sl = p.slots + static_cast<size_t>(2 * h + ((h == hf) ? wh_first : 0)) *
+                                              kRowsMax * kTileRows;
+  #pragma unroll
+              for (int j = 0; j < MC; ++j)
+                part[e][j] = (h <= hl && h != g && j < p.M) ? __ldcg(sl + j * kTileRows + row) : 0.0f;
+            }
+  #pragma unroll
+            for (int e = 0; e < kHB; ++e) {
+              const int h = h0 + e;
+              if (h <= hl) {
+  #pragma unroll
+                for (int j = 0; j < MC; ++j) acc[j] += (h == g) ? v[j] : part[e][j];
+              }
             }
           }
         }
-      }
-      if (p.r > 0) {
-        if (named_barrier_or(kBarFin2, kFinThreads, !ok)) {
-          ok = false;
-          break;
-        }
-        if constexpr (Cfg<MC>::kTensorU) {
-          // the correction: the U-side MMAs left sum_i U[n][i] zhi[m][i] in column m
-          // and sum_i U[n][i] zlo[m][i] in column MC + m of lane n
-          const bool got = group_wait(ud_bar, nfin & 1, kBarEpi, kEpiThreads, ctl);
-          ++nfin;
-          if (!got) {
-            ok = false;
-            continue;                                    // the next vote tells the CUDA-core warps
-          }
-          tc_fence_after();
-          uint32_t du[L::kUN];
-          tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + kUTmem, *reinterpret_cast<uint32_t(*)[16]>(du));
-          if constexpr (L::kUN > 16)
-            tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + kUTmem + 16,
-                      *reinterpret_cast<uint32_t(*)[16]>(du + 16));
-          tmem_wait_ld();
-          tc_fence_before();
+        uint16_t* yb = p.y + static_cast<size_t>(t) * kTileRows + row;
   #pragma unroll
-          for (int j = 0; j < MC; ++j) acc[j] += __uint_as_float(du[j]) + __uint_as_float(du[MC + j]);
-        } else {
-          const float* corr = reinterpret_cast<const float*>(smem + L::kCorr);
-#pragma unroll
-          for (int j = 0; j < MC; ++j)
-            acc[j] = (acc[j] + corr[j * kTileRows + row]) + corr[(MC + j) * kTileRows + row];
-        }
+        for (int j = 0; j < MC; ++j)
+          if (j < p.M) yb[static_cast<size_t>(j) * p.N] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[j]));
       }
-      uint16_t* yb = p.y + static_cast<size_t>(t) * kTileRows + row;
-#pragma unroll
-      for (int j = 0; j < MC; ++j)
-        if (j < p.M) yb[static_cast<size_t>(j) * p.N] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[j]));
+    } else {
+      bool ok = true;
+      int nfin = 0;                                      // tiles completed here (U-side results read)
+      for (int seg = 0; seg < nseg; ++seg) {
+        const int t = t_first + seg;
+        const int b = seg & 1;
+        const int hf = owner_cta(static_cast<uint32_t>(t * p.KC), p.G, p.U);
+        const int hl = owner_cta(static_cast<uint32_t>((t + 1) * p.KC - 1), p.G, p.U);
+        const bool sole = hf == hl;
+        const int which = (t == t_first) ? 0 : 1;
+        float v[MC];
+        bool fin = false;
+        if (ok) ok = group_wait(accf_bar(b), (seg >> 1) & 1, kBarEpi, kEpiThreads, ctl);
+        if (ok) {
+          tc_fence_after();
+          uint32_t raw[16];
+          tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(b * kBN), raw);
+          tmem_wait_ld();
+  #pragma unroll
+          for (int j = 0; j < MC; ++j) v[j] = __fmul_rn(gs, __uint_as_float(raw[j]));
+          tc_fence_before();
+          mbar_arrive(acce_bar(b));
+          if (sole) {
+            fin = true;
+          } else {
+            // publish this partial; the last contributor of the tile completes it
+            float* my_slot = p.slots + static_cast<size_t>(2 * g + which) * kRowsMax * kTileRows;
+  #pragma unroll
+            for (int j = 0; j < MC; ++j)
+              if (j < p.M) my_slot[j * kTileRows + row] = v[j];
+            named_barrier(kBarEpi, kEpiThreads);
+            if (etid == 0) {
+              // release: this CTA's partial; acquire: every earlier contributor's
+              const uint32_t nh = static_cast<uint32_t>(hl - hf + 1);
+              const uint32_t old = atom_add_acq_rel_gpu(p.tickets + t, 1u);
+              const bool last = old == nh - 1;
+              if (last) atomicExch(p.tickets + t, 0u);
+              *epi_last = last ? 1 : 0;
+            }
+            named_barrier(kBarEpi, kEpiThreads);
+            fin = *epi_last != 0;
+            named_barrier(kBarEpi, kEpiThreads);
+          }
+        }
+        if (p.r > 0) {
+          // tell the CUDA-core warps whether this tile's correction is needed here
+          if (etid == 0) fin_flag[seg] = fin ? 1 : 0;
+          if (named_barrier_or(kBarFin, kFinThreads, !ok)) {
+            if (ok) fail(ctl);
+            ok = false;
+          }
+        }
+        if (!ok) break;
+        if (!fin) continue;
+        float acc[MC];
+        if (sole) {
+  #pragma unroll
+          for (int j = 0; j < MC; ++j) acc[j] = v[j];
+        } else {
+          // every contributor's partial, summed in contributor order
+  #pragma unroll
+          for (int j = 0; j < MC; ++j) acc[j] = 0.0f;
+          const int wh_first = (t == first_unit(hf, p.G, p.U) / p.KC) ? 0 : 1;
+          for (int h0 = hf; h0 <= hl; h0 += kHB) {
+            float part[kHB][MC];
+  #pragma unroll
+            for (int e = 0; e < kHB; ++e) {
+              const int h = h0 + e;
+              const float* sl = p.slots + static_cast<size_t>(2 * h + ((h == hf) ? wh_first : 0)) *
+                                              kRowsMax * kTileRows;
+  #pragma unroll
+              for (int j = 0; j < MC; ++j)
+                part[e][j] = (h <= hl && h != g && j < p.M) ? __ldcg(sl + j * kTileRows + row) : 0.0f;
+            }
+  #pragma unroll
+            for (int e = 0; e < kHB; ++e) {
+              const int h = h0 + e;
+              if (h <= hl) {
+  #pragma unroll
+                for (int j = 0; j < MC; ++j) acc[j] += (h == g) ? v[j] : part[e][j];
+              }
+            }
+          }
+        }
+        if (p.r > 0) {
+          if (named_barrier_or(kBarFin2, kFinThreads, !ok)) {
+            ok = false;
+            break;
+          }
+          if constexpr (Cfg<MC>::kTensorU) {
+            // the correction: the U-side MMAs left sum_i U[n][i] zhi[m][i] in column m
+            // and sum_i U[n][i] zlo[m][i] in column MC + m of lane n
+            const bool got = group_wait(ud_bar, nfin & 1, kBarEpi, kEpiThreads, ctl);
+            ++nfin;
+            if (!got) {
+              ok = false;
+              continue;                                    // the next vote tells the CUDA-core warps
+            }
+            tc_fence_after();
+            uint32_t du[L::kUN];
+            tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + kUTmem, *reinterpret_cast<uint32_t(*)[16]>(du));
+            if constexpr (L::kUN > 16)
+              tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + kUTmem + 16,
+                        *reinterpret_cast<uint32_t(*)[16]>(du + 16));
+            tmem_wait_ld();
+            tc_fence_before();
+    #pragma unroll
+            for (int j = 0; j < MC; ++j) acc[j] += __uint_as_float(du[j]) + __uint_as_float(du[MC + j]);
+          } else {
+            const float* corr = reinterpret_cast<const float*>(smem + L::kCorr);
+  #pragma unroll
+            for (int j = 0; j < MC; ++j)
+              acc[j] = (acc[j] + corr[j * kTileRows + row]) + corr[(MC + j) * kTileRows + row];
+          }
+        }
+        uint16_t* yb = p.y + static_cast<size_t>(t) * kTileRows + row;
+  #pragma unroll
+        for (int j = 0; j < MC; ++j)
+          if (j < p.M) yb[static_cast<size_t>(j) * p.N] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[j]));
+      }
     }
   } else {
     // ---------------------------------------------------------------- CUDA cores
@@ -972,11 +1099,14 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
       if (tid == 0) red_add_release_gpu(p.z_ready, 1u);   // covers the slice the CTA wrote
 
       if constexpr (Cfg<MC>::kTensorU) {
-        // ---- 3. U side of every tile this CTA completes, on the tensor cores:
-        // corr[n][m] = sum_i U[n][i] z[m][i] as one BF16 MMA chain per tile, 64 ranks
-        // per chunk.  A = the tile's sign bits expanded to +-1 BF16 (exact); B = z split
-        // into a BF16 high part and the BF16 rounding of the rest (rows m and MC + m),
-        // so the product keeps about 16 bits of z.  The epilogue adds both columns.
+        // ---- 3. This CTA's share of U z for each of its tiles, on the tensor cores:
+        // corr[n][m] = sum_i U[n][i] z[m][i] over the 64-rank chunks [cs0, cs1) of the
+        // share, as one BF16 MMA chain.  A tile's contributors split its chunks in
+        // proportion to their units of it, so every contributor adds its share to the
+        // partial it publishes and the completing CTA only sums partials.  A = the
+        // tile's sign bits expanded to +-1 BF16 (exact); B = z split into a BF16 high
+        // part and the BF16 rounding of the rest (rows m and MC + m), so the product
+        // keeps about 16 bits of z.  The epilogue adds both columns.
         const int nuc = (p.r + kUChunk - 1) / kUChunk;
         const int row = tid & (kTileRows - 1), half = tid >> 7;
         const uint32_t idesc_u = (1u << 4) | (1u << 7) | (1u << 10) |
@@ -1001,9 +1131,11 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
             ok = false;
             break;
           }
-          if (!fin_flag[seg]) continue;
-          if (!ztiles) {
-            // first tile this CTA completes: wait for every slice of z, then the B tiles
+          const int t = t_first + seg;
+          const int ua = max(u0, t * p.KC), ub = min(u1, (t + 1) * p.KC);
+          const int cs0 = (ua - t * p.KC) * nuc / p.KC, cs1 = (ub - t * p.KC) * nuc / p.KC;
+          if (cs1 > cs0 && !ztiles) {
+            // first non-empty share: wait for every slice of z, then the B tiles
             bool okw = true;
             if (tid == 0) okw = spin_until_geq(p.z_ready, static_cast<uint32_t>(p.G), ctl);
             if (named_barrier_or(kBarAlu, kAluThreads, !okw)) {
@@ -1045,11 +1177,11 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
           // the chunk's MMAs and commits them to the buffer's free barrier, which the
           // threads wait on before they write the buffer again.
 #pragma unroll 1
-          for (int c2 = 0; c2 < kUChunksMax; c2 += 2) {
+          for (int c2 = cs0; c2 < cs1; c2 += 2) {
 #pragma unroll
           for (int buf = 0; buf < 2; ++buf) {
             const int c = c2 + buf;
-            if (c < nuc) {
+            if (c < cs1) {
               int& uses = buf ? uses1 : uses0;
               if (uses > 0) {
                 // the MMAs that read this buffer last are done
@@ -1084,7 +1216,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
                   const uint64_t b_d = smem_desc(smem_u32(smem + L::kUZ + c * L::kUN * 128), 16, 1024, 2);
   #pragma unroll
                   for (int j = 0; j < 4; ++j)
-                    tc_mma_bf16(tmem + kUTmem, a_d + 2 * j, b_d + 2 * j, idesc_u, (c > 0 || j > 0) ? 1u : 0u);
+                    tc_mma_bf16(tmem + kUTmem, a_d + 2 * j, b_d + 2 * j, idesc_u, (c > cs0 || j > 0) ? 1u : 0u);
                   tc_commit(ubuf_bar(buf));
                 } else {
                   fail(ctl);
@@ -1095,7 +1227,10 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
             }
           }
           }
-          if (tid == 0) tc_commit(ud_bar);
+          if (tid == 0) {
+            fin_flag[seg] = (cs1 > cs0) ? 1 : 0;           // a share to add, in kUTmem
+            tc_commit(ud_bar);                             // arrives at once if nothing was issued
+          }
           if (named_barrier_or(kBarFin2, kFinThreads, !ok)) {
             ok = false;
             break;
