@@ -1298,9 +1298,12 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
           }
           if (ok) {
             if (seg >= 2) load_words(t, uw1);            // segments past the second: load now
-            float acc[MC];
+            // four interleaved sums per row: a dependency chain a quarter as long
+            float acc4[MC][4];
   #pragma unroll
-            for (int m = 0; m < MC; ++m) acc[m] = 0.0f;
+            for (int m = 0; m < MC; ++m)
+  #pragma unroll
+              for (int jj = 0; jj < 4; ++jj) acc4[m][jj] = 0.0f;
             for (int w = 0; w < wb - wa; ++w) {
               uint32_t word = 0;
   #pragma unroll
@@ -1316,12 +1319,15 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
   #pragma unroll
                     for (int jj = 0; jj < 4; ++jj) {
                       const uint32_t sgn = (word << (31 - (4 * j4 + jj))) & 0x80000000u;
-                      acc[m] += __uint_as_float(__float_as_uint(zz[jj]) ^ sgn);
+                      acc4[m][jj] += __uint_as_float(__float_as_uint(zz[jj]) ^ sgn);
                     }
                   }
                 }
               }
             }
+            float acc[MC];
+  #pragma unroll
+            for (int m = 0; m < MC; ++m) acc[m] = (acc4[m][0] + acc4[m][1]) + (acc4[m][2] + acc4[m][3]);
   #pragma unroll
             for (int m = 0; m < MC; ++m) corr[(half * MC + m) * kTileRows + row] = acc[m];
           }
