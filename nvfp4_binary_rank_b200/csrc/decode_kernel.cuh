@@ -90,6 +90,7 @@ constexpr int kBarAlu = 1;
 constexpr int kBarEpi = 2;
 constexpr int kBarFin = 3;                // epilogue + CUDA cores: finisher decision
 constexpr int kBarFin2 = 4;               // epilogue + CUDA cores: correction ready
+constexpr int kBarZ = 5;                  // epilogue + CUDA cores: z staged (1-2 rows)
 
 // Per batch class (MC = most activation rows): weight stages and V-side ranks
 // per pass (the largest class trades stages and ranks for its z and register
@@ -610,7 +611,6 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
       }
     } else {
       bool ok = true;
-      int nfin = 0;                                      // tiles completed here (U-side results read)
       for (int seg = 0; seg < nseg; ++seg) {
         const int t = t_first + seg;
         const int b = seg & 1;
@@ -693,35 +693,58 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
           }
         }
         if (p.r > 0) {
+          // the correction in three parts: the CUDA-core warps sum the first two
+          // thirds of the rank words for every row, this thread the last third for
+          // its own row, once the CUDA-core warps have staged z
+          static_assert(!Cfg<MC>::kTensorU, "the completing-CTA U side is the sign-add one");
+          const int w2 = 2 * p.RW / 3;
+          const uint32_t* ur = p.Ubits + (static_cast<size_t>(t) * kTileRows + row) * p.RW;
+          uint32_t uw[16];
+  #pragma unroll
+          for (int w = 0; w < 16; ++w) uw[w] = (w2 + w < p.RW) ? __ldcg(ur + w2 + w) : 0u;
+          if (named_barrier_or(kBarZ, kFinThreads, !ok)) ok = false;
+          float own[MC];
+  #pragma unroll
+          for (int m = 0; m < MC; ++m) own[m] = 0.0f;
+          if (ok) {
+            const float* zs = reinterpret_cast<const float*>(smem + L::kZ);
+            float acc4[MC][4];
+  #pragma unroll
+            for (int m = 0; m < MC; ++m)
+  #pragma unroll
+              for (int jj = 0; jj < 4; ++jj) acc4[m][jj] = 0.0f;
+            for (int w = 0; w < p.RW - w2; ++w) {
+              uint32_t word = 0;
+  #pragma unroll
+              for (int e = 0; e < 16; ++e) word = (e == w) ? uw[e] : word;
+              const float* zw = zs + (w2 + w) * 32;
+  #pragma unroll
+              for (int j4 = 0; j4 < 8; ++j4) {
+  #pragma unroll
+                for (int m = 0; m < MC; ++m) {
+                  if (m < p.M) {
+                    const float4 z4 = *reinterpret_cast<const float4*>(zw + m * kMaxRanks + 4 * j4);
+                    const float zz[4] = {z4.x, z4.y, z4.z, z4.w};
+  #pragma unroll
+                    for (int jj = 0; jj < 4; ++jj) {
+                      const uint32_t sgn = (word << (31 - (4 * j4 + jj))) & 0x80000000u;
+                      acc4[m][jj] += __uint_as_float(__float_as_uint(zz[jj]) ^ sgn);
+                    }
+                  }
+                }
+              }
+            }
+  #pragma unroll
+            for (int m = 0; m < MC; ++m) own[m] = (acc4[m][0] + acc4[m][1]) + (acc4[m][2] + acc4[m][3]);
+          }
           if (named_barrier_or(kBarFin2, kFinThreads, !ok)) {
             ok = false;
             break;
           }
-          if constexpr (Cfg<MC>::kTensorU) {
-            // the correction: the U-side MMAs left sum_i U[n][i] zhi[m][i] in column m
-            // and sum_i U[n][i] zlo[m][i] in column MC + m of lane n
-            const bool got = group_wait(ud_bar, nfin & 1, kBarEpi, kEpiThreads, ctl);
-            ++nfin;
-            if (!got) {
-              ok = false;
-              continue;                                    // the next vote tells the CUDA-core warps
-            }
-            tc_fence_after();
-            uint32_t du[L::kUN];
-            tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + kUTmem, *reinterpret_cast<uint32_t(*)[16]>(du));
-            if constexpr (L::kUN > 16)
-              tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + kUTmem + 16,
-                        *reinterpret_cast<uint32_t(*)[16]>(du + 16));
-            tmem_wait_ld();
-            tc_fence_before();
-    #pragma unroll
-            for (int j = 0; j < MC; ++j) acc[j] += __uint_as_float(du[j]) + __uint_as_float(du[MC + j]);
-          } else {
-            const float* corr = reinterpret_cast<const float*>(smem + L::kCorr);
+          const float* corr = reinterpret_cast<const float*>(smem + L::kCorr);
   #pragma unroll
-            for (int j = 0; j < MC; ++j)
-              acc[j] = (acc[j] + corr[j * kTileRows + row]) + corr[(MC + j) * kTileRows + row];
-          }
+          for (int j = 0; j < MC; ++j)
+            acc[j] = ((acc[j] + corr[j * kTileRows + row]) + corr[(MC + j) * kTileRows + row]) + own[j];
         }
         uint16_t* yb = p.y + static_cast<size_t>(t) * kTileRows + row;
   #pragma unroll
@@ -1260,11 +1283,12 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
         float* zs = reinterpret_cast<float*>(smem + L::kZ);
         float* corr = reinterpret_cast<float*>(smem + L::kCorr);
         bool ok = true, staged = false;
-        // thread (row, half) sums ranks [32 wa, 32 wb) of weight row `row`; the sign
-        // words of the first two tiles are requested now, before z is complete
+        // thread (row, half) sums ranks [32 wa, 32 wb) of weight row `row`: the first
+        // and second thirds of the words (the epilogue threads take the last third);
+        // the sign words of the first two tiles are requested now, before z is complete
         const int row = tid & (kTileRows - 1), half = tid >> 7;
-        const int wsplit = (p.RW + 1) >> 1;
-        const int wa = half ? wsplit : 0, wb = half ? p.RW : wsplit;
+        const int w1 = p.RW / 3, w2 = 2 * p.RW / 3;
+        const int wa = half ? w1 : 0, wb = half ? w2 : w1;
         auto load_words = [&](int t, uint32_t (&uw)[16]) {
           const uint32_t* ur = p.Ubits + (static_cast<size_t>(t) * kTileRows + row) * p.RW;
   #pragma unroll
@@ -1296,6 +1320,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
               staged = true;
             }
           }
+          if (named_barrier_or(kBarZ, kFinThreads, !ok)) ok = false;   // z staged for the epilogue's third
           if (ok) {
             if (seg >= 2) load_words(t, uw1);            // segments past the second: load now
             // four interleaved sums per row: a dependency chain a quarter as long
