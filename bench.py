@@ -403,13 +403,16 @@ def run_ours(args):
 
 # ----------------------------------------------------------------------------- CPU oracle
 
-def _oracle_sample(w, rows):
-    """Inputs for the oracle on output rows [0, rows) of the workload."""
+def _oracle_sample(w, rows, kk=None, rr=None):
+    """Inputs for the oracle on output rows [0, rows), the first kk elements of K and
+    the first rr ranks of the workload: the same problem at a smaller size."""
     from oracle import nvfp4 as on
+    kk = w.K if kk is None else kk
+    rr = w.r if rr is None else rr
     d = workloads.make_inputs(w)
     wq, ws, g = on.quant_weight(d["R"])
-    return dict(x=d["x"], wq=wq[:rows], ws=ws[:rows], g=g, U=d["U"][:rows], V=d["V"],
-                alpha=d["alpha"])
+    return dict(x=d["x"][:, :kk], wq=wq[:rows, :kk // 2], ws=ws[:rows, :kk // 16], g=g,
+                U=d["U"][:rows, :rr], V=d["V"][:kk, :rr], alpha=d["alpha"][:rr])
 
 
 def _oracle_step(s):
@@ -453,31 +456,54 @@ def run_reference(args):
     if rank != 0:
         return
     w = workloads.CONFIGS[args.workload]
-    # each step is a bounded row slice so that warm-up + steps stay within ~2 minutes
-    probe = _oracle_sample(w, 128)
-    t0 = time.perf_counter()
-    _oracle_step(probe)
-    t_row = (time.perf_counter() - t0) / 128
-    per_step = 100.0 / max(args.steps + args.warmup, 1)
-    rows = int(max(1, min(w.N, per_step / max(t_row, 1e-9))))
-    s = _oracle_sample(w, rows)
+    # Each step is a bounded sample of the workload (output rows, a K slice in
+    # multiples of 256, a rank slice), shrunk by halving until one step fits
+    # 100 s / (steps + warm-up), so that the whole run stays within about 2 minutes.
+    target = 100.0 / max(args.steps + args.warmup, 1)
+    rows, kk, rr = min(w.N, 128), w.K, w.r
+
+    def step_time(rows, kk, rr):
+        smp = _oracle_sample(w, rows, kk, rr)
+        _oracle_step(smp)
+        t0 = time.perf_counter()
+        n = 0
+        while n < 3 or time.perf_counter() - t0 < 0.05:
+            _oracle_step(smp)
+            n += 1
+        return (time.perf_counter() - t0) / n
+
+    t = step_time(rows, kk, rr)
+    while t > target:
+        if rows > 1:
+            rows = max(1, rows // 2)
+        elif kk > 256:
+            kk = max(256, (kk // 2) // 256 * 256)
+        elif rr > 1:
+            rr = max(1, rr // 2)
+        else:
+            break
+        t = step_time(rows, kk, rr)
+    if t < target / 4 and rows == min(w.N, 128) and kk == w.K and rr == w.r:
+        rows = int(max(1, min(w.N, rows * 0.5 * target / max(t, 1e-9))))
+    s = _oracle_sample(w, rows, kk, rr)
     for _ in range(args.warmup):
         _oracle_step(s)
     t0 = time.perf_counter()
     for _ in range(args.steps):
         _oracle_step(s)
     dt = (time.perf_counter() - t0) / args.steps
-    b = algo_bytes(w.M, rows, w.K, w.r)
+    b = algo_bytes(w.M, rows, kk, rr)
     val = b / dt / 1e9
+    sample = f"oracle on output rows 0..{rows}, K elements 0..{kk}, ranks 0..{rr} of {w.name} per step"
     line = {
         "metric": METRIC, "value": round(val, 4), "unit": UNIT, "n_gpus": int(args.gpus),
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "impl": "reference",
         "config": {"workload": w.name, "M": w.M, "N": w.N, "K": w.K, "r": w.r, "seed": w.seed,
-                   "rows_per_step": rows},
+                   "rows_per_step": rows, "k_per_step": kk, "ranks_per_step": rr},
         "cpu_baseline": {"value": round(val, 4), "unit": UNIT, "cores": _threads(), "kind": "oracle",
-                         "sample": f"oracle on rows 0..{rows} of {w.name} per step"},
+                         "sample": sample},
         "e2e": {"value": round(val, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
