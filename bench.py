@@ -269,7 +269,7 @@ def time_e2e(prob, steps, stream):
 
 
 class DistCtx:
-    """One process per GPU (torchrun env vars).  NCCL on the GPU machine; `gloo`
+    """One process per GPU (torchrun env vars).  NCCL between GPUs; `gloo`
     serves the CPU tests of the rank logic."""
 
     def __init__(self, backend: str = "nccl"):
