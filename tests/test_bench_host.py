@@ -1,0 +1,54 @@
+"""Host-side pieces of bench.py on the CPU: the algorithmic byte count behind
+every GB/s figure, the reference arm's bounded sample, and the rule that a
+committed ncu summary's DRAM traffic is reported only for the kernel sources it
+was captured from."""
+
+import os
+import sys
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+import workloads  # noqa: E402
+
+
+def test_algorithmic_bytes_of_the_workloads():
+    # codes N K / 2 + scales N K / 16 + sign bits (N + K) r / 8 + BF16 x and y + FP32
+    # alpha, tabulated independently for the decode and MLP shapes
+    want = {"decode": 15_423_488, "mlp_up": 41_633_792, "mlp_down": 42_240_000}
+    for name, b in want.items():
+        w = workloads.CONFIGS[name]
+        assert bench.algo_bytes(w.M, w.N, w.K, w.r) == b, name
+
+
+def test_algorithmic_bytes_grow_with_each_term():
+    base = bench.algo_bytes(1, 128, 256, 32)
+    assert bench.algo_bytes(1, 256, 256, 32) - base == 128 * 256 // 2 + 128 * 256 // 16 + 128 * 32 // 8 + 2 * 128
+    assert bench.algo_bytes(2, 128, 256, 32) - base == 2 * 256 + 2 * 128
+    assert bench.algo_bytes(1, 128, 256, 64) - base == (128 + 256) * 32 // 8 + 4 * 32
+
+
+def test_reference_sample_is_the_same_problem_smaller():
+    w = workloads.CONFIGS["tiny"]
+    s = bench._oracle_sample(w, 3, 128, 8)
+    assert s["x"].shape == (w.M, 128)
+    assert s["wq"].shape == (3, 64) and s["ws"].shape == (3, 8)
+    assert s["U"].shape == (3, 8) and s["V"].shape == (128, 8) and s["alpha"].shape == (8,)
+    y = bench._oracle_step(s)
+    assert y.shape == (w.M, 3) and np.all(np.isfinite(y))
+    # the full sample reproduces the oracle's output rows on the same inputs
+    full = bench._oracle_step(bench._oracle_sample(w, w.N))
+    part = bench._oracle_step(bench._oracle_sample(w, 5))
+    np.testing.assert_array_equal(part, full[:, :5])
+
+
+def test_ncu_traffic_follows_the_source_digest(monkeypatch):
+    got = bench.ncu_traffic("decode", 1)
+    if got is not None:
+        assert got > 14_000_000                      # about the 15.4 MB a decode call moves
+    monkeypatch.setattr(bench, "kernel_source_digest", lambda: "0000000000000000")
+    assert bench.ncu_traffic("decode", 1) is None
+    assert bench.ncu_traffic("no_such_workload", 1) is None
