@@ -61,7 +61,8 @@ enum {
   BILOCO_ERR_CUDA = -4,    /* a CUDA runtime call or a kernel launch failed       */
   BILOCO_ERR_TIMEOUT = -5, /* a bounded device-side wait expired (see last_error) */
   BILOCO_ERR_NOMEM = -6,   /* library scratch could not be allocated              */
-  BILOCO_ERR_DEVICE = -7   /* the current device is not an sm_100 GPU             */
+  BILOCO_ERR_DEVICE = -7,  /* the current device is not an sm_100 GPU             */
+  BILOCO_ERR_RESIDENCY = -8 /* the GEMM grid cannot be resident on the GPU at once  */
 };
 
 /* Size limits of biloco_gemm.  The weight is cut into (N/128) * ceil(K/256) units
@@ -133,6 +134,39 @@ int biloco_pack_weight(const float *R, int N, int K, uint8_t *W_fp4, uint8_t *W_
 size_t biloco_weight_sf_bytes(int N, int K);
 
 /*
+ * biloco_decompose - W ~= U diag(alpha) V^T + R with binary sign factors.
+ * (BiLoCo README, section "Decomposition": each rank-one term starts from random
+ * signs and alternates u = sign(R v), v = sign(R^T u) for T steps, takes the
+ * Frobenius-optimal coefficient and deflates the residual; after all r terms the
+ * coefficients are refit jointly by least squares for the fixed signs.)
+ *
+ *   W          [N][K] float, 4-byte aligned, not modified (R_out may alias it)
+ *   r, T       0 <= r <= 1024 terms, T >= 1 alternations per term
+ *   v0bits     [r][ceil(K/32)] uint32: the start signs of each term's v, packed
+ *              like pack_signs (bit 1 = -1); the caller draws them (the README
+ *              seeds a generator); may be NULL when r == 0
+ *   Ubits      out [N][ceil(r/32)] uint32 = pack_signs(U)    (biloco_gemm's Ubits)
+ *   Vbits      out [r][ceil(K/32)] uint32 = pack_signs(V^T)  (biloco_gemm's Vbits)
+ *   alpha      out [r] float, the refit coefficients
+ *   R_out      out [N][K] float, W - U diag(alpha) V^T (feed it to
+ *              biloco_pack_weight for the NVFP4 residual)
+ *   workspace  device memory of at least biloco_decompose_workspace_bytes(N, K, r)
+ *              bytes, 256-byte aligned, owned by the caller (it holds the FP64
+ *              residual: about 8 N K bytes)
+ * Every sign is decided on an FP64 sum, with sign(0) = +1; alpha_i = u^T R v /
+ * (N K) for the current residual; the refit solves the normal equations
+ * (u_i . u_j)(v_i . v_j) alpha = u_i^T W v_i by conjugate gradients (the
+ * minimum-norm solution if terms repeat).  Asynchronous on `stream`; about
+ * r (3 T + 2) kernel launches.  Errors: BILOCO_ERR_ARG (NULL pointer, workspace
+ * too small), _SHAPE (N, K < 1, r out of range, T < 1, N K > 2^31), _ALIGN,
+ * _DEVICE, _CUDA.
+ */
+size_t biloco_decompose_workspace_bytes(int N, int K, int r);
+int biloco_decompose(const float *W, int N, int K, int r, int T, const uint32_t *v0bits,
+                     uint32_t *Ubits, uint32_t *Vbits, float *alpha, float *R_out,
+                     void *workspace, size_t workspace_bytes, biloco_stream_t stream);
+
+/*
  * biloco_gemm - y = FP4(x) FP4(R)^T + sum_i alpha_i (x . v_i) u_i, in BF16.
  * (BiLoCo README, section "Kernel": one launch for decode batches; the FP4 GEMM
  * on tensor cores, z = alpha . (V x) on CUDA cores from bit-packed V, U z expanded
@@ -148,7 +182,7 @@ size_t biloco_weight_sf_bytes(int N, int K);
  *   limits  1 <= M <= 128, N % 128 == 0, N <= 2^24, K % 64 == 0, 0 <= r <= 1024,
  *           (N/128) * ceil(K/256) <= 2^24
  * Accumulation is FP32 in an unspecified order; results are deterministic for a
- * fixed shape, mode and GPU.  Decode batches (M <= 16, shared-z schedule) run
+ * fixed shape, mode and GPU.  Decode batches (M <= 32, shared-z schedule) run
  * one kernel that quantises the activation itself; otherwise an activation
  * quantiser runs first for M > 8 (biloco_gemm_kernel_count).
  * The fused kernel is launched with programmatic dependent launch: it may start
@@ -157,6 +191,18 @@ size_t biloco_weight_sf_bytes(int N, int K);
  * operand must not be written by a preceding kernel that triggers early launch
  * of its dependents (griddepcontrol.launch_dependents); kernels without that
  * trigger, biloco_pack_weight's included, are fully ordered before the call.
+ *
+ * Residency: the GEMM kernel runs one CTA per SM on G = min(#SMs, units) CTAs
+ * that exchange data behind grid-wide arrival counters, so all G CTAs must be
+ * resident together.  The host checks that one CTA per SM fits
+ * (BILOCO_ERR_RESIDENCY otherwise).  With the default launch form
+ * (BILOCO_LAUNCH_PDL) the GPU must also not be shared with long-running kernels
+ * on other streams, or with another biloco_gemm call running concurrently on
+ * another stream: CTAs that cannot start leave the others waiting, and after
+ * their bounded wait (about 1 s) they give up and biloco_last_error reports
+ * BILOCO_ERR_TIMEOUT (y is then not valid).  Where the GPU is shared, select
+ * BILOCO_LAUNCH_COOPERATIVE (biloco_set_launch): the driver then starts the
+ * grid only once all of its CTAs can be resident.
  */
 int biloco_gemm(const void *x_bf16, const uint8_t *W_fp4, const uint8_t *W_sf,
                 const float *gscale, const uint32_t *Ubits, const uint32_t *Vbits,
@@ -176,13 +222,22 @@ int biloco_gemm(const void *x_bf16, const uint8_t *W_fp4, const uint8_t *W_sf,
  * device code; the call never calls cudaMalloc or cudaFree.  Extra limits,
  * checked on the host before anything is launched (BILOCO_ERR_SHAPE otherwise):
  *   N <= BILOCO_NOALLOC_MAX_N, and the call's scratch fits the array.  That
- *   scratch is 16 896 bytes of status and counters plus, each rounded up to 256:
- *     M > 8:  M*K/2 + ceil(K/256)*2048          (quantised activation)
- *     r > 0:  (ceil(K/256) + 1) * M * rpad * 4  (z partials and z; rpad = 16*ceil(r/16))
- *     always: 2 * G * BN * 512                  (split-K partials)
- *   with G = min(#SMs, (N/128)*ceil(K/256)) and BN = 16, 32, 64, 128 for
- *   M <= 16, 32, 64, 128.  On a 148-SM B200 every M <= 32 shape with
- *   K <= 13824 and r <= 512 fits; M > 64 fits only tiny weights.
+ *   scratch is 16 896 bytes of status and counters plus, each rounded up to 256,
+ *   with KC = ceil(K/256), G = min(#SMs, (N/128)*KC) and rpad = 16*ceil(r/16):
+ *   decode-batch kernel (M <= 32, shared-z schedule, ceil(units/G) <= 16 for
+ *   M <= 16 or <= 64 above; BN = 16 for M <= 16, else 32):
+ *     KC * (M <= 16 ? 2304 : 6144)             (quantised activation image)
+ *     ztile + max(G, ceil(r/128)) * BN * 512   (z tiles, V-side partial sums;
+ *                                               ztile = 65536 or 131072)
+ *     M * rpad * 4                             (z)
+ *     2 * G * BN * 512                         (split-K partials)
+ *   general kernel (every other shape; BN = 16, 32, 64, 128 for M <= 16, 32,
+ *   64, 128):
+ *     M > 8:  M*K/2 + KC*2048                  (quantised activation)
+ *     r > 0:  (KC + 1) * M * rpad * 4          (z partials and z)
+ *     always: 2 * G * BN * 512                 (split-K partials)
+ *   On a 148-SM B200 every M <= 32 shape with K <= 13824 and r <= 1024 fits;
+ *   M > 64 fits only tiny weights.
  * Caveats:
  *   - There is one array per device, shared by all streams and host threads:
  *     calls that overlap in time (on different streams, or from several threads
@@ -200,6 +255,41 @@ int biloco_gemm_noalloc(const void *x_bf16, const uint8_t *W_fp4, const uint8_t 
                         const float *alpha, void *y_bf16, int M, int N, int K, int r,
                         biloco_stream_t stream);
 
+/*
+ * Launch form of the GEMM kernels for later biloco_gemm / biloco_gemm_noalloc
+ * calls (process-wide), a combination of:
+ *   BILOCO_LAUNCH_PDL          programmatic dependent launch: the kernel may start
+ *                              while the kernel before it on the stream finishes
+ *                              (its weight stream overlaps that kernel's tail)
+ *   BILOCO_LAUNCH_COOPERATIVE  cooperative launch: every CTA of the grid is
+ *                              resident together, whatever else runs on the GPU
+ * Default BILOCO_LAUNCH_PDL.  With both flags the grid is launched with both
+ * attributes where the driver accepts the pair, else cooperative only.  Not part
+ * of the BiLoCo pages.  BILOCO_ERR_ARG for unknown flags.
+ */
+enum { BILOCO_LAUNCH_PDL = 1, BILOCO_LAUNCH_COOPERATIVE = 2 };
+int biloco_set_launch(int flags);
+int biloco_get_launch(void);
+
+/*
+ * Arithmetic of the correction's U side on the CUDA cores (the decode-batch
+ * kernel at 1-2 rows; every other shape ignores it), for later calls
+ * (process-wide):
+ *   BILOCO_CORR_SIGNS  sign-adds: every rank's z added or subtracted per weight row
+ *   BILOCO_CORR_LUT    table lookups: each CTA that completes a tile builds, from
+ *                      z, the 16 signed sums of every group of four ranks
+ *                      (FluxBin, "LUT-based Multiplication"; the BiLoCo README's
+ *                      LUT branch), and a weight row adds one entry per four ranks
+ *   BILOCO_CORR_AUTO   the measured choice per shape
+ * Both give y within the stated tolerance of the oracle (different FP32 summation
+ * orders).  BILOCO_ERR_ARG for an unknown value.  Not part of the BiLoCo pages'
+ * API.
+ */
+enum { BILOCO_CORR_AUTO = 0, BILOCO_CORR_SIGNS = 1, BILOCO_CORR_LUT = 2 };
+int biloco_set_correction(int arith);
+/* The arithmetic biloco_gemm would use for this shape under the current setting. */
+int biloco_resolve_correction(int M, int N, int K, int r);
+
 /* Select the z schedule for later biloco_gemm calls (process-wide). */
 int biloco_set_mode(int mode);
 /* The schedule biloco_gemm would use for this shape under the current setting. */
@@ -208,9 +298,12 @@ int biloco_resolve_mode(int M, int N, int K, int r);
 /*
  * biloco_last_error - synchronise `stream`, return and clear the first error a
  * kernel on it recorded (BILOCO_ERR_TIMEOUT when a bounded wait expired), or
- * BILOCO_OK.  After an error the stream's scratch counters are reset.  The
- * static scratch of biloco_gemm_noalloc on the current device is checked and
- * reset the same way.
+ * BILOCO_OK.  After an error the stream's scratch counters are reset.  Once
+ * biloco_gemm_noalloc has run on the current device, its static scratch is
+ * checked and reset the same way; because that array serves every stream, the
+ * call then synchronises the whole device first (cudaDeviceSynchronize), so that
+ * a no-allocation call still running on another stream is neither missed nor
+ * cleared while it runs.
  */
 int biloco_last_error(biloco_stream_t stream);
 
@@ -225,12 +318,27 @@ int biloco_last_error(biloco_stream_t stream);
  */
 int biloco_selftest_wait_timeout(biloco_stream_t stream);
 
+/*
+ * biloco_selftest_drop_arrivals - exercise the GEMM's own failure path on the GPU
+ * without a fault.  The next biloco_gemm or biloco_gemm_noalloc call that runs
+ * the decode-batch kernel (M <= 16, shared-z schedule) leaves out the grid-wide
+ * arrivals selected by `mask` (1: the z slices, 2: the activation image, 3:
+ * both); every other call, and every call after that one, is unaffected.  The
+ * CTAs waiting on those arrivals give up after their bounded wait (about 1 s),
+ * leave together, drain their copies and tensor-core work, free their tensor
+ * memory and record BILOCO_ERR_TIMEOUT; y of that call is not valid.  A following
+ * biloco_last_error(stream) reports the timeout and resets the counters, after
+ * which calls on the stream are correct again.  BILOCO_ERR_ARG for a mask outside
+ * 0..3.  The BiLoCo pages have no counterpart of this call.
+ */
+int biloco_selftest_drop_arrivals(int mask);
+
 /* Human-readable name of a status code (static storage). */
 const char *biloco_status_string(int status);
 
 /* Number of kernels biloco_gemm would launch per call for this shape under the
  * current schedule setting: 1 when the GEMM kernel quantises the activation
- * itself (the decode-batch kernel, M <= 16, or the general kernel at M <= 8),
+ * itself (the decode-batch kernel, M <= 32, or the general kernel at M <= 8),
  * else 2 (quantiser + GEMM).  BILOCO_ERR_SHAPE for shapes biloco_gemm rejects.
  * Uses the device's SM count (the current device must be set). */
 int biloco_gemm_kernel_count(int M, int N, int K, int r);

@@ -8,8 +8,9 @@ is its thin ctypes binding.  Build the library with
 """
 
 from ._lib import (  # noqa: F401
-    BilocoError, MODE_AUTO, MODE_LOCAL_Z, MODE_SHARED_Z, MAX_M, MAX_R, gemm, gemm_kernel_count,
-    gemm_noalloc, selftest_wait_timeout,
+    BilocoError, CORR_AUTO, CORR_LUT, CORR_SIGNS, LAUNCH_COOPERATIVE, LAUNCH_PDL, MODE_AUTO, MODE_LOCAL_Z, MODE_SHARED_Z, MAX_M, MAX_R,
+    decompose, gemm, gemm_kernel_count, gemm_noalloc, get_launch, selftest_drop_arrivals, selftest_wait_timeout,
+    resolve_correction, set_correction, set_launch,
     last_error, load, pack_signs, pack_weight, quant_act, resolve_mode, set_mode, shutdown,
     status_string, weight_sf_bytes,
 )

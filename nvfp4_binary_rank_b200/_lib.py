@@ -18,7 +18,9 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libbiloco.so")
 
 OK = 0
-ERR_ARG, ERR_SHAPE, ERR_ALIGN, ERR_CUDA, ERR_TIMEOUT, ERR_NOMEM, ERR_DEVICE = range(-1, -8, -1)
+ERR_ARG, ERR_SHAPE, ERR_ALIGN, ERR_CUDA, ERR_TIMEOUT, ERR_NOMEM, ERR_DEVICE, ERR_RESIDENCY = range(-1, -9, -1)
+LAUNCH_PDL, LAUNCH_COOPERATIVE = 1, 2
+CORR_AUTO, CORR_SIGNS, CORR_LUT = 0, 1, 2
 MODE_AUTO, MODE_SHARED_Z, MODE_LOCAL_Z = 0, 1, 2
 MAX_M, MAX_R = 128, 1024
 
@@ -34,12 +36,19 @@ SIGNATURES = {
     "biloco_pack_signs": (_I, [_P, _I, _I, _P, _P]),
     "biloco_pack_weight": (_I, [_P, _I, _I, _P, _P, _P, _P]),
     "biloco_weight_sf_bytes": (ctypes.c_size_t, [_I, _I]),
+    "biloco_decompose_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I]),
+    "biloco_decompose": (_I, [_P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "biloco_gemm": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
     "biloco_gemm_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
     "biloco_set_mode": (_I, [_I]),
     "biloco_resolve_mode": (_I, [_I, _I, _I, _I]),
     "biloco_last_error": (_I, [_P]),
     "biloco_selftest_wait_timeout": (_I, [_P]),
+    "biloco_selftest_drop_arrivals": (_I, [_I]),
+    "biloco_set_launch": (_I, [_I]),
+    "biloco_get_launch": (_I, []),
+    "biloco_set_correction": (_I, [_I]),
+    "biloco_resolve_correction": (_I, [_I, _I, _I, _I]),
     "biloco_status_string": (ctypes.c_char_p, [_I]),
     "biloco_gemm_kernel_count": (_I, [_I, _I, _I, _I]),
     "biloco_shutdown": (None, []),
@@ -134,6 +143,31 @@ def pack_weight(R: torch.Tensor, stream=None):
     return W, sf, g
 
 
+def decompose(W: torch.Tensor, r: int, T: int, v0bits: torch.Tensor | None, stream=None):
+    """float32 [N, K] -> (Ubits int32 [N, ceil(r/32)], Vbits int32 [r, ceil(K/32)],
+    alpha float32 [r], R float32 [N, K]) with W ~= U diag(alpha) V^T + R.
+    v0bits: int32 [r, ceil(K/32)], the packed start signs of each term."""
+    _need_cuda(W, "W", torch.float32)
+    N, K = W.shape
+    RW, KW = (r + 31) // 32, (K + 31) // 32
+    if r:
+        _need_cuda(v0bits, "v0bits", torch.int32)
+        if tuple(v0bits.shape) != (r, KW):
+            raise ValueError("v0bits must be [r, ceil(K/32)]")
+    Ub = torch.empty((N, max(RW, 1)), dtype=torch.int32, device=W.device)
+    Vb = torch.empty((max(r, 1), KW), dtype=torch.int32, device=W.device)
+    alpha = torch.empty((max(r, 1),), dtype=torch.float32, device=W.device)
+    R = torch.empty_like(W)
+    nbytes = int(load().biloco_decompose_workspace_bytes(N, K, r))
+    if nbytes == 0:
+        raise BilocoError("biloco_decompose_workspace_bytes", ERR_SHAPE)
+    ws = torch.empty((nbytes,), dtype=torch.uint8, device=W.device)
+    _check("biloco_decompose", load().biloco_decompose(
+        _ptr(W), N, K, r, T, _ptr(v0bits if r else None), _ptr(Ub), _ptr(Vb), _ptr(alpha), _ptr(R),
+        _ptr(ws), nbytes, _stream(stream)))
+    return Ub[:, :RW], Vb[:r], alpha[:r], R
+
+
 def _gemm_call(fn: str, x, W_fp4, W_sf, gscale, Ubits, Vbits, alpha, out, stream):
     _need_cuda(x, "x", torch.bfloat16)
     _need_cuda(W_fp4, "W_fp4", torch.uint8)
@@ -189,6 +223,31 @@ def selftest_wait_timeout(stream=None):
     """Launch the bounded-wait self test (about 1 s on the GPU); biloco_last_error
     on the same stream then reports BILOCO_ERR_TIMEOUT."""
     _check("biloco_selftest_wait_timeout", load().biloco_selftest_wait_timeout(_stream(stream)))
+
+
+def selftest_drop_arrivals(mask: int):
+    """Make the next decode-kernel GEMM call leave out the grid arrivals in `mask`
+    (1: z slices, 2: activation image); its bounded waits expire after about 1 s
+    and biloco_last_error then reports BILOCO_ERR_TIMEOUT."""
+    _check("biloco_selftest_drop_arrivals", load().biloco_selftest_drop_arrivals(int(mask)))
+
+
+def set_launch(flags: int):
+    """Launch form of the GEMM kernels: LAUNCH_PDL, LAUNCH_COOPERATIVE or both."""
+    _check("biloco_set_launch", load().biloco_set_launch(int(flags)))
+
+
+def set_correction(arith: int):
+    """Correction arithmetic of the 1-2-row U side: CORR_AUTO, CORR_SIGNS or CORR_LUT."""
+    _check("biloco_set_correction", load().biloco_set_correction(int(arith)))
+
+
+def resolve_correction(M: int, N: int, K: int, r: int) -> int:
+    return int(load().biloco_resolve_correction(M, N, K, r))
+
+
+def get_launch() -> int:
+    return int(load().biloco_get_launch())
 
 
 def last_error(stream=None) -> int:

@@ -19,6 +19,9 @@ namespace {
 
 std::mutex g_mu;
 std::atomic<int> g_mode{BILOCO_MODE_AUTO};
+std::atomic<int> g_launch{BILOCO_LAUNCH_PDL};
+std::atomic<int> g_arith{BILOCO_CORR_AUTO};
+std::atomic<int> g_drop{0};   // failure-path self test, consumed by the next GEMM call
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
@@ -174,7 +177,17 @@ int check_gemm_args(const void* x_bf16, const uint8_t* W_fp4, const uint8_t* W_s
   a->K = K;
   a->r = r;
   a->mode = resolve_mode(M, N, K, r, g_mode.load());
+  a->arith = resolve_arith(M, N, K, r, g_arith.load());
+  a->drop = g_drop.exchange(0);
   return BILOCO_OK;
+}
+
+LaunchOpts current_launch_opts() {
+  LaunchOpts o;
+  const int f = g_launch.load();
+  o.pdl = (f & BILOCO_LAUNCH_PDL) != 0;
+  o.cooperative = (f & BILOCO_LAUNCH_COOPERATIVE) != 0;
+  return o;
 }
 
 }  // namespace biloco
@@ -245,6 +258,28 @@ int biloco_selftest_wait_timeout(biloco_stream_t stream) {
   return launch_wait_timeout(sc->status, s) == cudaSuccess ? BILOCO_OK : BILOCO_ERR_CUDA;
 }
 
+int biloco_selftest_drop_arrivals(int mask) {
+  if (mask < 0 || mask > 3) return BILOCO_ERR_ARG;
+  g_drop.store(mask);
+  return BILOCO_OK;
+}
+
+int biloco_set_launch(int flags) {
+  if (flags < 0 || flags > (BILOCO_LAUNCH_PDL | BILOCO_LAUNCH_COOPERATIVE)) return BILOCO_ERR_ARG;
+  g_launch.store(flags);
+  return BILOCO_OK;
+}
+
+int biloco_get_launch(void) { return g_launch.load(); }
+
+int biloco_set_correction(int arith) {
+  if (arith != BILOCO_CORR_AUTO && arith != BILOCO_CORR_SIGNS && arith != BILOCO_CORR_LUT) return BILOCO_ERR_ARG;
+  g_arith.store(arith);
+  return BILOCO_OK;
+}
+
+int biloco_resolve_correction(int M, int N, int K, int r) { return resolve_arith(M, N, K, r, g_arith.load()); }
+
 int biloco_set_mode(int mode) {
   if (mode != BILOCO_MODE_AUTO && mode != BILOCO_MODE_SHARED_Z && mode != BILOCO_MODE_LOCAL_Z)
     return BILOCO_ERR_ARG;
@@ -290,6 +325,7 @@ const char* biloco_status_string(int status) {
     case BILOCO_ERR_TIMEOUT: return "device-side wait timed out";
     case BILOCO_ERR_NOMEM: return "scratch allocation failed";
     case BILOCO_ERR_DEVICE: return "device is not sm_100";
+    case BILOCO_ERR_RESIDENCY: return "grid cannot be resident on the GPU at once";
     default: return "unknown status";
   }
 }

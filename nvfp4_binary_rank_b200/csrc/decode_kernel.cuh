@@ -65,21 +65,13 @@ constexpr int kAluWarp0 = 6;
 constexpr int kAluWarps = 8;
 constexpr int kAluThreads = kAluWarps * 32;
 constexpr int kFinThreads = kEpiThreads + kAluThreads;
-constexpr int kBN = 16;                   // MMA N (activation rows, padded)
-constexpr int kRowsMax = 16;              // activation rows handled
+constexpr int kRowsMax = 32;              // activation rows handled (the largest class)
 constexpr int kTileRows = 128;            // weight rows per tile = MMA M
 constexpr int kUnitK = 256;               // K elements per unit
 constexpr int kUnitBytesA = kTileRows * 128;
 constexpr int kSfBytes = 2048;            // 4 scale atoms of 512 B per unit
-constexpr int kMaxUnits = 16;             // units per CTA (operand cache entries)
 constexpr int kMaxRanks = 1024;
-// TMEM columns: accumulators [0, 32); activation scales per unit [32, 288);
-// weight scales per stage [288, 384); the U-side product [384, 416)
 constexpr int kTmemCols = 512;
-constexpr int kSfbTmemBase = 32;
-constexpr int kSfaTmemBase = kSfbTmemBase + 16 * 16;
-constexpr int kUTmem = 384;
-constexpr int kVTmem = 448;               // V side on the tensor cores: 16 columns
 constexpr int kVAtoms = 3;                // K atoms (64 elements) per V-side MMA batch
 constexpr int kUChunk = 64;               // ranks per U-side MMA chunk (one 128-byte BF16 row)
 constexpr int kUChunksMax = 16;           // r <= 1024
@@ -93,11 +85,19 @@ constexpr int kBarFin2 = 4;               // epilogue + CUDA cores: correction r
 constexpr int kBarZ = 5;                  // epilogue + CUDA cores: z staged (1-2 rows)
 
 // Per batch class (MC = most activation rows): weight stages and V-side ranks
-// per pass (the largest class trades stages and ranks for its z and register
+// per pass (the larger classes trade stages for their z and register
 // footprint).
 template <int MC>
 struct Cfg {
-  static constexpr int kStages = (MC >= 16) ? 4 : 6;
+  // Up to 16 rows the activation chunks of all of a CTA's units sit in an operand
+  // cache in shared memory (at most kMaxUnits units per CTA).  The 32-row class
+  // streams them instead: each stage carries one weight unit and the matching
+  // activation chunk (codes and scale atoms) from the grid's activation image,
+  // and both sets of block scales go to TMEM per stage.
+  static constexpr bool kStream = MC > 16;
+  static constexpr int kBN = kStream ? 32 : 16;            // MMA N (activation rows, padded)
+  static constexpr int kMaxUnits = kStream ? 64 : 16;      // units per CTA
+  static constexpr int kStages = kStream ? 5 : ((MC >= 16) ? 4 : 6);
   static constexpr int kRankGroup = 4;                     // ranks per V-side pass
   // V-side load ring depth (blocks in flight per warp); below 8 rows a warp walks
   // only two or three K blocks
@@ -118,44 +118,84 @@ struct Cfg {
   // x a slice of K, with the partial sums reduced across CTAs (with 8 the CUDA-core
   // loop is faster, measured on B200)
   static constexpr bool kTensorV = MC >= 16;
+  // z tiles of the tensor-core U side held in shared memory at once (64 ranks
+  // each); the 32-row class cycles larger ranks through them
+  static constexpr int kZSlots = kStream ? 8 : 16;
 };
 
-// Global activation image (8+ rows): per 256-element K chunk, the 16 x 128 B code
-// rows exactly as the operand cache holds them (128-byte swizzle), then 256 B of
-// block scales, 64 B per 64-element K step (row m at byte 4 m, block b of the step
-// at byte b).
-constexpr int kQImgCodes = kBN * 128;
-constexpr int kQImgBytes = kQImgCodes + 256;
-static_assert(kQImgBytes == kDecodeQImgBytes, "activation image size differs from the host's");
+// Global activation image (8+ rows), per 256-element K chunk:
+//  * classes 8 and 16: the 16 x 128 B code rows exactly as the operand cache holds
+//    them (128-byte swizzle), then 256 B of block scales, 64 B per 64-element K
+//    step (row m at byte 4 m, block b of the step at byte b);
+//  * class 32: the 32 x 128 B code rows (128-byte swizzle), then the block scales
+//    as four 512-byte scale atoms, one per K step, in the layout the tensor
+//    memory copy expects (row m's four scales at bytes 16 m .. 16 m + 3, the other
+//    12 bytes of the row zero).  A stage's activation part is one bulk copy of it.
+template <int MC>
+struct QImg {
+  static constexpr int kCodes = Cfg<MC>::kBN * 128;
+  static constexpr int kBytes = kCodes + (Cfg<MC>::kStream ? 4 * 512 : 256);
+};
 
 template <int MC>
 struct Layout {
   static constexpr int kStages = Cfg<MC>::kStages;
   static constexpr int kRankGroup = Cfg<MC>::kRankGroup;
-  static constexpr int kA = 0;                                        // [ST][128][128 B]
+  static constexpr int kBN = Cfg<MC>::kBN;
+  static constexpr int kMaxUnits = Cfg<MC>::kMaxUnits;
+  static constexpr bool kStream = Cfg<MC>::kStream;
+  // a stage: the weight unit's codes and scale atoms, and (streamed classes) the
+  // activation chunk's codes and scale atoms
+  static constexpr int kStageA = 0;
+  static constexpr int kStageSFA = kUnitBytesA;
+  static constexpr int kStageB = kStageSFA + kSfBytes;
+  static constexpr int kStageSFB = kStageB + kBN * 128;
+  static constexpr int kStageBytes = kStageSFB + kSfBytes;
+  static_assert(kStageBytes == kUnitBytesA + kSfBytes + QImg<MC>::kBytes || !kStream,
+                "a stage's activation part is one image chunk");
+  static constexpr int kA = 0;                                        // [ST][128][128 B] (cache classes)
   static constexpr int kSFA = kA + kStages * kUnitBytesA;              // [ST][2 KB]
-  static constexpr int kB = kSFA + kStages * kSfBytes;                 // [NU][16][128 B]
+  static constexpr int kB = kSFA + kStages * kSfBytes;                 // [NU][16][128 B] operand cache
   static constexpr int kSFB = kB + kMaxUnits * kBN * 128;              // [NU][4 steps][32 rows] u32
+  static constexpr int kCacheEnd = kSFB + kMaxUnits * 512;
+  // first byte past the stages (streamed) or the operand cache
+  static constexpr int kFree = kStream ? kStages * kStageBytes : kCacheEnd;
   // U side on the tensor cores: A = the tile's U signs as +-1 BF16, 64 ranks per
   // chunk (two buffers); B = z as BF16 high and low parts, kUN rows per chunk
   static constexpr int kUN = (2 * MC < 16) ? 16 : 2 * MC;               // MMA N of the U side
-  static constexpr int kUA = kSFB + kMaxUnits * 512;                   // [2][128][128 B]
-  static constexpr int kUZ = kUA + 2 * kTileRows * 128;                // [16][kUN][128 B]
-  // without the tensor-core U side: z staged as floats and the two half sums
-  static constexpr int kZ = kSFB + kMaxUnits * 512;                    // [MC][1024] floats
+  static constexpr int kUA = kFree;                                     // [2][128][128 B]
+  static constexpr int kUZ = kUA + 2 * kTileRows * 128;                // [kZSlots][kUN][128 B]
+  // without the tensor-core U side: z staged as floats, the two half sums, and the
+  // signed-sum table of z (16 entries per 4 ranks)
+  static constexpr int kZ = kFree;                                     // [MC][1024] floats
   static constexpr int kCorr = kZ + MC * kMaxRanks * 4;                // [2][MC][128] floats
-  static constexpr int kUEnd = Cfg<MC>::kTensorU ? kUZ + kUChunksMax * kUN * 128
-                                                 : kCorr + 2 * MC * kTileRows * 4;
+  static constexpr int kLut = kCorr + 2 * MC * kTileRows * 4;          // [MC][256 groups][16] floats
+  static constexpr int kUEnd = Cfg<MC>::kTensorU ? kUZ + Cfg<MC>::kZSlots * kUN * 128
+                                                 : kLut + MC * kMaxRanks * 16;
   static constexpr int kVRed = kUEnd;                                  // [8][MC * ranks] floats
-  static constexpr int kBar = kVRed + kAluWarps * MC * kRankGroup * 4;
+  static constexpr int kVRedBytes = Cfg<MC>::kTensorV ? 0 : kAluWarps * MC * kRankGroup * 4;
+  static constexpr int kBar = kVRed + kVRedBytes;
   static constexpr int kNumBars = 2 * kStages + 13;
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kFinFlags = kMisc + 32;                         // [kMaxUnits + 1] ints
   static constexpr int kTotal = kFinFlags + (kMaxUnits + 1) * 4;
   static constexpr int kAlloc = kTotal + 1024;
-  static_assert(kSFA % 1024 == 0 && kB % 1024 == 0 && kUA % 1024 == 0 && kUZ % 1024 == 0,
-                "swizzled tiles need 1 KB alignment");
+  // TMEM columns.  Cache classes: accumulators [0, 32), activation scales per unit
+  // [32, 288), weight scales per stage [288, 384), the U-side product [384, 416),
+  // the V-side product [448, 464).  Streamed class: accumulators [0, 64), weight
+  // and activation scales per stage, then the U-side (64) and V-side (32) products.
+  static constexpr int kTmSfb = kStream ? 2 * kBN + kStages * 16 : 32;
+  static constexpr int kTmSfa = kStream ? 2 * kBN : kTmSfb + kMaxUnits * 16;
+  static constexpr int kTmU = kStream ? kTmSfb + kStages * 16 : 384;
+  static constexpr int kTmV = kStream ? kTmU + kUN : 448;
+  static_assert(kTmV + kBN <= kTmemCols, "tensor memory budget");
+  static_assert(kStream || kTmSfa + kStages * 16 <= kTmU, "tensor memory budget");
+  static_assert(kSFA % 1024 == 0 && kB % 1024 == 0 && kUA % 1024 == 0 && kUZ % 1024 == 0 &&
+                kStageBytes % 1024 == 0 && kStageB % 1024 == 0, "swizzled tiles need 1 KB alignment");
   static_assert(kAlloc <= 232448, "shared memory budget");
+  // the tensor-core V side's buffers alias the U side's (unused until z is complete)
+  static_assert(!Cfg<MC>::kTensorV || kVAtoms * (kTileRows + kBN) * 128 <= kUEnd - kUA,
+                "V-side buffers fit the U side's");
 };
 
 // One z value's two BF16 parts into the global tile image of the U side's B
@@ -297,11 +337,154 @@ __device__ __forceinline__ void vside_rows(const DecodeParams& p, int ig, int nr
     for (int i = 0; i < kRankGroup; ++i) acc[j][i] = f32x2_sum(acc2[j][i]);
 }
 
+// Signed-sum table of z for the CUDA-core U side (the LUT form of the correction
+// arithmetic): for every row m and group g of four ranks, entry b (0..15) is
+// sum_j (bit j of b ? -z[4 g + j] : z[4 g + j]), so that the four sign bits of a
+// weight row select the row's contribution of those ranks with one load.  Built
+// from the staged z (zero past r) by `nthreads` threads.
 template <int MC>
+__device__ __forceinline__ void build_z_table(const float* zs, float* lut, int M, int RW, int tid, int nthreads) {
+  const int groups = 8 * RW;
+  for (int idx = tid; idx < M * groups; idx += nthreads) {
+    const int m = idx / groups, g = idx - m * groups;
+    const float4 z = *reinterpret_cast<const float4*>(zs + m * kMaxRanks + 4 * g);
+    float4* t = reinterpret_cast<float4*>(lut + (m * (kMaxRanks / 4) + g) * 16);
+    float e[16];
+#pragma unroll
+    for (int b = 0; b < 16; ++b)
+      e[b] = (((b & 1) ? -z.x : z.x) + ((b & 2) ? -z.y : z.y)) + (((b & 4) ? -z.z : z.z) + ((b & 8) ? -z.w : z.w));
+#pragma unroll
+    for (int q4 = 0; q4 < 4; ++q4) t[q4] = make_float4(e[4 * q4], e[4 * q4 + 1], e[4 * q4 + 2], e[4 * q4 + 3]);
+  }
+}
+
+// One rank word (32 ranks from word index w) of a weight row's U z, added into
+// four interleaved sums per activation row: sign-adds on the staged z, or (lut)
+// eight lookups in the signed-sum table.
+template <int MC, bool kLut>
+__device__ __forceinline__ void u_word_sum(const float* zs, const float* lut, uint32_t word, int w, int M,
+                                           float (&acc4)[MC][4]) {
+  if constexpr (kLut) {
+    const float* tw = lut + w * 8 * 16;
+#pragma unroll
+    for (int nb = 0; nb < 8; ++nb) {
+      const uint32_t nib = (word >> (4 * nb)) & 15u;
+#pragma unroll
+      for (int m = 0; m < MC; ++m)
+        if (m < M) acc4[m][nb & 3] += tw[m * (kMaxRanks / 4) * 16 + nb * 16 + nib];
+    }
+  } else {
+    const float* zw = zs + w * 32;
+#pragma unroll
+    for (int j4 = 0; j4 < 8; ++j4) {
+#pragma unroll
+      for (int m = 0; m < MC; ++m) {
+        if (m < M) {
+          const float4 z4 = *reinterpret_cast<const float4*>(zw + m * kMaxRanks + 4 * j4);
+          const float zz[4] = {z4.x, z4.y, z4.z, z4.w};
+#pragma unroll
+          for (int jj = 0; jj < 4; ++jj) {
+            const uint32_t sgn = (word << (31 - (4 * j4 + jj))) & 0x80000000u;
+            acc4[m][jj] += __uint_as_float(__float_as_uint(zz[jj]) ^ sgn);
+          }
+        }
+      }
+    }
+  }
+}
+
+// The operand cache starts zero: rows >= M and blocks past K stay zero.
+template <int MC>
+__device__ __forceinline__ void zero_cache(uint8_t* smem, int nunits, int tid, int nthreads) {
+  using L = Layout<MC>;
+  for (int idx = tid; idx < nunits * 160; idx += nthreads) {
+    const int k = idx / 160, o = idx - k * 160;
+    uint4* dst = (o < 128) ? reinterpret_cast<uint4*>(smem + L::kB + k * L::kBN * 128) + o
+                           : reinterpret_cast<uint4*>(smem + L::kSFB + k * 512) + (o - 128);
+    *dst = make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
+// Quantise the activation chunks of every unit of this CTA into the operand cache
+// (codes in the MMA's 128-byte-swizzled rows, scales staged for TMEM): two blocks
+// per thread per round, the loop rolled (the quantiser is long straight-line code;
+// unrolled deeper it would crowd the instruction cache).
+template <int MC>
+__device__ __forceinline__ void quant_into_cache(const DecodeParams& p, uint8_t* smem, int u0, int nunits, int tid,
+                                                 int nthreads) {
+  using L = Layout<MC>;
+  constexpr int kQB = 2;
+  const int per_unit = p.M * 16;
+  const int items = nunits * per_unit;
+#pragma unroll 1
+  for (int base = 0; base < items; base += nthreads * kQB) {
+    uint4 lo[kQB], hi[kQB];
+#pragma unroll
+    for (int e = 0; e < kQB; ++e) {
+      const int idx = base + e * nthreads + tid;
+      lo[e] = hi[e] = make_uint4(0u, 0u, 0u, 0u);
+      if (idx < items) {
+        const int k = idx / per_unit, rem = idx - k * per_unit, m = rem >> 4, blk = rem & 15;
+        const int kk = ((u0 + k) % p.KC) * kUnitK + blk * 16;
+        if (kk < p.K) {
+          const uint4* src = reinterpret_cast<const uint4*>(p.x + static_cast<size_t>(m) * p.K + kk);
+          lo[e] = __ldcg(src);
+          hi[e] = __ldcg(src + 1);
+        }
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < kQB; ++e) {
+      const int idx = base + e * nthreads + tid;
+      if (idx < items) {
+        const int k = idx / per_unit, rem = idx - k * per_unit, m = rem >> 4, blk = rem & 15;
+        const int kk = ((u0 + k) % p.KC) * kUnitK + blk * 16;
+        if (kk < p.K) {
+          float v[16];
+          bf16x16_to_f32(lo[e], hi[e], v);
+          uint2 codes;
+          const uint32_t s = quant_act_block_fast(v, codes);
+          const int j = blk * 8;
+          *reinterpret_cast<uint2*>(smem + L::kB + k * L::kBN * 128 + m * 128 +
+                                    ((((j >> 4) ^ (m & 7)) << 4) | (j & 15))) = codes;
+          smem[L::kSFB + k * 512 + (blk >> 2) * 128 + m * 4 + (blk & 3)] = static_cast<uint8_t>(s);
+        }
+      }
+    }
+  }
+}
+
+// Activation scales to TMEM, in the layout a 32x128b.warpx4 copy of scale atoms
+// would give: lane i of every lane quarter holds, in column 16 k + 4 j, the four
+// block scales of row i for K step j of unit k (rows >= 16 and the other three
+// columns of a step are zero).  Called by one warp per lane quarter.
+template <int MC>
+__device__ __forceinline__ void sfb_to_tmem(const uint8_t* smem, uint32_t tmem, int nunits, uint32_t quarter,
+                                            int lane) {
+  using L = Layout<MC>;
+  for (int k = 0; k < nunits; ++k) {
+    const uint32_t* sfb = reinterpret_cast<const uint32_t*>(smem + L::kSFB + k * 512) + lane;
+    uint32_t v[16];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      v[4 * j] = sfb[j * 32];
+      v[4 * j + 1] = v[4 * j + 2] = v[4 * j + 3] = 0u;
+    }
+    tmem_st16(tmem + ((quarter * 32) << 16) + L::kTmSfb + k * 16, v);
+  }
+  tmem_wait_st();
+}
+
+// kLut (1-2 rows): the U side adds lookups in the signed-sum table of z instead of
+// sign-adds (each instance carries only its own loop: the code size of these
+// kernels shows in their instruction-cache misses)
+template <int MC, bool kLut>
 __global__ void __launch_bounds__(kThreads, 1)
 decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ DecodeParams p) {
   using L = Layout<MC>;
   constexpr int kStages = Cfg<MC>::kStages, kRankGroup = Cfg<MC>::kRankGroup;
+  constexpr int kBN = Cfg<MC>::kBN;
+  constexpr bool kStream = Cfg<MC>::kStream;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -376,18 +559,64 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
       int s = 0;
       uint32_t ph = 0;                                   // parity of the stage's current use
       const uint8_t* sf = p.w_sf + static_cast<size_t>(u0) * kSfBytes;
-      for (int k = 0; k < nunits; ++k) {
-        if (k >= kStages && !mbar_wait(empty_bar(s), ph ^ 1u, abort_flag)) {
-          fail(ctl);
-          break;
+      if constexpr (!kStream) {
+        for (int k = 0; k < nunits; ++k) {
+          if (k >= kStages && !mbar_wait(empty_bar(s), ph ^ 1u, abort_flag)) {
+            fail(ctl);
+            break;
+          }
+          mbar_arrive_expect_tx(full_bar(s), kStageTx);
+          tma_load_2d(smem_u32(smem + L::kA + s * kUnitBytesA), &tmap_w, full_bar(s), c * 128, t * kTileRows);
+          bulk_load(smem_u32(smem + L::kSFA + s * kSfBytes), sf, kSfBytes, full_bar(s));
+          ++issued;
+          sf += kSfBytes;
+          if (++c == p.KC) { c = 0; ++t; }
+          if (++s == kStages) { s = 0; ph ^= 1u; }
         }
-        mbar_arrive_expect_tx(full_bar(s), kStageTx);
-        tma_load_2d(smem_u32(smem + L::kA + s * kUnitBytesA), &tmap_w, full_bar(s), c * 128, t * kTileRows);
-        bulk_load(smem_u32(smem + L::kSFA + s * kSfBytes), sf, kSfBytes, full_bar(s));
-        ++issued;
-        sf += kSfBytes;
-        if (++c == p.KC) { c = 0; ++t; }
-        if (++s == kStages) { s = 0; ph ^= 1u; }
+      } else {
+        // A stage = the weight unit (TMA tile + scale atoms) and the activation
+        // chunk of the same K range (one bulk copy of its image chunk).  The weight
+        // parts of the first stages are requested at once; the activation parts
+        // once the CTA's CUDA-core warps have seen every CTA publish its part of
+        // the image (actr_bar), always issued so that every stage's transaction
+        // count completes even after a failed wait.
+        constexpr uint32_t kImg = QImg<MC>::kBytes;
+        const int pre = min(nunits, kStages);
+        for (int k = 0; k < pre; ++k) {
+          uint8_t* st = smem + k * L::kStageBytes;
+          mbar_arrive_expect_tx(full_bar(k), kStageTx + kImg);
+          tma_load_2d(smem_u32(st + L::kStageA), &tmap_w, full_bar(k), c * 128, t * kTileRows);
+          bulk_load(smem_u32(st + L::kStageSFA), sf, kSfBytes, full_bar(k));
+          sf += kSfBytes;
+          if (++c == p.KC) { c = 0; ++t; }
+        }
+        bool ok = mbar_wait(actr_bar, 0, abort_flag);
+        if (!ok) fail(ctl);
+        fence_proxy_async_global();                      // the image was written through the generic proxy
+        int ca = u0 % p.KC;
+        for (int k = 0; k < pre; ++k) {
+          bulk_load(smem_u32(smem + k * L::kStageBytes + L::kStageB), p.xq + static_cast<size_t>(ca) * kImg, kImg,
+                    full_bar(k));
+          if (++ca == p.KC) ca = 0;
+        }
+        issued = pre;
+        s = pre % kStages;
+        ph = (pre == kStages) ? 1u : 0u;
+        for (int k = pre; k < nunits && ok; ++k) {
+          if (!mbar_wait(empty_bar(s), ph ^ 1u, abort_flag)) {
+            fail(ctl);
+            break;
+          }
+          uint8_t* st = smem + s * L::kStageBytes;
+          mbar_arrive_expect_tx(full_bar(s), kStageTx + kImg);
+          tma_load_2d(smem_u32(st + L::kStageA), &tmap_w, full_bar(s), c * 128, t * kTileRows);
+          bulk_load(smem_u32(st + L::kStageSFA), sf, kSfBytes, full_bar(s));
+          bulk_load(smem_u32(st + L::kStageB), p.xq + static_cast<size_t>(c) * kImg, kImg, full_bar(s));
+          ++issued;
+          sf += kSfBytes;
+          if (++c == p.KC) { c = 0; ++t; }
+          if (++s == kStages) { s = 0; ph ^= 1u; }
+        }
       }
       // never leave the CTA with copies in flight
       for (int k = max(0, issued - kStages); k < issued; ++k) {
@@ -409,14 +638,20 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
     if (lane == 0) {
       const uint32_t idesc = (1u << 7) | (1u << 10) | (static_cast<uint32_t>(kBN >> 3) << 17) |
                              (static_cast<uint32_t>(kTileRows >> 4) << 24);
-      const uint64_t a_desc0 = smem_desc(smem_u32(smem + L::kA), 16, 1024, 2);
-      const uint64_t b_desc0 = smem_desc(smem_u32(smem + L::kB), 16, 1024, 2);
-      const uint64_t sfa_desc0 = smem_desc(smem_u32(smem + L::kSFA), 0, 128, 0);
-      constexpr uint64_t kAtom = 512 >> 4, kUnitSf = kSfBytes >> 4;
-      constexpr uint64_t kUnitA = kUnitBytesA >> 4, kUnitB = (kBN * 128) >> 4;
-      // weight scales of the stages already requested go to TMEM while the
-      // activation is still being quantised
-      const int pre = min(nunits, kStages);
+      // cache classes: stage s at kA + s 16 KB (codes) and kSFA + s 2 KB (scales),
+      // activation unit k in the operand cache; streamed class: everything in
+      // stage s at s * kStageBytes
+      const uint64_t a_desc0 = smem_desc(smem_u32(smem + (kStream ? L::kStageA : L::kA)), 16, 1024, 2);
+      const uint64_t b_desc0 = smem_desc(smem_u32(smem + (kStream ? L::kStageB : L::kB)), 16, 1024, 2);
+      const uint64_t sfa_desc0 = smem_desc(smem_u32(smem + (kStream ? L::kStageSFA : L::kSFA)), 0, 128, 0);
+      const uint64_t sfb_desc0 = smem_desc(smem_u32(smem + L::kStageSFB), 0, 128, 0);
+      constexpr uint64_t kAtom = 512 >> 4;
+      constexpr uint64_t kUnitSf = (kStream ? L::kStageBytes : kSfBytes) >> 4;
+      constexpr uint64_t kUnitA = (kStream ? L::kStageBytes : kUnitBytesA) >> 4;
+      constexpr uint64_t kUnitB = (kBN * 128) >> 4, kStageB = L::kStageBytes >> 4;
+      // cache classes: the weight scales of the stages already requested go to
+      // TMEM while the activation is still being quantised
+      const int pre = kStream ? 0 : min(nunits, kStages);
       bool ok = true;
       for (int j = 0; j < pre && ok; ++j) {
         if (!mbar_wait(full_bar(j), 0, abort_flag)) {
@@ -428,10 +663,10 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
         const uint64_t sfa_d = sfa_desc0 + static_cast<uint64_t>(j) * kUnitSf;
 #pragma unroll
         for (int q = 0; q < 4; ++q)
-          tc_cp_32x128b_warpx4(tmem + kSfaTmemBase + j * 16 + 4 * q, sfa_d + kAtom * q);
+          tc_cp_32x128b_warpx4(tmem + L::kTmSfa + j * 16 + 4 * q, sfa_d + kAtom * q);
       }
       // the activation codes (shared memory) and scales (TMEM) are in place
-      if (ok && !mbar_wait(actr_bar, 0, abort_flag)) {
+      if (!kStream && ok && !mbar_wait(actr_bar, 0, abort_flag)) {
         fail(ctl);
         ok = false;
       }
@@ -450,8 +685,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
         tc_fence_after();
         const uint32_t d_tmem = tmem + static_cast<uint32_t>(b * kBN);
         for (int u = ua; u < ub; ++u, ++k) {
-          const uint32_t sfa_t = tmem + kSfaTmemBase + s * 16;
-          const uint32_t sfb_t = tmem + kSfbTmemBase + k * 16;
+          const uint32_t sfa_t = tmem + L::kTmSfa + s * 16;
+          const uint32_t sfb_t = tmem + L::kTmSfb + (kStream ? s : k) * 16;
           if (k >= pre) {
             if (!mbar_wait(full_bar(s), ph, abort_flag)) {
               fail(ctl);
@@ -462,9 +697,15 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
             const uint64_t sfa_d = sfa_desc0 + static_cast<uint64_t>(s) * kUnitSf;
 #pragma unroll
             for (int q = 0; q < 4; ++q) tc_cp_32x128b_warpx4(sfa_t + 4 * q, sfa_d + kAtom * q);
+            if constexpr (kStream) {
+              const uint64_t sfb_d = sfb_desc0 + static_cast<uint64_t>(s) * kStageB;
+#pragma unroll
+              for (int q = 0; q < 4; ++q) tc_cp_32x128b_warpx4(sfb_t + 4 * q, sfb_d + kAtom * q);
+            }
           }
           const uint64_t a_d = a_desc0 + static_cast<uint64_t>(s) * kUnitA;
-          const uint64_t b_d = b_desc0 + static_cast<uint64_t>(k) * kUnitB;
+          const uint64_t b_d = kStream ? b_desc0 + static_cast<uint64_t>(s) * kStageB
+                                       : b_desc0 + static_cast<uint64_t>(k) * kUnitB;
 #pragma unroll
           for (int j = 0; j < 4; ++j)
             tc_mma_nvf4(d_tmem, a_d + 2 * j, b_d + 2 * j, idesc, sfa_t + 4 * j, sfb_t + 4 * j,
@@ -487,12 +728,24 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
     __syncwarp();
   } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + 4) {
     // ---------------------------------------------------------------- epilogue
-    griddep_wait();
     const int q = warp & 3;                            // TMEM lane quarter of this warp
     const int row = q * 32 + lane;                     // weight row within the tile
     const int etid = threadIdx.x - kEpiWarp0 * 32;
+    griddep_wait();
     const float gs = __ldcg(p.gscale);
-    constexpr int kHB = (MC <= 2) ? 16 : (MC <= 4 ? 8 : (MC <= 8 ? 4 : 2));   // partials loaded per batch
+    constexpr int kHB = (MC <= 2) ? 16 : (MC <= 4 ? 8 : (MC <= 8 ? 4 : (MC <= 16 ? 2 : 1)));   // partials loaded per batch
+    // the accumulator of buffer b for this warp's lane quarter, times g
+    auto load_acc = [&](int b, float (&v)[MC]) {
+#pragma unroll
+      for (int c0 = 0; c0 < MC; c0 += 16) {
+        uint32_t raw[16];
+        tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(b * kBN + c0), raw);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          if (c0 + j < MC) v[c0 + j] = __fmul_rn(gs, __uint_as_float(raw[j]));
+      }
+    };
     if constexpr (Cfg<MC>::kUShares) {
       bool ok = true;
       for (int seg = 0; seg < nseg; ++seg) {
@@ -506,11 +759,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
         if (ok) ok = group_wait(accf_bar(b), (seg >> 1) & 1, kBarEpi, kEpiThreads, ctl);
         if (ok) {
           tc_fence_after();
-          uint32_t raw[16];
-          tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(b * kBN), raw);
-          tmem_wait_ld();
-  #pragma unroll
-          for (int j = 0; j < MC; ++j) v[j] = __fmul_rn(gs, __uint_as_float(raw[j]));
+          load_acc(b, v);
           tc_fence_before();
           mbar_arrive(acce_bar(b));
         }
@@ -532,20 +781,35 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
             // sum_i U[n][i] zlo[m][i] in column MC + m of lane n
             const bool got = group_wait(ud_bar, seg & 1, kBarEpi, kEpiThreads, ctl);
             if (!got) {
+              // not a break: the next segment's kBarFin / kBarFin2 still have to be
+              // taken with the CUDA-core warps, which leave after kBarFin2
               ok = false;
-              break;
+              continue;
             }
             if (fin_flag[seg]) {
               tc_fence_after();
-              uint32_t du[L::kUN];
-              tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + kUTmem, *reinterpret_cast<uint32_t(*)[16]>(du));
-              if constexpr (L::kUN > 16)
-                tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + kUTmem + 16,
-                          *reinterpret_cast<uint32_t(*)[16]>(du + 16));
-              tmem_wait_ld();
-              tc_fence_before();
+              if constexpr (L::kUN <= 32) {
+                uint32_t du[L::kUN];
+                tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + L::kTmU, *reinterpret_cast<uint32_t(*)[16]>(du));
+                if constexpr (L::kUN > 16)
+                  tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + L::kTmU + 16,
+                            *reinterpret_cast<uint32_t(*)[16]>(du + 16));
+                tmem_wait_ld();
     #pragma unroll
-              for (int j = 0; j < MC; ++j) v[j] += __uint_as_float(du[j]) + __uint_as_float(du[MC + j]);
+                for (int j = 0; j < MC; ++j) v[j] += __uint_as_float(du[j]) + __uint_as_float(du[MC + j]);
+              } else {
+                // high parts in columns [0, MC), low parts in [MC, 2 MC): 16 rows at a time
+    #pragma unroll
+                for (int c0 = 0; c0 < MC; c0 += 16) {
+                  uint32_t hi[16], lo[16];
+                  tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + L::kTmU + c0, hi);
+                  tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + L::kTmU + MC + c0, lo);
+                  tmem_wait_ld();
+    #pragma unroll
+                  for (int j = 0; j < 16; ++j) v[c0 + j] += __uint_as_float(hi[j]) + __uint_as_float(lo[j]);
+                }
+              }
+              tc_fence_before();
             }
           } else {
             const float* corr = reinterpret_cast<const float*>(smem + L::kCorr);
@@ -562,7 +826,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
         } else {
           // publish this partial (FP4 product and U z share); the last contributor
           // of the tile completes it
-          float* my_slot = p.slots + static_cast<size_t>(2 * g + which) * kRowsMax * kTileRows;
+          float* my_slot = p.slots + static_cast<size_t>(2 * g + which) * kBN * kTileRows;
   #pragma unroll
           for (int j = 0; j < MC; ++j)
             if (j < p.M) my_slot[j * kTileRows + row] = v[j];
@@ -579,27 +843,33 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
           const bool fin = *epi_last != 0;
           named_barrier(kBarEpi, kEpiThreads);
           if (!fin) continue;
-          // every contributor's partial, summed in contributor order
+          // every contributor's partial, summed in contributor order (the 32-row
+          // class in two halves of 16 rows, two contributors per batch of loads)
   #pragma unroll
           for (int j = 0; j < MC; ++j) acc[j] = 0.0f;
           const int wh_first = (t == first_unit(hf, p.G, p.U) / p.KC) ? 0 : 1;
-          for (int h0 = hf; h0 <= hl; h0 += kHB) {
-            float part[kHB][MC];
+          constexpr int kRC = (MC > 16) ? 16 : MC;
+          constexpr int kHBc = (MC > 16) ? 2 : kHB;
   #pragma unroll
-            for (int e = 0; e < kHB; ++e) {
-              const int h = h0 + e;
-              const float* sl = p.slots + static_cast<size_t>(2 * h + ((h == hf) ? wh_first : 0)) *
-                                              kRowsMax * kTileRows;
+          for (int j0 = 0; j0 < MC; j0 += kRC) {
+            for (int h0 = hf; h0 <= hl; h0 += kHBc) {
+              float part[kHBc][kRC];
   #pragma unroll
-              for (int j = 0; j < MC; ++j)
-                part[e][j] = (h <= hl && h != g && j < p.M) ? __ldcg(sl + j * kTileRows + row) : 0.0f;
-            }
+              for (int e = 0; e < kHBc; ++e) {
+                const int h = h0 + e;
+                const float* sl = p.slots + static_cast<size_t>(2 * h + ((h == hf) ? wh_first : 0)) *
+                                                kBN * kTileRows;
   #pragma unroll
-            for (int e = 0; e < kHB; ++e) {
-              const int h = h0 + e;
-              if (h <= hl) {
+                for (int jj = 0; jj < kRC; ++jj)
+                  part[e][jj] = (h <= hl && h != g && j0 + jj < p.M) ? __ldcg(sl + (j0 + jj) * kTileRows + row) : 0.0f;
+              }
   #pragma unroll
-                for (int j = 0; j < MC; ++j) acc[j] += (h == g) ? v[j] : part[e][j];
+              for (int e = 0; e < kHBc; ++e) {
+                const int h = h0 + e;
+                if (h <= hl) {
+  #pragma unroll
+                  for (int jj = 0; jj < kRC; ++jj) acc[j0 + jj] += (h == g) ? v[j0 + jj] : part[e][jj];
+                }
               }
             }
           }
@@ -623,18 +893,14 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
         if (ok) ok = group_wait(accf_bar(b), (seg >> 1) & 1, kBarEpi, kEpiThreads, ctl);
         if (ok) {
           tc_fence_after();
-          uint32_t raw[16];
-          tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(b * kBN), raw);
-          tmem_wait_ld();
-  #pragma unroll
-          for (int j = 0; j < MC; ++j) v[j] = __fmul_rn(gs, __uint_as_float(raw[j]));
+          load_acc(b, v);
           tc_fence_before();
           mbar_arrive(acce_bar(b));
           if (sole) {
             fin = true;
           } else {
             // publish this partial; the last contributor of the tile completes it
-            float* my_slot = p.slots + static_cast<size_t>(2 * g + which) * kRowsMax * kTileRows;
+            float* my_slot = p.slots + static_cast<size_t>(2 * g + which) * kBN * kTileRows;
   #pragma unroll
             for (int j = 0; j < MC; ++j)
               if (j < p.M) my_slot[j * kTileRows + row] = v[j];
@@ -677,7 +943,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
             for (int e = 0; e < kHB; ++e) {
               const int h = h0 + e;
               const float* sl = p.slots + static_cast<size_t>(2 * h + ((h == hf) ? wh_first : 0)) *
-                                              kRowsMax * kTileRows;
+                                              kBN * kTileRows;
   #pragma unroll
               for (int j = 0; j < MC; ++j)
                 part[e][j] = (h <= hl && h != g && j < p.M) ? __ldcg(sl + j * kTileRows + row) : 0.0f;
@@ -708,6 +974,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
           for (int m = 0; m < MC; ++m) own[m] = 0.0f;
           if (ok) {
             const float* zs = reinterpret_cast<const float*>(smem + L::kZ);
+            const float* lut = reinterpret_cast<const float*>(smem + L::kLut);
             float acc4[MC][4];
   #pragma unroll
             for (int m = 0; m < MC; ++m)
@@ -717,22 +984,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
               uint32_t word = 0;
   #pragma unroll
               for (int e = 0; e < 16; ++e) word = (e == w) ? uw[e] : word;
-              const float* zw = zs + (w2 + w) * 32;
-  #pragma unroll
-              for (int j4 = 0; j4 < 8; ++j4) {
-  #pragma unroll
-                for (int m = 0; m < MC; ++m) {
-                  if (m < p.M) {
-                    const float4 z4 = *reinterpret_cast<const float4*>(zw + m * kMaxRanks + 4 * j4);
-                    const float zz[4] = {z4.x, z4.y, z4.z, z4.w};
-  #pragma unroll
-                    for (int jj = 0; jj < 4; ++jj) {
-                      const uint32_t sgn = (word << (31 - (4 * j4 + jj))) & 0x80000000u;
-                      acc4[m][jj] += __uint_as_float(__float_as_uint(zz[jj]) ^ sgn);
-                    }
-                  }
-                }
-              }
+              u_word_sum<MC, kLut>(zs, lut, word, w2 + w, p.M, acc4);
             }
   #pragma unroll
             for (int m = 0; m < MC; ++m) own[m] = (acc4[m][0] + acc4[m][1]) + (acc4[m][2] + acc4[m][3]);
@@ -756,13 +1008,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
     // ---------------------------------------------------------------- CUDA cores
     const int tid = threadIdx.x - kAluWarp0 * 32;      // 0..255
     const int a = warp - kAluWarp0;                     // warp slot 0..7
-    // The operand cache starts zero: rows >= M and blocks past K stay zero.
-    for (int idx = tid; idx < nunits * 160; idx += kAluThreads) {
-      const int k = idx / 160, o = idx - k * 160;
-      uint4* dst = (o < 128) ? reinterpret_cast<uint4*>(smem + L::kB + k * kBN * 128) + o
-                             : reinterpret_cast<uint4*>(smem + L::kSFB + k * 512) + (o - 128);
-      *dst = make_uint4(0u, 0u, 0u, 0u);
-    }
+    if constexpr (!kStream) zero_cache<MC>(smem, nunits, tid, kAluThreads);
     // this CTA's slice of the ranks for z (empty for CTAs outside the sharing set)
     const int zg = shared_work_ctas(p);
     const int i0 = g < zg ? static_cast<int>(static_cast<uint32_t>(g) * static_cast<uint32_t>(p.r) /
@@ -789,71 +1035,72 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
     // ---- 1. quantise the activation chunks of every unit of this CTA
     {
       if constexpr (!Cfg<MC>::kGlobalQ) {
-        // two blocks per thread per round, the loop rolled (the quantiser is long
-        // straight-line code; unrolled deeper it would crowd the instruction cache)
-        constexpr int kQB = 2;
-        const int per_unit = p.M * 16;
-        const int items = nunits * per_unit;
-#pragma unroll 1
-        for (int base = 0; base < items; base += kAluThreads * kQB) {
-          uint4 lo[kQB], hi[kQB];
-#pragma unroll
-          for (int e = 0; e < kQB; ++e) {
-            const int idx = base + e * kAluThreads + tid;
-            lo[e] = hi[e] = make_uint4(0u, 0u, 0u, 0u);
-            if (idx < items) {
-              const int k = idx / per_unit, rem = idx - k * per_unit, m = rem >> 4, blk = rem & 15;
-              const int kk = ((u0 + k) % p.KC) * kUnitK + blk * 16;
-              if (kk < p.K) {
-                const uint4* src = reinterpret_cast<const uint4*>(p.x + static_cast<size_t>(m) * p.K + kk);
-                lo[e] = __ldcg(src);
-                hi[e] = __ldcg(src + 1);
-              }
-            }
-          }
-#pragma unroll
-          for (int e = 0; e < kQB; ++e) {
-            const int idx = base + e * kAluThreads + tid;
-            if (idx < items) {
-              const int k = idx / per_unit, rem = idx - k * per_unit, m = rem >> 4, blk = rem & 15;
-              const int kk = ((u0 + k) % p.KC) * kUnitK + blk * 16;
-              if (kk < p.K) {
-                float v[16];
-                bf16x16_to_f32(lo[e], hi[e], v);
-                uint2 codes;
-                const uint32_t s = quant_act_block_fast(v, codes);
-                const int j = blk * 8;
-                *reinterpret_cast<uint2*>(smem + L::kB + k * kBN * 128 + m * 128 +
-                                          ((((j >> 4) ^ (m & 7)) << 4) | (j & 15))) = codes;
-                smem[L::kSFB + k * 512 + (blk >> 2) * 128 + m * 4 + (blk & 3)] = static_cast<uint8_t>(s);
-              }
-            }
-          }
-        }
+        quant_into_cache<MC>(p, smem, u0, nunits, tid, kAluThreads);
       } else {
-        // CTA g < Z (Z = shared_work_ctas) quantises items [g I / Z, (g + 1) I / Z) of the I = 16 KC blocks of
-        // 16 rows x 16 elements (rows >= M and blocks past K as zero codes and scales)
-        // into the global image, publishes them, and after every CTA has done so
-        // copies the chunks of its units into the operand cache
-        const uint32_t items = static_cast<uint32_t>(p.KC) * 256u;
-        const uint32_t q0 = g < zg ? static_cast<uint32_t>(static_cast<uint64_t>(g) * items / static_cast<uint32_t>(zg)) : 0u;
-        const uint32_t q1 = g < zg ? static_cast<uint32_t>(static_cast<uint64_t>(g + 1) * items / static_cast<uint32_t>(zg)) : 0u;
-        for (uint32_t it = q0 + static_cast<uint32_t>(tid); it < q1; it += kAluThreads) {
-          const int kc = static_cast<int>(it >> 8), m = static_cast<int>((it >> 4) & 15u), blk = static_cast<int>(it & 15u);
-          const int kk = kc * kUnitK + blk * 16;
-          uint2 codes = make_uint2(0u, 0u);
-          uint32_t sc = 0u;
-          if (m < p.M && kk < p.K) {
-            const uint4* src = reinterpret_cast<const uint4*>(p.x + static_cast<size_t>(m) * p.K + kk);
-            const uint4 lo = __ldcg(src), hi = __ldcg(src + 1);
-            float v[16];
-            bf16x16_to_f32(lo, hi, v);
-            sc = quant_act_block_fast(v, codes);
+        constexpr int kImgBytes = QImg<MC>::kBytes, kImgCodes = QImg<MC>::kCodes;
+        if constexpr (!kStream) {
+          // CTA g < Z (Z = shared_work_ctas) quantises items [g I / Z, (g + 1) I / Z) of the I = 16 KC blocks of
+          // 16 rows x 16 elements (rows >= M and blocks past K as zero codes and scales)
+          // into the global image, publishes them, and after every CTA has done so
+          // copies the chunks of its units into the operand cache
+          const uint32_t items = static_cast<uint32_t>(p.KC) * 256u;
+          const uint32_t q0 = g < zg ? static_cast<uint32_t>(static_cast<uint64_t>(g) * items / static_cast<uint32_t>(zg)) : 0u;
+          const uint32_t q1 = g < zg ? static_cast<uint32_t>(static_cast<uint64_t>(g + 1) * items / static_cast<uint32_t>(zg)) : 0u;
+          for (uint32_t it = q0 + static_cast<uint32_t>(tid); it < q1; it += kAluThreads) {
+            const int kc = static_cast<int>(it >> 8), m = static_cast<int>((it >> 4) & 15u), blk = static_cast<int>(it & 15u);
+            const int kk = kc * kUnitK + blk * 16;
+            uint2 codes = make_uint2(0u, 0u);
+            uint32_t sc = 0u;
+            if (m < p.M && kk < p.K) {
+              const uint4* src = reinterpret_cast<const uint4*>(p.x + static_cast<size_t>(m) * p.K + kk);
+              const uint4 lo = __ldcg(src), hi = __ldcg(src + 1);
+              float v[16];
+              bf16x16_to_f32(lo, hi, v);
+              sc = quant_act_block_fast(v, codes);
+            }
+            uint8_t* img = p.xq + static_cast<size_t>(kc) * kImgBytes;
+            const int j = blk * 8;
+            *reinterpret_cast<uint2*>(img + m * 128 + ((((j >> 4) ^ (m & 7)) << 4) | (j & 15))) = codes;
+            img[kImgCodes + (blk >> 2) * 64 + m * 4 + (blk & 3)] = static_cast<uint8_t>(sc);
           }
-          uint8_t* img = p.xq + static_cast<size_t>(kc) * kQImgBytes;
-          const int j = blk * 8;
-          *reinterpret_cast<uint2*>(img + m * 128 + ((((j >> 4) ^ (m & 7)) << 4) | (j & 15))) = codes;
-          img[kQImgCodes + (blk >> 2) * 64 + m * 4 + (blk & 3)] = static_cast<uint8_t>(sc);
+        } else {
+          // Streamed class: items of (chunk, row, 64-element K step), I = 128 KC of
+          // them, CTA g < Z taking [g I / Z, (g + 1) I / Z).  An item is four blocks:
+          // 32 code bytes (two 16-byte pieces of the swizzled row) and the row's line
+          // of the step's scale atom (four scales, twelve zero bytes).  Rows >= M and
+          // steps past K are written as zeros.
+          const uint32_t items = static_cast<uint32_t>(p.KC) * 128u;
+          const uint32_t q0 = g < zg ? static_cast<uint32_t>(static_cast<uint64_t>(g) * items / static_cast<uint32_t>(zg)) : 0u;
+          const uint32_t q1 = g < zg ? static_cast<uint32_t>(static_cast<uint64_t>(g + 1) * items / static_cast<uint32_t>(zg)) : 0u;
+#pragma unroll 1
+          for (uint32_t it = q0 + static_cast<uint32_t>(tid); it < q1; it += kAluThreads) {
+            const int kc = static_cast<int>(it >> 7), m = static_cast<int>((it >> 2) & 31u), st = static_cast<int>(it & 3u);
+            const int kk = kc * kUnitK + st * 64;
+            const bool live = m < p.M && kk < p.K;
+            uint4 xv[8];
+            const uint4* src = reinterpret_cast<const uint4*>(p.x + static_cast<size_t>(live ? m : 0) * p.K + (live ? kk : 0));
+#pragma unroll
+            for (int e = 0; e < 8; ++e) xv[e] = live ? __ldcg(src + e) : make_uint4(0u, 0u, 0u, 0u);
+            uint32_t cw[8];
+            uint32_t sc4 = 0u;
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+              float v[16];
+              bf16x16_to_f32(xv[2 * b], xv[2 * b + 1], v);
+              uint2 codes;
+              const uint32_t sc = quant_act_block_fast(v, codes);
+              cw[2 * b] = codes.x;
+              cw[2 * b + 1] = codes.y;
+              sc4 |= sc << (8 * b);
+            }
+            uint8_t* img = p.xq + static_cast<size_t>(kc) * kImgBytes;
+            // elements 64 st .. 64 st + 63 = bytes 32 st .. 32 st + 31 of the row: pieces 2 st, 2 st + 1
+            *reinterpret_cast<uint4*>(img + m * 128 + (((2 * st) ^ (m & 7)) << 4)) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+            *reinterpret_cast<uint4*>(img + m * 128 + (((2 * st + 1) ^ (m & 7)) << 4)) = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+            *reinterpret_cast<uint4*>(img + kImgCodes + st * 512 + m * 16) = make_uint4(sc4, 0u, 0u, 0u);
+          }
+          // the producers read the image with bulk copies (the async proxy)
+          fence_proxy_async_global();
         }
         if constexpr (Cfg<MC>::kTensorV) {
           if (p.r > 0) {
@@ -891,7 +1138,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
 #pragma unroll
                 for (int e = 0; e < kXL; ++e) {
                   const int idx = e * kAluThreads + tid;
-                  const int j = idx >> 7, m = (idx >> 3) & 15, c = idx & 7;
+                  const int j = idx / (kBN * 8), m = (idx >> 3) & (kBN - 1), c = idx & 7;
                   xv[e] = (j < nb && m < p.M)
                               ? __ldcg(reinterpret_cast<const uint4*>(p.x + static_cast<size_t>(m) * p.K + 64 * (b0 + j) + 8 * c))
                               : make_uint4(0u, 0u, 0u, 0u);
@@ -917,7 +1164,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
 #pragma unroll
                 for (int e = 0; e < kXL; ++e) {
                   const int idx = e * kAluThreads + tid;
-                  const int j = idx >> 7, m = (idx >> 3) & 15, c = idx & 7;
+                  const int j = idx / (kBN * 8), m = (idx >> 3) & (kBN - 1), c = idx & 7;
                   if (j < nb) *reinterpret_cast<uint4*>(vbt + j * (kBN * 128) + m * 128 + ((c ^ (m & 7)) << 4)) = xv[e];
                 }
                 fence_proxy_async_smem();
@@ -930,7 +1177,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
                   for (int j = 0; j < nb; ++j)
 #pragma unroll
                     for (int k4 = 0; k4 < 4; ++k4)
-                      tc_mma_bf16(tmem + kVTmem, a_d + static_cast<uint64_t>(j) * ((kTileRows * 128) >> 4) + 2 * k4,
+                      tc_mma_bf16(tmem + L::kTmV, a_d + static_cast<uint64_t>(j) * ((kTileRows * 128) >> 4) + 2 * k4,
                                   b_d + static_cast<uint64_t>(j) * ((kBN * 128) >> 4) + 2 * k4, idesc_v,
                                   (b0 > a0 || j > 0 || k4 > 0) ? 1u : 0u);
                   tc_commit(vmma_bar);
@@ -944,13 +1191,16 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
               tc_fence_after();
               if (a < 4) {
                 const int quarter = warp & 3;
-                uint32_t v[16];
-                tmem_ld16(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + kVTmem, v);
-                tmem_wait_ld();
                 float* dst = p.vpart + static_cast<size_t>(rb * S + sl) * kBN * kTileRows + quarter * 32 + lane;
 #pragma unroll
-                for (int m = 0; m < kBN; ++m)
-                  if (m < p.M) dst[m * kTileRows] = __uint_as_float(v[m]);
+                for (int c0 = 0; c0 < kBN; c0 += 16) {
+                  uint32_t v[16];
+                  tmem_ld16(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + L::kTmV + c0, v);
+                  tmem_wait_ld();
+#pragma unroll
+                  for (int m = 0; m < 16; ++m)
+                    if (c0 + m < p.M) dst[(c0 + m) * kTileRows] = __uint_as_float(v[m]);
+                }
               }
               tc_fence_before();
               named_barrier(kBarAlu, kAluThreads);           // TMEM read before the next piece
@@ -960,7 +1210,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
         named_barrier(kBarAlu, kAluThreads);
         bool okq = true;
         if (tid == 0) {
-          red_add_release_gpu(p.q_ready, 1u);              // covers the items the CTA wrote
+          if (!(p.drop & 2)) red_add_release_gpu(p.q_ready, 1u);   // covers the items the CTA wrote
           okq = spin_until_geq(p.q_ready, static_cast<uint32_t>(p.G), ctl);
           if (okq) {
             // the last CTA past the wait resets both counters for the next call
@@ -972,51 +1222,42 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
           }
         }
         if (named_barrier_or(kBarAlu, kAluThreads, !okq)) fail(ctl);
-        // one round of 16-byte loads: 144 per unit (128 of codes, 16 of scales)
-        constexpr int kPer = kQImgBytes / 16;
-        constexpr int kLd = (kMaxUnits * kPer + kAluThreads - 1) / kAluThreads;
-        uint4 buf[kLd];
+        if constexpr (kStream) {
+          // the image is complete: the producer may fetch its chunks (after a
+          // failed wait too, so that its stages complete)
+          if (tid == 0) mbar_arrive(actr_bar);
+        } else {
+          // one round of 16-byte loads: 144 per unit (128 of codes, 16 of scales)
+          constexpr int kPer = kImgBytes / 16;
+          constexpr int kLd = (L::kMaxUnits * kPer + kAluThreads - 1) / kAluThreads;
+          uint4 buf[kLd];
 #pragma unroll
-        for (int e = 0; e < kLd; ++e) {
-          const int idx = e * kAluThreads + tid;
-          if (idx < nunits * kPer) {
-            const int k = idx / kPer, o = idx - k * kPer;
-            const int kc = (u0 + k) % p.KC;
-            buf[e] = __ldcg(reinterpret_cast<const uint4*>(p.xq + static_cast<size_t>(kc) * kQImgBytes) + o);
+          for (int e = 0; e < kLd; ++e) {
+            const int idx = e * kAluThreads + tid;
+            if (idx < nunits * kPer) {
+              const int k = idx / kPer, o = idx - k * kPer;
+              const int kc = (u0 + k) % p.KC;
+              buf[e] = __ldcg(reinterpret_cast<const uint4*>(p.xq + static_cast<size_t>(kc) * kImgBytes) + o);
+            }
           }
-        }
 #pragma unroll
-        for (int e = 0; e < kLd; ++e) {
-          const int idx = e * kAluThreads + tid;
-          if (idx < nunits * kPer) {
-            const int k = idx / kPer, o = idx - k * kPer;
-            uint8_t* dst = (o < 128) ? smem + L::kB + k * kBN * 128 + o * 16
-                                     : smem + L::kSFB + k * 512 + ((o - 128) >> 2) * 128 + ((o - 128) & 3) * 16;
-            *reinterpret_cast<uint4*>(dst) = buf[e];
+          for (int e = 0; e < kLd; ++e) {
+            const int idx = e * kAluThreads + tid;
+            if (idx < nunits * kPer) {
+              const int k = idx / kPer, o = idx - k * kPer;
+              uint8_t* dst = (o < 128) ? smem + L::kB + k * kBN * 128 + o * 16
+                                       : smem + L::kSFB + k * 512 + ((o - 128) >> 2) * 128 + ((o - 128) & 3) * 16;
+              *reinterpret_cast<uint4*>(dst) = buf[e];
+            }
           }
         }
       }
+    }
+    if constexpr (!kStream) {
       fence_proxy_async_smem();
       named_barrier(kBarAlu, kAluThreads);
-      // Activation scales to TMEM, in the layout a 32x128b.warpx4 copy of scale
-      // atoms would give: lane i of every lane quarter holds, in column 16 k + 4 j,
-      // the four block scales of row i for K step j of unit k (rows >= 16 and the
-      // other three columns of a step are zero).  Warps 6..9 cover the four lane
-      // quarters.
-      if (a < 4) {
-        const uint32_t quarter = static_cast<uint32_t>(warp & 3);
-        for (int k = 0; k < nunits; ++k) {
-          const uint32_t* sfb = reinterpret_cast<const uint32_t*>(smem + L::kSFB + k * 512) + lane;
-          uint32_t v[16];
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            v[4 * j] = sfb[j * 32];
-            v[4 * j + 1] = v[4 * j + 2] = v[4 * j + 3] = 0u;
-          }
-          tmem_st16(tmem + ((quarter * 32) << 16) + kSfbTmemBase + k * 16, v);
-        }
-        tmem_wait_st();
-      }
+      // activation scales to TMEM: warps 6..9 cover the four lane quarters
+      if (a < 4) sfb_to_tmem<MC>(smem, tmem, nunits, static_cast<uint32_t>(warp & 3), lane);
       tc_fence_before();
       named_barrier(kBarAlu, kAluThreads);
       if (tid == 0) mbar_arrive(actr_bar);
@@ -1119,7 +1360,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
         }
       }
       named_barrier(kBarAlu, kAluThreads);
-      if (tid == 0) red_add_release_gpu(p.z_ready, 1u);   // covers the slice the CTA wrote
+      if (tid == 0 && !(p.drop & 1)) red_add_release_gpu(p.z_ready, 1u);   // covers the slice the CTA wrote
 
       if constexpr (Cfg<MC>::kTensorU) {
         // ---- 3. This CTA's share of U z for each of its tiles, on the tensor cores:
@@ -1147,50 +1388,77 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
         uint32_t uw0[kUChunksMax], uw1[kUChunksMax];
         load_words(t_first, uw0);
         if (nseg > 1) load_words(t_first + 1, uw1);
-        bool ok = true, ztiles = false;
+        bool ok = true, zwaited = false;
+        int zgroup = -1;                                 // z chunks [zgroup S, zgroup S + S) are in the slots
         int uses0 = 0, uses1 = 0;                        // MMA rounds issued on each A buffer
-        for (int seg = 0; seg < nseg; ++seg) {
-          if (named_barrier_or(kBarFin, kFinThreads, !ok)) {
-            ok = false;
-            break;
+        // wait (lane 0 of each warp) until the MMAs that last read A buffer `buf` are done
+        auto buffer_free = [&](int buf, int uses) {
+          if (uses > 0) {
+            bool okb = true;
+            if (lane == 0) okb = mbar_wait(ubuf_bar(buf), (uses - 1) & 1, abort_flag);
+            if (__shfl_sync(0xffffffffu, okb ? 1 : 0, 0) == 0) {
+              fail(ctl);
+              ok = false;
+            }
           }
-          const int t = t_first + seg;
-          const int ua = max(u0, t * p.KC), ub = min(u1, (t + 1) * p.KC);
-          const int cs0 = (ua - t * p.KC) * nuc / p.KC, cs1 = (ub - t * p.KC) * nuc / p.KC;
-          if (cs1 > cs0 && !ztiles) {
-            // first non-empty share: wait for every slice of z, then the B tiles
+        };
+        // The B tiles of z chunks [grp S, grp S + S) (S = kZSlots) into the slots.  They
+        // were written in their final layout by the CTAs that computed z (rows past 2 M
+        // only feed output columns nobody reads).  The first time, wait for every slice
+        // of z; later (ranks beyond S chunks), for the MMAs still reading the slots.
+        auto stage_z = [&](int grp) {
+          constexpr int S = Cfg<MC>::kZSlots;
+          if (!zwaited) {
             bool okw = true;
             if (tid == 0) okw = spin_until_geq(p.z_ready, static_cast<uint32_t>(p.G), ctl);
             if (named_barrier_or(kBarAlu, kAluThreads, !okw)) {
               fail(ctl);
               ok = false;
             }
-            // the B tiles were written in their final layout by the CTAs that computed
-            // z: copy them (rows past 2 M only feed output columns nobody reads)
-            {
-              uint4* zt4 = reinterpret_cast<uint4*>(smem + L::kUZ);
-              const uint4* src = reinterpret_cast<const uint4*>(p.ztiles);
-              constexpr int kZR = 8;
-              const int n16 = nuc * L::kUN * 8;
-              for (int base = 0; base < n16; base += kAluThreads * kZR) {
-                uint4 t4[kZR];
-#pragma unroll
-                for (int e = 0; e < kZR; ++e) {
-                  const int idx = base + e * kAluThreads + tid;
-                  t4[e] = (idx < n16) ? __ldcg(src + idx) : make_uint4(0u, 0u, 0u, 0u);
-                }
-#pragma unroll
-                for (int e = 0; e < kZR; ++e) {
-                  const int idx = base + e * kAluThreads + tid;
-                  if (idx < n16) zt4[idx] = t4[e];
-                }
-              }
-            }
-            fence_proxy_async_smem();
+            zwaited = true;
+          } else if constexpr (S < kUChunksMax) {
+            // a reload (only the 32-row class has fewer slots than chunks)
+            buffer_free(0, uses0);
+            buffer_free(1, uses1);
             named_barrier(kBarAlu, kAluThreads);
-            ztiles = true;
           }
-          if (seg >= 2) load_words(t_first + seg, uw1);    // segments past the second: load now
+          uint4* zt4 = reinterpret_cast<uint4*>(smem + L::kUZ);
+          const uint4* src = reinterpret_cast<const uint4*>(p.ztiles + static_cast<size_t>(grp) * S * L::kUN * 128);
+          constexpr int kZR = 8;
+          const int n16 = min(S, nuc - grp * S) * L::kUN * 8;
+          for (int base = 0; base < n16; base += kAluThreads * kZR) {
+            uint4 t4[kZR];
+#pragma unroll
+            for (int e = 0; e < kZR; ++e) {
+              const int idx = base + e * kAluThreads + tid;
+              t4[e] = (idx < n16) ? __ldcg(src + idx) : make_uint4(0u, 0u, 0u, 0u);
+            }
+#pragma unroll
+            for (int e = 0; e < kZR; ++e) {
+              const int idx = base + e * kAluThreads + tid;
+              if (idx < n16) zt4[idx] = t4[e];
+            }
+          }
+          fence_proxy_async_smem();
+          named_barrier(kBarAlu, kAluThreads);
+          zgroup = grp;
+        };
+        for (int seg = 0; seg < nseg; ++seg) {
+          // Every segment takes both barriers shared with the epilogue (kBarFin,
+          // kBarFin2), on every path: when either side has given up, the share is
+          // skipped (an empty one), and both sides leave together after kBarFin2.
+          const bool gone = named_barrier_or(kBarFin, kFinThreads, !ok);
+          if (gone) ok = false;
+          const int t = t_first + seg;
+          const int ua = max(u0, t * p.KC), ub = min(u1, (t + 1) * p.KC);
+          const int cs0 = gone ? 0 : (ua - t * p.KC) * nuc / p.KC;
+          const int cs1 = gone ? 0 : (ub - t * p.KC) * nuc / p.KC;
+          if (seg >= 2 && !gone) load_words(t_first + seg, uw1);    // segments past the second: load now
+          // the classes whose slots hold every chunk stage z once, before their first
+          // chunk; the 32-row class cycles larger ranks through its slots below
+          if constexpr (Cfg<MC>::kZSlots >= kUChunksMax) {
+            if (cs1 > cs0 && zgroup < 0) stage_z(0);
+          }
           // chunk pairs in a rolled loop (fully unrolled, the body would make the
           // kernel's code outgrow the instruction cache; the chunk's word is picked
           // out of the registers by compare-and-select, so the word arrays stay in
@@ -1205,16 +1473,11 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
           for (int buf = 0; buf < 2; ++buf) {
             const int c = c2 + buf;
             if (c < cs1) {
-              int& uses = buf ? uses1 : uses0;
-              if (uses > 0) {
-                // the MMAs that read this buffer last are done
-                bool okb = true;
-                if (lane == 0) okb = mbar_wait(ubuf_bar(buf), (uses - 1) & 1, abort_flag);
-                if (__shfl_sync(0xffffffffu, okb ? 1 : 0, 0) == 0) {
-                  fail(ctl);
-                  ok = false;
-                }
+              if constexpr (Cfg<MC>::kZSlots < kUChunksMax) {
+                if (c / Cfg<MC>::kZSlots != zgroup) stage_z(c / Cfg<MC>::kZSlots);
               }
+              int& uses = buf ? uses1 : uses0;
+              buffer_free(buf, uses);                      // the MMAs that read this buffer last are done
               uint32_t word = 0u;
   #pragma unroll
               for (int e = 0; e < kUChunksMax; ++e) word = (e == c) ? ((seg == 0) ? uw0[e] : uw1[e]) : word;
@@ -1236,10 +1499,11 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
                 if (mbar_wait(ufull_bar(buf), uses & 1, abort_flag)) {
                   tc_fence_after();
                   const uint64_t a_d = smem_desc(smem_u32(smem + L::kUA + buf * (kTileRows * 128)), 16, 1024, 2);
-                  const uint64_t b_d = smem_desc(smem_u32(smem + L::kUZ + c * L::kUN * 128), 16, 1024, 2);
+                  const uint64_t b_d =
+                      smem_desc(smem_u32(smem + L::kUZ + (c % Cfg<MC>::kZSlots) * L::kUN * 128), 16, 1024, 2);
   #pragma unroll
                   for (int j = 0; j < 4; ++j)
-                    tc_mma_bf16(tmem + kUTmem, a_d + 2 * j, b_d + 2 * j, idesc_u, (c > cs0 || j > 0) ? 1u : 0u);
+                    tc_mma_bf16(tmem + L::kTmU, a_d + 2 * j, b_d + 2 * j, idesc_u, (c > cs0 || j > 0) ? 1u : 0u);
                   tc_commit(ubuf_bar(buf));
                 } else {
                   fail(ctl);
@@ -1251,7 +1515,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
           }
           }
           if (tid == 0) {
-            fin_flag[seg] = (cs1 > cs0) ? 1 : 0;           // a share to add, in kUTmem
+            fin_flag[seg] = (cs1 > cs0) ? 1 : 0;           // a share to add, in TMEM at kTmU
             tc_commit(ud_bar);                             // arrives at once if nothing was issued
           }
           if (named_barrier_or(kBarFin2, kFinThreads, !ok)) {
@@ -1317,6 +1581,10 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
                 zs[m * kMaxRanks + i] = (i < p.r) ? __ldcg(p.z + static_cast<size_t>(m) * p.rpad + i) : 0.0f;
               }
               named_barrier(kBarAlu, kAluThreads);
+              if constexpr (kLut) {
+                build_z_table<MC>(zs, reinterpret_cast<float*>(smem + L::kLut), p.M, p.RW, tid, kAluThreads);
+                named_barrier(kBarAlu, kAluThreads);
+              }
               staged = true;
             }
           }
@@ -1329,26 +1597,12 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
             for (int m = 0; m < MC; ++m)
   #pragma unroll
               for (int jj = 0; jj < 4; ++jj) acc4[m][jj] = 0.0f;
+            const float* lut = reinterpret_cast<const float*>(smem + L::kLut);
             for (int w = 0; w < wb - wa; ++w) {
               uint32_t word = 0;
   #pragma unroll
               for (int e = 0; e < 16; ++e) word = (e == w) ? ((seg == 0) ? uw0[e] : uw1[e]) : word;
-              const float* zw = zs + (wa + w) * 32;
-  #pragma unroll
-              for (int j4 = 0; j4 < 8; ++j4) {
-  #pragma unroll
-                for (int m = 0; m < MC; ++m) {
-                  if (m < p.M) {
-                    const float4 z4 = *reinterpret_cast<const float4*>(zw + m * kMaxRanks + 4 * j4);
-                    const float zz[4] = {z4.x, z4.y, z4.z, z4.w};
-  #pragma unroll
-                    for (int jj = 0; jj < 4; ++jj) {
-                      const uint32_t sgn = (word << (31 - (4 * j4 + jj))) & 0x80000000u;
-                      acc4[m][jj] += __uint_as_float(__float_as_uint(zz[jj]) ^ sgn);
-                    }
-                  }
-                }
-              }
+              u_word_sum<MC, kLut>(zs, lut, word, wa + w, p.M, acc4);
             }
             float acc[MC];
   #pragma unroll
@@ -1394,4 +1648,32 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
 }
 
 }  // namespace decode
+}  // namespace biloco
+
+namespace biloco {
+
+static_assert(decode::kRowsMax == kDecodeMaxRows, "host and kernel limits agree");
+
+template <int MC>
+cudaError_t launch_decode(const CUtensorMap& tw, const DecodeParams& dp, cudaStream_t s,
+                          const LaunchOpts& o) {
+  // the table form exists for the classes with the CUDA-core U side (1-2 rows)
+  constexpr bool kHasLut = !decode::Cfg<MC>::kTensorU;
+  if constexpr (kHasLut) {
+    if (dp.lut) {
+      static KernelSetup ks_lut;
+      return launch_resident(ks_lut, decode::decode_kernel<MC, true>, dp.G, decode::kThreads,
+                             decode::Layout<MC>::kAlloc, s, o, tw, dp);
+    }
+  }
+  static_assert(decode_class(MC) == MC && decode::Cfg<MC>::kBN == decode_bn(MC) &&
+                    decode::Cfg<MC>::kMaxUnits == decode_max_units(MC) &&
+                    decode::QImg<MC>::kBytes == decode_img_bytes(MC) &&
+                    decode::Layout<MC>::kUN * 128 * decode::kUChunksMax <= decode_ztile_bytes(MC),
+                "host and kernel views of the batch class agree");
+  static KernelSetup ks;
+  return launch_resident(ks, decode::decode_kernel<MC, false>, dp.G, decode::kThreads, decode::Layout<MC>::kAlloc, s,
+                         o, tw, dp);
+}
+
 }  // namespace biloco

@@ -27,6 +27,8 @@ struct DecodeParams {
   int* status;             // first device-side error
   int M, N, K, r;
   int KC, T, U, G, KW, RW, rpad;
+  int drop;                // failure-path self test: 1 skips the z arrivals, 2 the image arrivals
+  int lut;                 // 1-2 rows: U z from the signed-sum table of z instead of sign-adds
 };
 
 }  // namespace biloco

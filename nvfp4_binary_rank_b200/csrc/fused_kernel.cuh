@@ -56,6 +56,7 @@
 #include <cuda_runtime.h>
 
 #include "../../include/biloco.h"
+#include "fused_launch.h"
 #include "fused_params.h"
 #include "nvfp4_dev.cuh"
 #include "ptx.cuh"
@@ -1381,4 +1382,16 @@ fused_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
 }
 
 }  // namespace
+}  // namespace biloco
+
+namespace biloco {
+
+template <int BN, int ST, int MC>
+cudaError_t launch_fused(const CUtensorMap& tw, const CUtensorMap& tx, const CUtensorMap& txs,
+                         const CUtensorMap& tv, const FusedParams& fp, cudaStream_t s, const LaunchOpts& o) {
+  static KernelSetup ks;
+  return launch_resident(ks, fused_kernel<BN, ST, MC>, fp.G, kThreads, Layout<BN, ST>::kAlloc, s, o, tw, tx,
+                         txs, tv, fp);
+}
+
 }  // namespace biloco

@@ -30,6 +30,7 @@ struct FusedParams {
   int fast;            // 1: the producer stages each unit's x chunk and V rows by TMA
   int unit_alu;        // 1: the CUDA-core warps have per-unit work (quantise and/or V side)
   int bxr;             // rows of the staged x box (16 or 32)
+  int drop;            // failure-path self test (not used by this kernel)
 };
 
 }  // namespace biloco

@@ -81,15 +81,26 @@ int pick_bn(int M) {
 }
 
 cudaError_t launch_for(int M, const CUtensorMap& tw, const CUtensorMap& tx, const CUtensorMap& txs,
-                       const CUtensorMap& tv, const FusedParams& fp, cudaStream_t s, bool pdl) {
-  if (M <= 1) return launch_fused_16_1(tw, tx, txs, tv, fp, s, pdl);
-  if (M <= 2) return launch_fused_16_2(tw, tx, txs, tv, fp, s, pdl);
-  if (M <= 4) return launch_fused_16_4(tw, tx, txs, tv, fp, s, pdl);
-  if (M <= 8) return launch_fused_16_8(tw, tx, txs, tv, fp, s, pdl);
-  if (M <= 16) return launch_fused_16_16(tw, tx, txs, tv, fp, s, pdl);
-  if (M <= 32) return launch_fused_32_32(tw, tx, txs, tv, fp, s, pdl);
-  if (M <= 64) return launch_fused_64_32(tw, tx, txs, tv, fp, s, pdl);
-  return launch_fused_128_32(tw, tx, txs, tv, fp, s, pdl);
+                       const CUtensorMap& tv, const FusedParams& fp, cudaStream_t s, const LaunchOpts& o) {
+  if (M <= 1) return launch_fused<16, 5, 1>(tw, tx, txs, tv, fp, s, o);
+  if (M <= 2) return launch_fused<16, 5, 2>(tw, tx, txs, tv, fp, s, o);
+  if (M <= 4) return launch_fused<16, 5, 4>(tw, tx, txs, tv, fp, s, o);
+  if (M <= 8) return launch_fused<16, 5, 8>(tw, tx, txs, tv, fp, s, o);
+  if (M <= 16) return launch_fused<16, 5, 16>(tw, tx, txs, tv, fp, s, o);
+  if (M <= 32) return launch_fused<32, 3, 32>(tw, tx, txs, tv, fp, s, o);
+  if (M <= 64) return launch_fused<64, 4, 32>(tw, tx, txs, tv, fp, s, o);
+  return launch_fused<128, 3, 32>(tw, tx, txs, tv, fp, s, o);
+}
+
+// A launch error as a library status: a grid that cannot be resident at once is
+// reported as such, anything else as a CUDA failure.
+int launch_status(cudaError_t e) {
+  if (e == cudaSuccess) return BILOCO_OK;
+  if (e == cudaErrorCooperativeLaunchTooLarge) {
+    cudaGetLastError();
+    return BILOCO_ERR_RESIDENCY;
+  }
+  return BILOCO_ERR_CUDA;
 }
 
 }  // namespace
@@ -103,6 +114,16 @@ int resolve_mode(int M, int N, int K, int r, int requested) {
   (void)M; (void)N; (void)K; (void)r;
   if (requested == BILOCO_MODE_SHARED_Z || requested == BILOCO_MODE_LOCAL_Z) return requested;
   return BILOCO_MODE_SHARED_Z;
+}
+
+// AUTO: the signed-sum table of z for 1-2 rows (the decode kernel's CUDA-core U
+// side; every other shape ignores the setting).  Timed on a B200 at N = K = 5120,
+// M = 1 (CUDA-graph replay, weight copies past L2) it was faster at r = 512 (12.62
+// vs 13.14 us per call) and r = 1024 (19.69 vs 21.06), and equal at r = 128.
+int resolve_arith(int M, int N, int K, int r, int requested) {
+  (void)N; (void)K; (void)r;
+  if (requested == BILOCO_CORR_SIGNS || requested == BILOCO_CORR_LUT) return requested;
+  return M <= 2 ? BILOCO_CORR_LUT : BILOCO_CORR_SIGNS;
 }
 
 int gemm_kernel_count_for(const GemmArgs& a) {
@@ -128,20 +149,21 @@ GemmPlan plan_gemm(const GemmArgs& a) {
   const int ranks_per_tile = (r + p.T - 1) / p.T;
   p.fast = p.unit_alu && p.BN <= 32 && K % 128 == 0 && (!p.shared_z || ranks_per_tile <= kVStageRanks);
 
-  // decode batches take the decode kernel when its operand cache holds every
-  // unit of a CTA (ceil(U / G) units)
-  p.decode = M <= kDecodeMaxRows && (r == 0 || p.shared_z) && (p.U + p.G - 1) / p.G <= kDecodeMaxUnits;
+  // decode batches (up to 32 rows) take the decode kernel when a CTA's units fit
+  // its class (ceil(U / G) units: the operand cache up to 16 rows)
+  p.decode = M <= kDecodeMaxRows && (r == 0 || p.shared_z) && (p.U + p.G - 1) / p.G <= decode_max_units(M);
 
   ScratchNeed& need = p.need;
   if (p.decode) {
-    need.act_fp4 = static_cast<size_t>(p.KC) * kDecodeQImgBytes;   // the activation image (8+ rows)
+    const size_t bn = static_cast<size_t>(decode_bn(M));
+    need.act_fp4 = static_cast<size_t>(p.KC) * decode_img_bytes(M);   // the activation image (8+ rows)
     need.act_sf = 16;
-    // the decode kernel's z tiles, then the V-side partial sums: one 16 x 128 block
+    // the decode kernel's z tiles, then the V-side partial sums: one bn x 128 block
     // per piece, max(G, rank blocks) pieces at most
     const size_t vpieces = static_cast<size_t>(std::max(p.G, (r + kTileRows - 1) / kTileRows));
-    need.zpart = 16 * 32 * 128 + vpieces * kDecodeMaxRows * kTileRows * 4;
+    need.zpart = static_cast<size_t>(decode_ztile_bytes(M)) + vpieces * bn * kTileRows * 4;
     need.zfin = r ? static_cast<size_t>(M) * p.rpad * 4 : 16;
-    need.slots = static_cast<size_t>(2 * p.G) * kDecodeMaxRows * kTileRows * 4;
+    need.slots = static_cast<size_t>(2 * p.G) * bn * kTileRows * 4;
     need.counter_words = 4 + 2 * static_cast<size_t>(p.T);   // z, tickets, q counters
     return p;
   }
@@ -183,7 +205,7 @@ int launch_gemm(const GemmArgs& a, const GemmPlan& p, const Scratch& scr, cudaSt
     dp.y = a.y;
     dp.z = sc->zfin;
     dp.ztiles = reinterpret_cast<uint8_t*>(sc->zpart);
-    dp.vpart = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(sc->zpart) + 16 * 32 * 128);
+    dp.vpart = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(sc->zpart) + decode_ztile_bytes(M));
     dp.slots = sc->slots;
     dp.z_ready = sc->counters;
     dp.z_seen = sc->counters + 1;
@@ -196,12 +218,16 @@ int launch_gemm(const GemmArgs& a, const GemmPlan& p, const Scratch& scr, cudaSt
     dp.KC = KC; dp.T = T; dp.U = U; dp.G = G; dp.KW = KW;
     dp.RW = (r + 31) / 32;
     dp.rpad = rpad;
-    if (M <= 1) e = launch_decode_1(tw, dp, s);
-    else if (M <= 2) e = launch_decode_2(tw, dp, s);
-    else if (M <= 4) e = launch_decode_4(tw, dp, s);
-    else if (M <= 8) e = launch_decode_8(tw, dp, s);
-    else e = launch_decode_16(tw, dp, s);
-    return e == cudaSuccess ? BILOCO_OK : BILOCO_ERR_CUDA;
+    dp.drop = a.drop;
+    dp.lut = (a.arith == BILOCO_CORR_LUT) ? 1 : 0;
+    const LaunchOpts o = current_launch_opts();
+    if (M <= 1) e = launch_decode<1>(tw, dp, s, o);
+    else if (M <= 2) e = launch_decode<2>(tw, dp, s, o);
+    else if (M <= 4) e = launch_decode<4>(tw, dp, s, o);
+    else if (M <= 8) e = launch_decode<8>(tw, dp, s, o);
+    else if (M <= 16) e = launch_decode<16>(tw, dp, s, o);
+    else e = launch_decode<32>(tw, dp, s, o);
+    return launch_status(e);
   }
   if (!inq) {
     e = launch_prep_act(a.x, M, K, sc->act_fp4, sc->act_sf, s);
@@ -257,10 +283,11 @@ int launch_gemm(const GemmArgs& a, const GemmPlan& p, const Scratch& scr, cudaSt
   fp.unit_alu = unit_alu ? 1 : 0;
   fp.bxr = bxr;
 
-  // always launched for programmatic overlap with the kernel before it (the
-  // activation quantiser, or the previous call)
-  e = launch_for(M, tw, tx, txs, tv, fp, s, true);
-  return e == cudaSuccess ? BILOCO_OK : BILOCO_ERR_CUDA;
+  // launched for programmatic overlap with the kernel before it (the activation
+  // quantiser, or the previous call)
+  fp.drop = a.drop;
+  e = launch_for(M, tw, tx, txs, tv, fp, s, current_launch_opts());
+  return launch_status(e);
 }
 
 }  // namespace biloco

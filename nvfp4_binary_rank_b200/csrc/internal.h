@@ -5,6 +5,8 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
+#include "launch_common.h"
+
 namespace biloco {
 
 // Library-owned scratch of one (device, stream) pair.  All regions live in one
@@ -55,6 +57,8 @@ struct GemmArgs {
   uint16_t* y;
   int M, N, K, r;
   int mode;   // resolved: 1 shared z, 2 local z
+  int drop;   // failure-path self test: grid arrivals the decode kernel skips
+  int arith;  // resolved correction arithmetic: BILOCO_CORR_SIGNS or BILOCO_CORR_LUT
 };
 
 // Host checks of biloco_gemm's arguments (include/biloco.h); fills `a` with the
@@ -80,10 +84,14 @@ int launch_gemm(const GemmArgs& a, const GemmPlan& p, const Scratch& sc, cudaStr
 // Validated arguments; per-stream scratch, then launch_gemm.  Returns a BILOCO_* status.
 int run_gemm(const GemmArgs& a, cudaStream_t s);
 int resolve_mode(int M, int N, int K, int r, int requested);
+int resolve_arith(int M, int N, int K, int r, int requested);
 
 // Status word of biloco_gemm_noalloc's static scratch on the current device:
 // returned and, if non-zero, cleared together with its counters (synchronous).
 int noalloc_take_status();
 int gemm_kernel_count_for(const GemmArgs& a);
+
+// Launch form of the GEMM kernels (biloco_set_launch).
+LaunchOpts current_launch_opts();
 
 }  // namespace biloco

@@ -36,7 +36,6 @@ constexpr size_t kStatusOff = 0;
 constexpr size_t kCounterOff = 256;
 constexpr size_t kCounterWordsMax = 4 + 2 * static_cast<size_t>(BILOCO_NOALLOC_MAX_N / 128);
 constexpr size_t kDataOff = (kCounterOff + kCounterWordsMax * 4 + 255) / 256 * 256;
-constexpr size_t kSfChunkBytes = 2048;        // scale atoms of one 256-element chunk of K
 
 __device__ __align__(256) uint8_t g_noalloc_scratch[kCap];
 
@@ -74,6 +73,10 @@ int noalloc_take_status() {
   for (DeviceScratch& x : g_devices)
     if (x.device == dev && x.zeroed) d = &x;
   if (!d) return BILOCO_OK;
+  // The array is shared by every stream of the device, and a call on any of them
+  // (non-blocking ones included) may still be running: wait for all of them
+  // before reading the status, so that no error is missed or cleared early.
+  if (cudaDeviceSynchronize() != cudaSuccess) return BILOCO_ERR_CUDA;
   int status = 0;
   if (cudaMemcpy(&status, d->base + kStatusOff, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
     return BILOCO_ERR_CUDA;
@@ -128,15 +131,6 @@ extern "C" int biloco_gemm_noalloc(const void* x_bf16, const uint8_t* W_fp4, con
       d->zeroed = true;
     }
     base = d->base;
-  }
-
-  if (!p.inq && K % 256 != 0) {
-    // The activation quantiser writes no scale for the blocks past K in the last
-    // chunk, and the tensor cores still read them (against zero codes).  These
-    // bytes may hold whatever an earlier shape left in this part of the array,
-    // so they are cleared: an E4M3 NaN there would turn 0 * scale into NaN.
-    const size_t last = o_sf + (p.need.act_sf - kSfChunkBytes);
-    if (cudaMemsetAsync(base + last, 0, kSfChunkBytes, s) != cudaSuccess) return BILOCO_ERR_CUDA;
   }
 
   Scratch sc;

@@ -40,14 +40,22 @@ quant_act_rowmajor_kernel(const uint16_t* __restrict__ x, int M, int K, uint8_t*
 
 // Same quantiser, scales written into the GEMM's scale atoms.  Triggers the
 // dependent fused kernel at entry so that its prologue and weight stream overlap.
+// The scales of the blocks past K in the last 256-element chunk are written as
+// zero: the tensor cores read them against zero codes, and the scratch they sit
+// in may hold an earlier call's bytes.
 __global__ void __launch_bounds__(kQuantThreads)
 prep_act_kernel(const uint16_t* __restrict__ x, int M, int K, uint8_t* __restrict__ codes,
                 uint8_t* __restrict__ sf_atoms) {
   griddep_launch_dependents();
   const int nb = K / 16;
+  const int nb_pad = (K + 255) / 256 * 16;
   const long long id = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (id >= static_cast<long long>(M) * nb) return;
-  const int m = static_cast<int>(id / nb), b = static_cast<int>(id % nb);
+  if (id >= static_cast<long long>(M) * nb_pad) return;
+  const int m = static_cast<int>(id / nb_pad), b = static_cast<int>(id % nb_pad);
+  if (b >= nb) {
+    sf_atoms[sf_atom_offset(static_cast<uint32_t>(m), static_cast<uint32_t>(b))] = 0;
+    return;
+  }
   float v[16];
   load_bf16_block(x, K, m, b, v);
   uint2 c;
@@ -137,7 +145,7 @@ cudaError_t launch_quant_act_rowmajor(const uint16_t* x, int M, int K, uint8_t* 
 
 cudaError_t launch_prep_act(const uint16_t* x, int M, int K, uint8_t* codes, uint8_t* sf_atoms,
                             cudaStream_t s) {
-  const long long n = static_cast<long long>(M) * (K / 16);
+  const long long n = static_cast<long long>(M) * ((K + 255) / 256 * 16);
   prep_act_kernel<<<grid_for(n), kQuantThreads, 0, s>>>(x, M, K, codes, sf_atoms);
   return cudaGetLastError();
 }

@@ -30,7 +30,7 @@ from dataclasses import dataclass
 import numpy as np
 
 __all__ = ["Workload", "CONFIGS", "SWEEP_MS", "SWEEP_RS", "sweep_config", "make_inputs",
-           "f32_to_bf16_bits", "bf16_bits_to_f32"]
+           "decompose_inputs", "f32_to_bf16_bits", "bf16_bits_to_f32"]
 
 
 @dataclass(frozen=True)
@@ -98,3 +98,22 @@ def make_inputs(w: Workload, *, with_R: bool = True) -> dict:
     if with_R:
         out["R"] = R
     return out
+
+
+def decompose_inputs(N: int, K: int, r: int, seed: int, planted: int = 0) -> dict:
+    """A weight to decompose and the start signs of the decomposition's terms.
+
+    W      float32 [N, K]: N(0, 0.02^2), plus `planted` binary rank-one terms
+           0.03 * 0.9^j * u_j v_j^T with Rademacher u_j, v_j (a structured part for
+           the peeling to find); drawn in this order: noise, planted signs.
+    v0     int8 [r, K]: Rademacher start signs, one row per term (the random
+           draws the method makes, handed to both sides).
+    """
+    rng = np.random.default_rng(seed)
+    W = rng.standard_normal((N, K), dtype=np.float32) * np.float32(0.02)
+    for j in range(planted):
+        u = (2 * rng.integers(0, 2, size=N) - 1).astype(np.float32)
+        v = (2 * rng.integers(0, 2, size=K) - 1).astype(np.float32)
+        W += np.float32(0.03 * 0.9 ** j) * np.outer(u, v).astype(np.float32)
+    v0 = (2 * rng.integers(0, 2, size=(r, K), dtype=np.int8) - 1).astype(np.int8)
+    return dict(W=W.astype(np.float32), v0=v0)
