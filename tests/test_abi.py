@@ -87,8 +87,11 @@ def test_kernel_count_follows_the_schedule(lib):
     # decode batches run one kernel (it quantises the activation itself)
     assert lib.biloco_gemm_kernel_count(1, 5120, 5120, 512) == 1
     assert lib.biloco_gemm_kernel_count(16, 13824, 5120, 512) == 1
+    assert lib.biloco_gemm_kernel_count(32, 5120, 13824, 512) == 1
+    assert lib.biloco_gemm_kernel_count(17, 5120, 5120, 1024) == 1
     # larger batches: quantiser + GEMM
-    assert lib.biloco_gemm_kernel_count(32, 5120, 13824, 512) == 2
+    assert lib.biloco_gemm_kernel_count(33, 5120, 13824, 512) == 2
+    assert lib.biloco_gemm_kernel_count(128, 5120, 5120, 512) == 2
     # the local-z schedule runs the general kernel (in-kernel quantisation up to M = 8)
     assert lib.biloco_set_mode(_lib.MODE_LOCAL_Z) == 0
     try:
@@ -97,3 +100,27 @@ def test_kernel_count_follows_the_schedule(lib):
     finally:
         lib.biloco_set_mode(_lib.MODE_AUTO)
     assert lib.biloco_gemm_kernel_count(1, 100, 64, 0) == -2
+
+
+def test_launch_form_and_selftest_controls(lib):
+    from nvfp4_binary_rank_b200 import _lib
+    assert lib.biloco_get_launch() == _lib.LAUNCH_PDL
+    assert lib.biloco_set_launch(4) == -1
+    assert lib.biloco_set_launch(-1) == -1
+    for f in (0, 1, 2, 3):
+        assert lib.biloco_set_launch(f) == 0
+        assert lib.biloco_get_launch() == f
+    assert lib.biloco_set_launch(_lib.LAUNCH_PDL) == 0
+    assert lib.biloco_selftest_drop_arrivals(4) == -1
+    assert lib.biloco_selftest_drop_arrivals(-1) == -1
+    assert lib.biloco_status_string(-8).decode() == "grid cannot be resident on the GPU at once"
+
+
+def test_correction_setting(lib):
+    from nvfp4_binary_rank_b200 import _lib
+    assert lib.biloco_set_correction(3) == -1
+    for a in (_lib.CORR_SIGNS, _lib.CORR_LUT):
+        assert lib.biloco_set_correction(a) == 0
+        assert lib.biloco_resolve_correction(1, 5120, 5120, 512) == a
+    assert lib.biloco_set_correction(_lib.CORR_AUTO) == 0
+    assert lib.biloco_resolve_correction(1, 5120, 5120, 512) in (_lib.CORR_SIGNS, _lib.CORR_LUT)

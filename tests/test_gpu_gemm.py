@@ -139,3 +139,92 @@ def test_shape_and_alignment_errors(nb):
     with pytest.raises(nb.BilocoError) as e:
         nb.gemm(buf[1:65].view(1, 64), W, sf, g, None, None, None)
     assert e.value.status == -3
+
+
+# --- full-size grids for the small decode classes and the general kernel ---------
+
+@pytest.mark.parametrize("M", [2, 3, 4])
+def test_decode_small_classes_full_grid(nb, M):
+    # classes 2 and 4 on a full 148-CTA grid at N = K = 5120, r = 512: the late CTAs
+    # that take no share of z, and (4 rows) the per-contributor tensor-core U side
+    w = workloads.Workload(f"full_M{M}", M, 5120, 5120, 512, 40 + M)
+    d, ref = oracle_for(w)
+    y = _run(nb, device_problem(w, d))
+    assert_y_close(y, ref["y"], w.name)
+
+
+@pytest.mark.parametrize("M", [4, 12])
+def test_general_kernel_full_size_sampled_rows(nb, M):
+    # M <= 16 with more than 16 units per CTA runs the general kernel: quantising per
+    # unit at 4 rows, after the activation pre-pass at 12.  The oracle checks a sample
+    # of output rows: quantising a weight row depends only on that row and the tensor
+    # scale g, so the sampled rows plus the row holding amax|R| give the same codes
+    # and the same g as the whole matrix.
+    w = workloads.Workload(f"big_M{M}", M, 13824, 13824, 512, 50 + M)
+    d = workloads.make_inputs(w)
+    y = _run(nb, device_problem(w, d))
+    R = d["R"]
+    n_max = int(np.unravel_index(np.argmax(np.abs(R)), R.shape)[0])
+    rng = np.random.default_rng(M)
+    rows = np.unique(np.concatenate([rng.choice(w.N, 384, replace=False),
+                                     [0, 1, 127, 128, 5119, 5120, w.N - 1, n_max]]))
+    ref = ob.biloco_reference(d["x"], R[rows], d["U"][rows], d["V"], d["alpha"])
+    from oracle import nvfp4 as on
+    assert ref["g"] == on.weight_global_scale(R)
+    assert_y_close(y[:, rows], ref["y"], w.name)
+
+
+@pytest.mark.parametrize("flags", [2, 3])
+@pytest.mark.parametrize("name", ["decode", "mlp_down"])
+def test_cooperative_launch(nb, flags, name):
+    # the opt-in launch form that guarantees co-residency of the grid gives the same y
+    w = workloads.CONFIGS[name]
+    d, ref = oracle_for(w)
+    prob = device_problem(w, d)
+    y_pdl = _run(nb, prob)
+    nb.set_launch(flags)
+    try:
+        y = _run(nb, prob)
+        y2 = _run(nb, prob)
+    finally:
+        nb.set_launch(nb.LAUNCH_PDL)
+    assert_y_close(y, ref["y"], name)
+    np.testing.assert_array_equal(y, y2)
+    np.testing.assert_array_equal(y, y_pdl)
+
+
+# --- the 32-row class of the decode kernel (17 to 32 rows) ------------------------
+
+@pytest.mark.parametrize("M,N,K,r", [(17, 384, 832, 255), (20, 640, 1344, 0), (24, 1280, 4096, 1024),
+                                     (29, 2560, 5184, 600), (32, 128, 64, 3), (32, 5120, 13824, 1024),
+                                     (18, 13824, 5120, 512)])
+def test_batch32_class(nb, M, N, K, r):
+    # activation chunks streamed with the weight stages from the grid's image; ranks
+    # above 512 cycle the z tiles through the slot ring (r = 1024: two groups)
+    w = _small(M, N, K, r, seed=M * 5 + r)
+    d, ref = oracle_for(w)
+    y = _run(nb, device_problem(w, d))
+    assert_y_close(y, ref["y"], w.name)
+    if r == 0:
+        tol = np.abs(ref["gemm"]) * 2.0 ** -8 + 1e-6 * np.abs(ref["gemm"]).max()
+        assert np.all(np.abs(y - ref["gemm"]) <= tol)
+
+
+# --- the correction arithmetic of the 1-2-row U side: sign-adds and table lookups ---
+
+@pytest.mark.parametrize("arith", [1, 2])
+@pytest.mark.parametrize("M,N,K,r", [(1, 5120, 5120, 512), (2, 640, 1344, 100), (1, 128, 64, 1),
+                                     (2, 1280, 2560, 1024), (1, 13824, 5120, 33)])
+def test_correction_arithmetic(nb, arith, M, N, K, r):
+    w = _small(M, N, K, r, seed=M * 11 + r)
+    d, ref = oracle_for(w)
+    prob = device_problem(w, d)
+    nb.set_correction(arith)
+    try:
+        assert nb.resolve_correction(M, N, K, r) == arith
+        y = _run(nb, prob)
+        y2 = _run(nb, prob)
+    finally:
+        nb.set_correction(nb.CORR_AUTO)
+    assert_y_close(y, ref["y"], f"{w.name} arith {arith}")
+    np.testing.assert_array_equal(y, y2)

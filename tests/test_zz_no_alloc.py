@@ -54,6 +54,7 @@ SHAPES = [
     ("ragged_m16", workloads.Workload("na_16_256_320_17", 16, 256, 320, 17, 11), 1),
     ("ragged_m16", workloads.Workload("na_16_256_320_17", 16, 256, 320, 17, 11), 2),
     ("m40", workloads.Workload("na_40_384_576_40", 40, 384, 576, 40, 12), 1),
+    ("m24", workloads.Workload("na_24_640_1344_100", 24, 640, 1344, 100, 14), 1),
     ("m3_r0", workloads.Workload("na_3_256_512_0", 3, 256, 512, 0, 13), 1),
     ("mlp_up", workloads.CONFIGS["mlp_up"], 1),
 ]
