@@ -75,10 +75,10 @@ def kernel_source_digest() -> str:
 
 def ncu_traffic(workload: str, M: int):
     """DRAM bytes (read + write) per launch of the GEMM kernel that serves this
-    workload (decode_kernel for M <= 16, fused_kernel above), from the committed
+    workload (decode_kernel for M <= 32, fused_kernel above), from the committed
     ncu summary, or None when there is none or the kernel sources changed since
     it was captured."""
-    kernel = "decode_kernel" if M <= 16 else "fused_kernel"
+    kernel = "decode_kernel" if M <= 32 else "fused_kernel"
     path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
     try:
         fields = {}
@@ -180,7 +180,7 @@ def n_copies_for(w, l2_bytes):
     return max(2, int(np.ceil(1.25 * l2_bytes / per)))
 
 
-def time_graph(prob, steps, warmup, stream, dist_ctx):
+def time_graph(prob, steps, warmup, stream, dist_ctx, spread_pass=True):
     """Device time of exactly `steps` calls replayed from CUDA graphs."""
     import torch
     import nvfp4_binary_rank_b200 as nb
@@ -237,7 +237,64 @@ def time_graph(prob, steps, warmup, stream, dist_ctx):
     if st != 0:
         raise RuntimeError(f"timed region failed: {nb.status_string(st)}")
     del g_full, g_rem
+    time_graph.per_step_us, time_graph.chunk = [], chunk
+    if not spread_pass:
+        return ms
+    # The spread, outside the timed region: SPREAD_REPLAYS replays of a graph of
+    # `chunk` calls, each bracketed by events; per-step median and 10th percentile.
+    g_sp = capture(chunk)
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(SPREAD_REPLAYS + 1)]
+    with torch.cuda.stream(stream):
+        g_sp.replay()
+        evs[0].record(stream)
+        for i in range(SPREAD_REPLAYS):
+            g_sp.replay()
+            evs[i + 1].record(stream)
+    evs[-1].synchronize()
+    time_graph.per_step_us = [evs[i].elapsed_time(evs[i + 1]) * 1e3 / chunk for i in range(SPREAD_REPLAYS)]
+    time_graph.chunk = chunk
+    if nb.last_error(stream) != 0:
+        raise RuntimeError("spread pass failed")
+    del g_sp
     return ms
+
+
+SPREAD_REPLAYS = 30
+
+
+def spread(per_step_us, chunk):
+    """Median and 10th percentile of the per-step times of the spread pass."""
+    a = np.asarray(per_step_us, dtype=np.float64)
+    if a.size == 0:
+        return {"median_us": None, "p10_us": None, "replays": 0}
+    return {"median_us": round(float(np.median(a)), 3), "p10_us": round(float(np.percentile(a, 10)), 3),
+            "replays": int(a.size), "calls_per_replay": int(chunk)}
+
+
+def time_isolated(prob, calls, stream):
+    """One call at a time, not overlapped with another: each call is bracketed by
+    events with a synchronisation before it, and reads a weight copy the calls
+    before it did not touch.  Returns the median device time of one call (us)."""
+    import torch
+    import nvfp4_binary_rank_b200 as nb
+    copies = prob["copies"]
+    nc = len(copies)
+    times = []
+    with torch.cuda.stream(stream):
+        for i in range(calls + 3):
+            W, sf, g = copies[i % nc]
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            stream.synchronize()
+            a.record(stream)
+            nb.gemm(prob["x"], W, sf, g, prob["Ub"], prob["Vb"], prob["alpha"], out=prob["y"])
+            b.record(stream)
+            b.synchronize()
+            if i >= 3:
+                times.append(a.elapsed_time(b) * 1e3)
+    if nb.last_error(stream) != 0:
+        raise RuntimeError("isolated calls failed")
+    return round(float(np.median(times)), 3)
 
 
 def time_e2e(prob, steps, stream):
@@ -322,16 +379,51 @@ def step_metrics(bytes_per_step: int, ms_max: float, steps: int, world: int):
 
 def measure_config(w, steps, warmup, stream, dist_ctx, l2):
     import torch
+    import nvfp4_binary_rank_b200 as nb
     prob = setup_problem(w, n_copies_for(w, l2), torch.device("cuda", torch.cuda.current_device()))
     ms = dist_ctx.max(time_graph(prob, steps, warmup, stream, dist_ctx))
     us = ms * 1e3 / steps
     b = algo_bytes(w.M, w.N, w.K, w.r)
     peak, _ = hbm_peak()
     out = {"us": round(us, 3), "GBps": round(b / (us * 1e-6) / 1e9, 1),
-           "frac": round(b / (us * 1e-6) / 1e9 / peak, 4), "bytes": b}
+           "frac": round(b / (us * 1e-6) / 1e9 / peak, 4), "bytes": b,
+           "M": w.M, "N": w.N, "K": w.K, "r": w.r,
+           "kernels": nb.gemm_kernel_count(w.M, w.N, w.K, w.r)}
+    out.update(spread(time_graph.per_step_us, time_graph.chunk))
     del prob
     torch.cuda.empty_cache()
     return out
+
+
+EXTRA_CONFIGS = [
+    ("mlp_up", workloads.CONFIGS["mlp_up"]),
+    ("mlp_down", workloads.CONFIGS["mlp_down"]),
+    ("sweep_M8_r512", workloads.sweep_config(8, 512)),
+    ("sweep_M16_r512", workloads.sweep_config(16, 512)),
+    ("sweep_M32_r512", workloads.sweep_config(32, 512)),
+    ("sweep_M1_r0", workloads.sweep_config(1, 0)),
+    ("sweep_M32_r1024", workloads.sweep_config(32, 1024)),
+    ("sweep_M64_r512", workloads.sweep_config(64, 512)),
+    ("sweep_M128_r512", workloads.sweep_config(128, 512)),
+]
+
+
+def workload_config(w, world):
+    """The `config` object of both arms: the workload and how it is laid out."""
+    return {"workload": w.name, "M": w.M, "N": w.N, "K": w.K, "r": w.r, "seed": w.seed,
+            "parallelism": f"replicas x{world}", "l2": "inputs larger than L2"}
+
+
+def metric_range(head_us, head_frac, extra):
+    """The metric over its stated batch range at r = 512, K = 5120: the headline
+    (M = 1) and the sweep points M = 8, 16, 32, with the worst of them."""
+    pts = {"M1": {"us": round(head_us, 3), "frac": round(head_frac, 4)}}
+    for m in (8, 16, 32):
+        e = extra.get(f"sweep_M{m}_r512")
+        if e:
+            pts[f"M{m}"] = {"us": e["us"], "frac": e["frac"]}
+    worst = min(pts.items(), key=lambda kv: kv[1]["frac"])
+    return {"points": pts, "worst": {"M": int(worst[0][1:]), **worst[1]}}
 
 
 def run_ours(args):
@@ -352,12 +444,14 @@ def run_ours(args):
 
     prob = setup_problem(w, n_copies_for(w, l2), torch.device("cuda", ctx.local))
     with ClockSampler(ctx.local) as clk:
-        ms_local = time_graph(prob, args.steps, args.warmup, stream, ctx)
+        ms_local = time_graph(prob, args.steps, args.warmup, stream, ctx, spread_pass=not args.timed_only)
+    head_spread = spread(time_graph.per_step_us, time_graph.chunk)
     ms = ctx.max(ms_local)
     b = algo_bytes(w.M, w.N, w.K, w.r)
     us, gbs_rank, value = step_metrics(b, ms, args.steps, ctx.world)
+    isolated_us = None if args.timed_only else time_isolated(prob, 200, stream)
 
-    e2e_steps = min(args.steps, 2000)
+    e2e_steps = 3 if args.timed_only else min(args.steps, 2000)
     e2e_ms, h2d, d2h = time_e2e(prob, e2e_steps, stream)
     e2e_ms = ctx.max(e2e_ms)
     e2e_val = b * ctx.world / (e2e_ms * 1e-3) / 1e9
@@ -365,24 +459,24 @@ def run_ours(args):
     torch.cuda.empty_cache()
 
     extra = {}
+    rng_line = None
     if not args.no_extra:
         sub_steps = max(2000, args.steps // 20)
-        for name, ww in [("mlp_up", workloads.CONFIGS["mlp_up"]),
-                         ("mlp_down", workloads.CONFIGS["mlp_down"]),
-                         ("sweep_M8_r512", workloads.sweep_config(8, 512)),
-                         ("sweep_M32_r512", workloads.sweep_config(32, 512)),
-                         ("sweep_M1_r0", workloads.sweep_config(1, 0))]:
+        for name, ww in EXTRA_CONFIGS:
             extra[name] = measure_config(ww, sub_steps, args.warmup, stream, ctx, l2)
+        rng_line = metric_range(us, gbs_rank / peak, extra)
 
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": ctx.world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 6),
         "us_per_call": round(us, 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "nvfp4", "data": "synthetic",
-        "config": {"workload": w.name, "M": w.M, "N": w.N, "K": w.K, "r": w.r,
-                   "seed": w.seed, "parallelism": f"replicas x{ctx.world}",
-                   "l2": f"{n_copies_for(w, l2)} weight copies rotated (> L2 {l2 >> 20} MiB)",
-                   "launch": f"CUDA graph replay, {nb.gemm_kernel_count(w.M, w.N, w.K, w.r)} kernel(s) per step"},
+        "config": workload_config(w, ctx.world),
+        "timing": {"l2": f"{n_copies_for(w, l2)} weight copies rotated (> L2 {l2 >> 20} MiB)",
+                   "launch": f"CUDA graph replay, {nb.gemm_kernel_count(w.M, w.N, w.K, w.r)} kernel(s) per step",
+                   "spread": head_spread,
+                   "isolated_us": isolated_us,
+                   "isolated": "one call at a time (synchronised before it, not overlapped), median of 200"},
         "roofline": {"bound": "hbm", "achieved": round(gbs_rank, 1), "peak": peak,
                      "unit": "GB/s", "frac": round(gbs_rank / peak, 4),
                      "traffic": ncu_traffic(w.name, w.M),
@@ -393,9 +487,11 @@ def run_ours(args):
         "gpu_launches": nb.gemm_kernel_count(w.M, w.N, w.K, w.r) * args.steps,
         "clocks": clk.summary(),
         "extra_configs": extra,
+        "range_M1_32_r512_K5120": rng_line,
     }
     if ctx.world == 1 and ctx.rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, budget_s=12.0)
+        line["cpu_baseline_1thread"] = cpu_baseline(w, budget_s=6.0, threads=1)
     if ctx.rank == 0:
         print(json.dumps(line), flush=True)
     ctx.close()
@@ -434,19 +530,28 @@ def _threads():
         return os.cpu_count() or 1
 
 
-def cpu_baseline(w, budget_s=12.0, rows=None):
+def cpu_baseline(w, budget_s=12.0, rows=None, threads=None):
+    """The oracle as it stands, timed on the host's cores: NumPy's BLAS threads
+    (all cores by default), or `threads` of them."""
+    import contextlib
     rows = w.N if rows is None else rows
     s = _oracle_sample(w, rows)
     b = algo_bytes(w.M, rows, w.K, w.r)
-    t0 = time.perf_counter()
-    n = 0
-    while True:
-        _oracle_step(s)
-        n += 1
-        if time.perf_counter() - t0 >= budget_s:
-            break
-    dt = (time.perf_counter() - t0) / n
-    return {"value": round(b / dt / 1e9, 4), "unit": UNIT, "cores": _threads(), "kind": "oracle",
+    limit = contextlib.nullcontext()
+    if threads is not None:
+        from threadpoolctl import threadpool_limits
+        limit = threadpool_limits(threads)
+    with limit:
+        cores = _threads()
+        t0 = time.perf_counter()
+        n = 0
+        while True:
+            _oracle_step(s)
+            n += 1
+            if time.perf_counter() - t0 >= budget_s:
+                break
+        dt = (time.perf_counter() - t0) / n
+    return {"value": round(b / dt / 1e9, 4), "unit": UNIT, "cores": cores, "kind": "oracle",
             "sample": f"{n} full oracle passes (quantise x, FP64 GEMM part from packed weight, "
                       f"FP64 correction) over {w.name} rows 0..{rows}, {dt * 1e3:.1f} ms each"}
 
@@ -500,8 +605,9 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "impl": "reference",
-        "config": {"workload": w.name, "M": w.M, "N": w.N, "K": w.K, "r": w.r, "seed": w.seed,
-                   "rows_per_step": rows, "k_per_step": kk, "ranks_per_step": rr},
+        "config": workload_config(w, int(args.gpus)),
+        "sample": {"rows_per_step": rows, "k_per_step": kk, "ranks_per_step": rr,
+                   "whole_problem": bool(rows == w.N and kk == w.K and rr == w.r)},
         "cpu_baseline": {"value": round(val, 4), "unit": UNIT, "cores": _threads(), "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": round(val, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -518,9 +624,14 @@ def main():
     ap.add_argument("--workload", choices=sorted(workloads.CONFIGS), default="decode")
     ap.add_argument("--no-extra", action="store_true", help="skip the other workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--timed-only", action="store_true",
+                    help="setup and the timed region only (for profiler runs): no spread pass, isolated "
+                         "calls, end-to-end loop, other workloads or CPU baseline")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    if args.timed_only:
+        args.no_extra = args.no_cpu_baseline = True
     if args.impl == "reference":
         run_reference(args)
     else:
