@@ -577,9 +577,9 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
         // A stage = the weight unit (TMA tile + scale atoms) and the activation
         // chunk of the same K range (one bulk copy of its image chunk).  The weight
         // parts of the first stages are requested at once; the activation parts
-        // once the CTA's CUDA-core warps have seen every CTA publish its part of
-        // the image (actr_bar), always issued so that every stage's transaction
-        // count completes even after a failed wait.
+        // once every CTA has published its part of the image, which this thread
+        // waits for itself; always issued, so that every stage's transaction count
+        // completes even after a failed wait.
         constexpr uint32_t kImg = QImg<MC>::kBytes;
         const int pre = min(nunits, kStages);
         for (int k = 0; k < pre; ++k) {
@@ -590,8 +590,20 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
           sf += kSfBytes;
           if (++c == p.KC) { c = 0; ++t; }
         }
-        bool ok = mbar_wait(actr_bar, 0, abort_flag);
-        if (!ok) fail(ctl);
+        // every CTA has written its part of the activation image (the counter
+        // belongs to this call once the previous kernel of the stream has ended)
+        griddep_wait();
+        bool ok = spin_until_geq(p.q_ready, static_cast<uint32_t>(p.G), ctl);
+        if (ok) {
+          // the last CTA past the wait resets both counters for the next call
+          const uint32_t old = atomicAdd(p.q_seen, 1u);
+          if (old == static_cast<uint32_t>(p.G - 1)) {
+            atomicExch(p.q_ready, 0u);
+            atomicExch(p.q_seen, 0u);
+          }
+        } else {
+          fail(ctl);
+        }
         fence_proxy_async_global();                      // the image was written through the generic proxy
         int ca = u0 % p.KC;
         for (int k = 0; k < pre; ++k) {
@@ -1099,8 +1111,11 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
             *reinterpret_cast<uint4*>(img + m * 128 + (((2 * st + 1) ^ (m & 7)) << 4)) = make_uint4(cw[4], cw[5], cw[6], cw[7]);
             *reinterpret_cast<uint4*>(img + kImgCodes + st * 512 + m * 16) = make_uint4(sc4, 0u, 0u, 0u);
           }
-          // the producers read the image with bulk copies (the async proxy)
+          // the producers read the image with bulk copies (the async proxy); this
+          // CTA's part is published at once, ahead of the V pieces
           fence_proxy_async_global();
+          named_barrier(kBarAlu, kAluThreads);
+          if (tid == 0 && !(p.drop & 2)) red_add_release_gpu(p.q_ready, 1u);
         }
         if constexpr (Cfg<MC>::kTensorV) {
           if (p.r > 0) {
@@ -1125,16 +1140,16 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
               const int a0 = static_cast<int>(static_cast<int64_t>(sl) * KA / S);
               const int a1 = static_cast<int>(static_cast<int64_t>(sl + 1) * KA / S);
               const int rank = rb * kTileRows + row;
-              for (int b0 = a0; b0 < a1; b0 += kVAtoms) {
+              // Batches of kVAtoms atoms.  The next batch's sign words and activation
+              // pieces are requested before waiting for the current batch's MMAs, so
+              // that only the first batch of a piece waits on memory.
+              constexpr int kXL = (kVAtoms * kBN * 8 + kAluThreads - 1) / kAluThreads;
+              auto load_batch = [&](int b0, uint32_t (&vw)[kVAtoms], uint4 (&xv)[kXL]) {
                 const int nb = min(kVAtoms, a1 - b0);
-                // requests first: this thread's sign words and activation pieces
-                uint32_t vw[kVAtoms];
 #pragma unroll
                 for (int j = 0; j < kVAtoms; ++j)
                   vw[j] = (j < nb && rank < p.r) ? __ldcg(p.Vbits + static_cast<size_t>(rank) * p.KW + 2 * (b0 + j) + half)
                                                  : 0u;
-                constexpr int kXL = (kVAtoms * kBN * 8 + kAluThreads - 1) / kAluThreads;
-                uint4 xv[kXL];
 #pragma unroll
                 for (int e = 0; e < kXL; ++e) {
                   const int idx = e * kAluThreads + tid;
@@ -1143,6 +1158,12 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
                               ? __ldcg(reinterpret_cast<const uint4*>(p.x + static_cast<size_t>(m) * p.K + 64 * (b0 + j) + 8 * c))
                               : make_uint4(0u, 0u, 0u, 0u);
                 }
+              };
+              uint32_t vw[kVAtoms];
+              uint4 xv[kXL];
+              load_batch(a0, vw, xv);
+              for (int b0 = a0; b0 < a1; b0 += kVAtoms) {
+                const int nb = min(kVAtoms, a1 - b0);
 #pragma unroll
                 for (int j = 0; j < kVAtoms; ++j) {
                   if (j < nb) {
@@ -1169,6 +1190,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
                 }
                 fence_proxy_async_smem();
                 named_barrier(kBarAlu, kAluThreads);
+                if (b0 + kVAtoms < a1) load_batch(b0 + kVAtoms, vw, xv);   // the next batch, in flight during the MMAs
                 bool okv = true;
                 if (tid == 0) {
                   tc_fence_after();
@@ -1208,25 +1230,40 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
           }
         }
         named_barrier(kBarAlu, kAluThreads);
-        bool okq = true;
-        if (tid == 0) {
-          if (!(p.drop & 2)) red_add_release_gpu(p.q_ready, 1u);   // covers the items the CTA wrote
-          okq = spin_until_geq(p.q_ready, static_cast<uint32_t>(p.G), ctl);
-          if (okq) {
-            // the last CTA past the wait resets both counters for the next call
-            const uint32_t old = atomicAdd(p.q_seen, 1u);
-            if (old == static_cast<uint32_t>(p.G - 1)) {
-              atomicExch(p.q_ready, 0u);
-              atomicExch(p.q_seen, 0u);
+        if constexpr (kStream) {
+          // the V pieces' partial sums, behind their own counter (the image went out
+          // before them, and the producer waits for it)
+          if (p.r > 0) {
+            bool okv = true;
+            if (tid == 0) {
+              red_add_release_gpu(p.v_ready, 1u);             // covers the pieces the CTA wrote
+              okv = spin_until_geq(p.v_ready, static_cast<uint32_t>(p.G), ctl);
+              if (okv) {
+                // the last CTA past the wait resets both counters for the next call
+                const uint32_t old = atomicAdd(p.v_seen, 1u);
+                if (old == static_cast<uint32_t>(p.G - 1)) {
+                  atomicExch(p.v_ready, 0u);
+                  atomicExch(p.v_seen, 0u);
+                }
+              }
+            }
+            if (named_barrier_or(kBarAlu, kAluThreads, !okv)) fail(ctl);
+          }
+        } else {
+          bool okq = true;
+          if (tid == 0) {
+            if (!(p.drop & 2)) red_add_release_gpu(p.q_ready, 1u);   // covers the items the CTA wrote
+            okq = spin_until_geq(p.q_ready, static_cast<uint32_t>(p.G), ctl);
+            if (okq) {
+              // the last CTA past the wait resets both counters for the next call
+              const uint32_t old = atomicAdd(p.q_seen, 1u);
+              if (old == static_cast<uint32_t>(p.G - 1)) {
+                atomicExch(p.q_ready, 0u);
+                atomicExch(p.q_seen, 0u);
+              }
             }
           }
-        }
-        if (named_barrier_or(kBarAlu, kAluThreads, !okq)) fail(ctl);
-        if constexpr (kStream) {
-          // the image is complete: the producer may fetch its chunks (after a
-          // failed wait too, so that its stages complete)
-          if (tid == 0) mbar_arrive(actr_bar);
-        } else {
+          if (named_barrier_or(kBarAlu, kAluThreads, !okq)) fail(ctl);
           // one round of 16-byte loads: 144 per unit (128 of codes, 16 of scales)
           constexpr int kPer = kImgBytes / 16;
           constexpr int kLd = (L::kMaxUnits * kPer + kAluThreads - 1) / kAluThreads;
@@ -1322,30 +1359,44 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
         const int S = vside_slices(p, RB);
         constexpr int kParts = 4, kPerPart = kVSliceMax / kParts;
         const int P = (i1 - i0) * p.M;
-        for (int base = 0; base < P * kParts; base += kAluThreads) {
-          const int idx = base + tid, pair = idx >> 2, part = idx & 3;
-          const bool act = pair < P;
-          const int il = act ? pair / p.M : 0;
-          const int i = i0 + il, m = act ? pair - il * p.M : 0;
-          const float* src = p.vpart + (static_cast<size_t>(i / kTileRows) * S * kBN + m) * kTileRows + (i % kTileRows);
-          // every request of the round first: the partial sums and alpha
-          const float al = (act && part == 0) ? __ldcg(p.alpha + i) : 0.0f;
-          float t[kPerPart];
+        // rounds of kAluThreads (rank, row, part) items, kRounds of them per pass with
+        // every request of the pass issued first (the partial sums and alpha): one
+        // memory round trip per pass instead of per round (at 32 rows a slice takes two)
+        constexpr int kRounds = (MC > 16) ? 2 : 1;
+        for (int base = 0; base < P * kParts; base += kRounds * kAluThreads) {
+          float t[kRounds][kPerPart], al[kRounds];
+          int iv[kRounds], mv[kRounds];
+          bool actv[kRounds];
 #pragma unroll
-          for (int q = 0; q < kPerPart; ++q) {
-            const int sl = part + kParts * q;
-            t[q] = (act && sl < S) ? __ldcg(src + static_cast<size_t>(sl) * kBN * kTileRows) : 0.0f;
+          for (int e = 0; e < kRounds; ++e) {
+            const int idx = base + e * kAluThreads + tid, pair = idx >> 2, part = idx & 3;
+            const bool act = pair < P;
+            const int il = act ? pair / p.M : 0;
+            const int i = i0 + il, m = act ? pair - il * p.M : 0;
+            iv[e] = i;
+            mv[e] = m;
+            actv[e] = act && part == 0;
+            const float* src = p.vpart + (static_cast<size_t>(i / kTileRows) * S * kBN + m) * kTileRows + (i % kTileRows);
+            al[e] = (act && part == 0) ? __ldcg(p.alpha + i) : 0.0f;
+#pragma unroll
+            for (int q = 0; q < kPerPart; ++q) {
+              const int sl = part + kParts * q;
+              t[e][q] = (act && sl < S) ? __ldcg(src + static_cast<size_t>(sl) * kBN * kTileRows) : 0.0f;
+            }
           }
-          float sum = 0.0f;
 #pragma unroll
-          for (int q = 0; q < kPerPart; ++q) sum += t[q];
-          sum += __shfl_xor_sync(0xffffffffu, sum, 1);
-          sum += __shfl_xor_sync(0xffffffffu, sum, 2);
-          if (act && part == 0) {
-            const float zv = __fmul_rn(al, sum);
-            const __nv_bfloat16 hi = __float2bfloat16_rn(zv);
-            const __nv_bfloat16 lo = __float2bfloat16_rn(zv - __bfloat162float(hi));
-            store_ztile(p.ztiles, Layout<MC>::kUN, MC, m, i, hi, lo);
+          for (int e = 0; e < kRounds; ++e) {
+            float sum = 0.0f;
+#pragma unroll
+            for (int q = 0; q < kPerPart; ++q) sum += t[e][q];
+            sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+            sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+            if (actv[e]) {
+              const float zv = __fmul_rn(al[e], sum);
+              const __nv_bfloat16 hi = __float2bfloat16_rn(zv);
+              const __nv_bfloat16 lo = __float2bfloat16_rn(zv - __bfloat162float(hi));
+              store_ztile(p.ztiles, Layout<MC>::kUN, MC, mv[e], iv[e], hi, lo);
+            }
           }
         }
       }

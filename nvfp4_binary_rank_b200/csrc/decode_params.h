@@ -24,6 +24,8 @@ struct DecodeParams {
   uint32_t* tickets;       // [T] split-K arrivals per weight tile
   uint32_t* q_ready;       // CTAs that published their part of the activation image
   uint32_t* q_seen;        // CTAs done with q_ready (the last one resets both)
+  uint32_t* v_ready;       // 32-row class: CTAs that published their V pieces' partial sums
+  uint32_t* v_seen;        // CTAs done with v_ready (the last one resets both)
   int* status;             // first device-side error
   int M, N, K, r;
   int KC, T, U, G, KW, RW, rpad;
