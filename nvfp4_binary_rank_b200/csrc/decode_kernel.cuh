@@ -175,19 +175,21 @@ struct Layout {
   static constexpr int kVRed = kUEnd;                                  // [8][MC * ranks] floats
   static constexpr int kVRedBytes = Cfg<MC>::kTensorV ? 0 : kAluWarps * MC * kRankGroup * 4;
   static constexpr int kBar = kVRed + kVRedBytes;
-  static constexpr int kNumBars = 2 * kStages + 13;
+  static constexpr int kNumBars = 2 * kStages + 17;
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kFinFlags = kMisc + 32;                         // [kMaxUnits + 1] ints
   static constexpr int kTotal = kFinFlags + (kMaxUnits + 1) * 4;
   static constexpr int kAlloc = kTotal + 1024;
   // TMEM columns.  Cache classes: accumulators [0, 32), activation scales per unit
-  // [32, 288), weight scales per stage [288, 384), the U-side product [384, 416),
-  // the V-side product [448, 464).  Streamed class: accumulators [0, 64), weight
-  // and activation scales per stage, then the U-side (64) and V-side (32) products.
+  // [32, 288), weight scales per stage [288, 384), the two U-side product buffers
+  // [384, 384 + 2 kUN), the V-side product [448, 464).  Streamed class:
+  // accumulators [0, 64), weight and activation scales per stage, then the two
+  // U-side product buffers (2 x 64) and the V-side product (32).
   static constexpr int kTmSfb = kStream ? 2 * kBN + kStages * 16 : 32;
   static constexpr int kTmSfa = kStream ? 2 * kBN : kTmSfb + kMaxUnits * 16;
-  static constexpr int kTmU = kStream ? kTmSfb + kStages * 16 : 384;
-  static constexpr int kTmV = kStream ? kTmU + kUN : 448;
+  static constexpr int kTmU = kStream ? kTmSfb + kStages * 16 : 384;   // two buffers of kUN columns
+  static constexpr int kTmV = kStream ? kTmU + 2 * kUN : 448;
+  static_assert(!Cfg<MC>::kTensorU || kTmU + 2 * kUN <= kTmV, "two U-side product buffers");
   static_assert(kTmV + kBN <= kTmemCols, "tensor memory budget");
   static_assert(kStream || kTmSfa + kStages * 16 <= kTmU, "tensor memory budget");
   static_assert(kSFA % 1024 == 0 && kB % 1024 == 0 && kUA % 1024 == 0 && kUZ % 1024 == 0 &&
@@ -499,7 +501,11 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
   const uint32_t drain_bar = smem_u32(&bars[2 * kStages + 5]);
   const uint32_t done_bar = smem_u32(&bars[2 * kStages + 6]);
   auto ubuf_bar = [&](int b) { return smem_u32(&bars[2 * kStages + 7 + b]); };
-  const uint32_t ud_bar = smem_u32(&bars[2 * kStages + 9]);
+  // the U-side product of segment s lands in TMEM buffer s & 1: ud_bar(b) when it
+  // is ready (tcgen05.commit), uread_bar(b) when the epilogue has read it
+  auto ud_bar = [&](int b) { return smem_u32(&bars[b ? 2 * kStages + 13 : 2 * kStages + 9]); };
+  auto uread_bar = [&](int b) { return smem_u32(&bars[2 * kStages + 14 + b]); };
+  const uint32_t qpass_bar = smem_u32(&bars[2 * kStages + 16]);   // streamed class: the producer passed the image wait
   auto ufull_bar = [&](int b) { return smem_u32(&bars[2 * kStages + 10 + b]); };
   const uint32_t vmma_bar = smem_u32(&bars[2 * kStages + 12]);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMisc);
@@ -529,7 +535,11 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
     mbar_init(done_bar, kWarps);
     mbar_init(ubuf_bar(0), 1);
     mbar_init(ubuf_bar(1), 1);
-    mbar_init(ud_bar, 1);
+    mbar_init(ud_bar(0), 1);
+    mbar_init(ud_bar(1), 1);
+    mbar_init(uread_bar(0), kEpiThreads);
+    mbar_init(uread_bar(1), kEpiThreads);
+    mbar_init(qpass_bar, 1);
     mbar_init(ufull_bar(0), kAluThreads);
     mbar_init(ufull_bar(1), kAluThreads);
     mbar_init(vmma_bar, 1);
@@ -594,16 +604,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
         // belongs to this call once the previous kernel of the stream has ended)
         griddep_wait();
         bool ok = spin_until_geq(p.q_ready, static_cast<uint32_t>(p.G), ctl);
-        if (ok) {
-          // the last CTA past the wait resets both counters for the next call
-          const uint32_t old = atomicAdd(p.q_seen, 1u);
-          if (old == static_cast<uint32_t>(p.G - 1)) {
-            atomicExch(p.q_ready, 0u);
-            atomicExch(p.q_seen, 0u);
-          }
-        } else {
-          fail(ctl);
-        }
+        if (!ok) fail(ctl);
+        mbar_arrive(qpass_bar);                          // done with the grid counters
         fence_proxy_async_global();                      // the image was written through the generic proxy
         int ca = u0 % p.KC;
         for (int k = 0; k < pre; ++k) {
@@ -775,36 +777,24 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
           tc_fence_before();
           mbar_arrive(acce_bar(b));
         }
-        if (p.r > 0) {
-          // this CTA's share of U z for the tile: the CUDA-core warps compute it once
-          // z is complete (barrier 1: the previous segment's share has been read;
-          // barrier 2: this one is ready)
-          if (named_barrier_or(kBarFin, kFinThreads, !ok)) {
-            if (ok) fail(ctl);
-            ok = false;
-          }
-          if (named_barrier_or(kBarFin2, kFinThreads, !ok)) {
-            if (ok) fail(ctl);
-            ok = false;
-          }
-          if (!ok) break;
-          if constexpr (Cfg<MC>::kTensorU) {
-            // the U-side MMAs left sum_i U[n][i] zhi[m][i] in column m and
-            // sum_i U[n][i] zlo[m][i] in column MC + m of lane n
-            const bool got = group_wait(ud_bar, seg & 1, kBarEpi, kEpiThreads, ctl);
-            if (!got) {
-              // not a break: the next segment's kBarFin / kBarFin2 still have to be
-              // taken with the CUDA-core warps, which leave after kBarFin2
-              ok = false;
-              continue;
-            }
-            if (fin_flag[seg]) {
+        if constexpr (Cfg<MC>::kTensorU) {
+          if (p.r > 0) {
+            // This CTA's share of U z for the tile (the 64-rank chunks [cs0, cs1), the
+            // split the CUDA-core warps use), from TMEM buffer b once ud_bar(b) has
+            // completed for this segment; the MMAs left sum_i U[n][i] zhi[m][i] in
+            // column m and sum_i U[n][i] zlo[m][i] in column MC + m of lane n.
+            const int nuc = (p.r + kUChunk - 1) / kUChunk;
+            const int ua = max(u0, t * p.KC), ub = min(u1, (t + 1) * p.KC);
+            const int cs0 = (ua - t * p.KC) * nuc / p.KC, cs1 = (ub - t * p.KC) * nuc / p.KC;
+            if (ok) ok = group_wait(ud_bar(b), (seg >> 1) & 1, kBarEpi, kEpiThreads, ctl);
+            if (ok && cs1 > cs0) {
               tc_fence_after();
+              const uint32_t ucol = L::kTmU + static_cast<uint32_t>(b * L::kUN);
               if constexpr (L::kUN <= 32) {
                 uint32_t du[L::kUN];
-                tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + L::kTmU, *reinterpret_cast<uint32_t(*)[16]>(du));
+                tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + ucol, *reinterpret_cast<uint32_t(*)[16]>(du));
                 if constexpr (L::kUN > 16)
-                  tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + L::kTmU + 16,
+                  tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + ucol + 16,
                             *reinterpret_cast<uint32_t(*)[16]>(du + 16));
                 tmem_wait_ld();
     #pragma unroll
@@ -814,20 +804,18 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
     #pragma unroll
                 for (int c0 = 0; c0 < MC; c0 += 16) {
                   uint32_t hi[16], lo[16];
-                  tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + L::kTmU + c0, hi);
-                  tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + L::kTmU + MC + c0, lo);
+                  tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + ucol + c0, hi);
+                  tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + ucol + MC + c0, lo);
                   tmem_wait_ld();
     #pragma unroll
                   for (int j = 0; j < 16; ++j) v[c0 + j] += __uint_as_float(hi[j]) + __uint_as_float(lo[j]);
                 }
               }
-              tc_fence_before();
             }
-          } else {
-            const float* corr = reinterpret_cast<const float*>(smem + L::kCorr);
-  #pragma unroll
-            for (int j = 0; j < MC; ++j)
-              v[j] = (v[j] + corr[j * kTileRows + row]) + corr[(MC + j) * kTileRows + row];
+            // buffer b may take segment seg + 2's product (arrived on every path, so
+            // that the phases stay in step)
+            tc_fence_before();
+            mbar_arrive(uread_bar(b));
           }
         }
         if (!ok) break;
@@ -1211,17 +1199,21 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
               // the piece's partial sums: warps 0..3 of this group read the four lane
               // quarters of the accumulator
               tc_fence_after();
+              // (rank-major, rows contiguous: a thread holds one rank's kBN rows, and
+              // the reduce below reads consecutive rows with consecutive threads)
               if (a < 4) {
                 const int quarter = warp & 3;
-                float* dst = p.vpart + static_cast<size_t>(rb * S + sl) * kBN * kTileRows + quarter * 32 + lane;
+                float4* dst = reinterpret_cast<float4*>(p.vpart + static_cast<size_t>(rb * S + sl) * kBN * kTileRows +
+                                                        static_cast<size_t>(quarter * 32 + lane) * kBN);
 #pragma unroll
                 for (int c0 = 0; c0 < kBN; c0 += 16) {
                   uint32_t v[16];
                   tmem_ld16(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + L::kTmV + c0, v);
                   tmem_wait_ld();
 #pragma unroll
-                  for (int m = 0; m < 16; ++m)
-                    if (c0 + m < p.M) dst[(c0 + m) * kTileRows] = __uint_as_float(v[m]);
+                  for (int j = 0; j < 4; ++j)
+                    dst[c0 / 4 + j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                                                  __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
                 }
               }
               tc_fence_before();
@@ -1238,14 +1230,6 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
             if (tid == 0) {
               red_add_release_gpu(p.v_ready, 1u);             // covers the pieces the CTA wrote
               okv = spin_until_geq(p.v_ready, static_cast<uint32_t>(p.G), ctl);
-              if (okv) {
-                // the last CTA past the wait resets both counters for the next call
-                const uint32_t old = atomicAdd(p.v_seen, 1u);
-                if (old == static_cast<uint32_t>(p.G - 1)) {
-                  atomicExch(p.v_ready, 0u);
-                  atomicExch(p.v_seen, 0u);
-                }
-              }
             }
             if (named_barrier_or(kBarAlu, kAluThreads, !okv)) fail(ctl);
           }
@@ -1254,14 +1238,6 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
           if (tid == 0) {
             if (!(p.drop & 2)) red_add_release_gpu(p.q_ready, 1u);   // covers the items the CTA wrote
             okq = spin_until_geq(p.q_ready, static_cast<uint32_t>(p.G), ctl);
-            if (okq) {
-              // the last CTA past the wait resets both counters for the next call
-              const uint32_t old = atomicAdd(p.q_seen, 1u);
-              if (old == static_cast<uint32_t>(p.G - 1)) {
-                atomicExch(p.q_ready, 0u);
-                atomicExch(p.q_seen, 0u);
-              }
-            }
           }
           if (named_barrier_or(kBarAlu, kAluThreads, !okq)) fail(ctl);
           // one round of 16-byte loads: 144 per unit (128 of codes, 16 of scales)
@@ -1311,6 +1287,9 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
           constexpr int RPW = VS::kRows;
           for (int ig = i0; ig < i1; ig += kRankGroup) {
             const int nr = min(kRankGroup, i1 - ig);
+            // alpha of the (row, rank) this thread finishes below, requested with the
+            // V-side loads rather than after the reduction
+            const float al = (tid < p.M * nr) ? __ldcg(p.alpha + ig + tid % nr) : 0.0f;
             float acc[RPW][kRankGroup];
             vside_rows<MC>(p, ig, nr, a, lane, acc);
   #pragma unroll
@@ -1323,7 +1302,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
             // part in row m, the BF16 rounding of the rest in row MC + m, 128-byte
             // swizzled rows) or into the fp32 z scratch
             auto put = [&](int m, int i, float sum) {
-              const float zv = __fmul_rn(__ldcg(p.alpha + ig + i), sum);
+              const float zv = __fmul_rn(al, sum);
               if constexpr (Cfg<MC>::kTensorU) {
                 const __nv_bfloat16 hi = __float2bfloat16_rn(zv);
                 const __nv_bfloat16 lo = __float2bfloat16_rn(zv - __bfloat162float(hi));
@@ -1353,50 +1332,33 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
         }
       } else {
         // ---- V side, part 2: z for this CTA's rank slice [i0, i1), the pieces'
-        // partial sums added in a fixed order (four lanes per (rank, row) pair, each
-        // summing every fourth K slice, then an xor-shuffle tree), times alpha
+        // partial sums added in a fixed order (slice 0 first), times alpha.  One
+        // thread per (rank, row) with the rows of a rank on consecutive threads, so
+        // that each of a thread's S loads is part of one contiguous line per warp;
+        // all of them are requested before the first is added.
         const int RB = (p.r + kTileRows - 1) / kTileRows;
         const int S = vside_slices(p, RB);
-        constexpr int kParts = 4, kPerPart = kVSliceMax / kParts;
         const int P = (i1 - i0) * p.M;
-        // rounds of kAluThreads (rank, row, part) items, kRounds of them per pass with
-        // every request of the pass issued first (the partial sums and alpha): one
-        // memory round trip per pass instead of per round (at 32 rows a slice takes two)
-        constexpr int kRounds = (MC > 16) ? 2 : 1;
-        for (int base = 0; base < P * kParts; base += kRounds * kAluThreads) {
-          float t[kRounds][kPerPart], al[kRounds];
-          int iv[kRounds], mv[kRounds];
-          bool actv[kRounds];
+        for (int base = 0; base < P; base += kAluThreads) {
+          const int pair = base + tid;
+          const bool act = pair < P;
+          const int il = act ? pair / p.M : 0;
+          const int i = i0 + il, m = act ? pair - il * p.M : 0;
+          const float* src = p.vpart + static_cast<size_t>(i / kTileRows) * S * kBN * kTileRows +
+                             static_cast<size_t>(i % kTileRows) * kBN + m;
+          const float al = act ? __ldcg(p.alpha + i) : 0.0f;
+          float t[kVSliceMax];
 #pragma unroll
-          for (int e = 0; e < kRounds; ++e) {
-            const int idx = base + e * kAluThreads + tid, pair = idx >> 2, part = idx & 3;
-            const bool act = pair < P;
-            const int il = act ? pair / p.M : 0;
-            const int i = i0 + il, m = act ? pair - il * p.M : 0;
-            iv[e] = i;
-            mv[e] = m;
-            actv[e] = act && part == 0;
-            const float* src = p.vpart + (static_cast<size_t>(i / kTileRows) * S * kBN + m) * kTileRows + (i % kTileRows);
-            al[e] = (act && part == 0) ? __ldcg(p.alpha + i) : 0.0f;
+          for (int q = 0; q < kVSliceMax; ++q)
+            t[q] = (act && q < S) ? __ldcg(src + static_cast<size_t>(q) * kBN * kTileRows) : 0.0f;
+          float sum = 0.0f;
 #pragma unroll
-            for (int q = 0; q < kPerPart; ++q) {
-              const int sl = part + kParts * q;
-              t[e][q] = (act && sl < S) ? __ldcg(src + static_cast<size_t>(sl) * kBN * kTileRows) : 0.0f;
-            }
-          }
-#pragma unroll
-          for (int e = 0; e < kRounds; ++e) {
-            float sum = 0.0f;
-#pragma unroll
-            for (int q = 0; q < kPerPart; ++q) sum += t[e][q];
-            sum += __shfl_xor_sync(0xffffffffu, sum, 1);
-            sum += __shfl_xor_sync(0xffffffffu, sum, 2);
-            if (actv[e]) {
-              const float zv = __fmul_rn(al[e], sum);
-              const __nv_bfloat16 hi = __float2bfloat16_rn(zv);
-              const __nv_bfloat16 lo = __float2bfloat16_rn(zv - __bfloat162float(hi));
-              store_ztile(p.ztiles, Layout<MC>::kUN, MC, mv[e], iv[e], hi, lo);
-            }
+          for (int q = 0; q < kVSliceMax; ++q) sum += t[q];
+          if (act) {
+            const float zv = __fmul_rn(al, sum);
+            const __nv_bfloat16 hi = __float2bfloat16_rn(zv);
+            const __nv_bfloat16 lo = __float2bfloat16_rn(zv - __bfloat162float(hi));
+            store_ztile(p.ztiles, Layout<MC>::kUN, MC, m, i, hi, lo);
           }
         }
       }
@@ -1494,17 +1456,22 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
           named_barrier(kBarAlu, kAluThreads);
           zgroup = grp;
         };
+        // The product of segment seg goes to TMEM buffer seg & 1.  The two sides meet
+        // only through mbarriers (bounded waits): ud_bar(b) when a segment's MMAs are
+        // done (committed, also for an empty share), uread_bar(b) when the epilogue
+        // has read buffer b, which the next product of that buffer waits for.  So the
+        // share of a CTA's second tile runs while the epilogue still finishes its first.
         for (int seg = 0; seg < nseg; ++seg) {
-          // Every segment takes both barriers shared with the epilogue (kBarFin,
-          // kBarFin2), on every path: when either side has given up, the share is
-          // skipped (an empty one), and both sides leave together after kBarFin2.
-          const bool gone = named_barrier_or(kBarFin, kFinThreads, !ok);
-          if (gone) ok = false;
           const int t = t_first + seg;
+          const int ub_ = seg & 1;
           const int ua = max(u0, t * p.KC), ub = min(u1, (t + 1) * p.KC);
-          const int cs0 = gone ? 0 : (ua - t * p.KC) * nuc / p.KC;
-          const int cs1 = gone ? 0 : (ub - t * p.KC) * nuc / p.KC;
-          if (seg >= 2 && !gone) load_words(t_first + seg, uw1);    // segments past the second: load now
+          const int cs0 = (ua - t * p.KC) * nuc / p.KC;
+          const int cs1 = (ub - t * p.KC) * nuc / p.KC;
+          if (seg >= 2) load_words(t_first + seg, uw1);    // segments past the second: load now
+          if (seg >= 2 && tid == 0 && !mbar_wait(uread_bar(ub_), ((seg >> 1) - 1) & 1, abort_flag)) {
+            fail(ctl);
+            ok = false;
+          }
           // the classes whose slots hold every chunk stage z once, before their first
           // chunk; the 32-row class cycles larger ranks through its slots below
           if constexpr (Cfg<MC>::kZSlots >= kUChunksMax) {
@@ -1554,7 +1521,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
                       smem_desc(smem_u32(smem + L::kUZ + (c % Cfg<MC>::kZSlots) * L::kUN * 128), 16, 1024, 2);
   #pragma unroll
                   for (int j = 0; j < 4; ++j)
-                    tc_mma_bf16(tmem + L::kTmU, a_d + 2 * j, b_d + 2 * j, idesc_u, (c > cs0 || j > 0) ? 1u : 0u);
+                    tc_mma_bf16(tmem + L::kTmU + static_cast<uint32_t>(ub_ * L::kUN), a_d + 2 * j, b_d + 2 * j, idesc_u,
+                                (c > cs0 || j > 0) ? 1u : 0u);
                   tc_commit(ubuf_bar(buf));
                 } else {
                   fail(ctl);
@@ -1565,14 +1533,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
             }
           }
           }
-          if (tid == 0) {
-            fin_flag[seg] = (cs1 > cs0) ? 1 : 0;           // a share to add, in TMEM at kTmU
-            tc_commit(ud_bar);                             // arrives at once if nothing was issued
-          }
-          if (named_barrier_or(kBarFin2, kFinThreads, !ok)) {
-            ok = false;
-            break;
-          }
+          if (tid == 0) tc_commit(ud_bar(ub_));             // arrives at once if nothing was issued
         }
         // the U-side MMAs must be finished before TMEM is freed (bounded wait)
         if (tid == 0 && uses0 + uses1 > 0) {
@@ -1583,14 +1544,6 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
               record_error(p.status, kDevErrTimeout);
               break;
             }
-          }
-        }
-        // this CTA is done with z_ready; the last CTA to get here resets both counters
-        if (tid == 0 && ok) {
-          const uint32_t old = atomicAdd(p.z_seen, 1u);
-          if (old == static_cast<uint32_t>(p.G - 1)) {
-            atomicExch(p.z_ready, 0u);
-            atomicExch(p.z_seen, 0u);
           }
         }
       } else {
@@ -1666,13 +1619,24 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
             break;
           }
         }
-        // this CTA is done with z_ready; the last CTA to get here resets both counters
-        if (tid == 0 && ok) {
-          const uint32_t old = atomicAdd(p.z_seen, 1u);
-          if (old == static_cast<uint32_t>(p.G - 1)) {
-            atomicExch(p.z_ready, 0u);
-            atomicExch(p.z_seen, 0u);
-          }
+      }
+    }
+    // This CTA waits on no grid counter any more (in the streamed class its producer
+    // has passed the image wait too): count it done.  The last CTA resets every
+    // counter for the next call, which reads them only after its wait on this
+    // kernel.  Counted here, the atomic runs while the epilogue finishes, off its
+    // path; calls that use no counter (r = 0 below 8 rows) count nothing.
+    if (p.r > 0 || Cfg<MC>::kGlobalQ) {
+      if (tid == 0) {
+        if constexpr (kStream) {
+          if (!mbar_wait(qpass_bar, 0, abort_flag)) fail(ctl);
+        }
+        const uint32_t old = atomicAdd(p.done, 1u);
+        if (old == static_cast<uint32_t>(p.G - 1)) {
+          atomicExch(p.z_ready, 0u);
+          atomicExch(p.q_ready, 0u);
+          atomicExch(p.v_ready, 0u);
+          atomicExch(p.done, 0u);
         }
       }
     }

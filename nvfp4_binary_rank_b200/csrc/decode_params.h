@@ -20,12 +20,10 @@ struct DecodeParams {
   float* vpart;            // [G][16][128] scratch: V-side partial sums per piece (8+ rows)
   float* slots;            // [2 G][16][128] scratch: split-K partials
   uint32_t* z_ready;       // CTAs that published their z slice
-  uint32_t* z_seen;        // CTAs done with z_ready (the last one resets both)
+  uint32_t* done;          // CTAs that finished (the last one resets the grid counters)
   uint32_t* tickets;       // [T] split-K arrivals per weight tile
   uint32_t* q_ready;       // CTAs that published their part of the activation image
-  uint32_t* q_seen;        // CTAs done with q_ready (the last one resets both)
   uint32_t* v_ready;       // 32-row class: CTAs that published their V pieces' partial sums
-  uint32_t* v_seen;        // CTAs done with v_ready (the last one resets both)
   int* status;             // first device-side error
   int M, N, K, r;
   int KC, T, U, G, KW, RW, rpad;

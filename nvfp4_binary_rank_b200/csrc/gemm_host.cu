@@ -164,7 +164,7 @@ GemmPlan plan_gemm(const GemmArgs& a) {
     need.zpart = static_cast<size_t>(decode_ztile_bytes(M)) + vpieces * bn * kTileRows * 4;
     need.zfin = r ? static_cast<size_t>(M) * p.rpad * 4 : 16;
     need.slots = static_cast<size_t>(2 * p.G) * bn * kTileRows * 4;
-    need.counter_words = 6 + static_cast<size_t>(p.T);   // z, tickets, q and v counters
+    need.counter_words = 4 + static_cast<size_t>(p.T);   // z, done, tickets, q and v counters
     return p;
   }
   need.act_fp4 = p.inq ? 16 : static_cast<size_t>(M) * K / 2;
@@ -208,12 +208,10 @@ int launch_gemm(const GemmArgs& a, const GemmPlan& p, const Scratch& scr, cudaSt
     dp.vpart = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(sc->zpart) + decode_ztile_bytes(M));
     dp.slots = sc->slots;
     dp.z_ready = sc->counters;
-    dp.z_seen = sc->counters + 1;
+    dp.done = sc->counters + 1;
     dp.tickets = sc->counters + 2;
     dp.q_ready = sc->counters + 2 + T;
-    dp.q_seen = sc->counters + 3 + T;
-    dp.v_ready = sc->counters + 4 + T;
-    dp.v_seen = sc->counters + 5 + T;
+    dp.v_ready = sc->counters + 3 + T;
     dp.xq = sc->act_fp4;
     dp.status = sc->status;
     dp.M = M; dp.N = N; dp.K = K; dp.r = r;
