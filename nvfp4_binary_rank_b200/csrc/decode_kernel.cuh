@@ -175,7 +175,7 @@ struct Layout {
   static constexpr int kVRed = kUEnd;                                  // [8][MC * ranks] floats
   static constexpr int kVRedBytes = Cfg<MC>::kTensorV ? 0 : kAluWarps * MC * kRankGroup * 4;
   static constexpr int kBar = kVRed + kVRedBytes;
-  static constexpr int kNumBars = 2 * kStages + 17;
+  static constexpr int kNumBars = 2 * kStages + 18;
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kFinFlags = kMisc + 32;                         // [kMaxUnits + 1] ints
   static constexpr int kTotal = kFinFlags + (kMaxUnits + 1) * 4;
@@ -506,6 +506,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
   auto ud_bar = [&](int b) { return smem_u32(&bars[b ? 2 * kStages + 13 : 2 * kStages + 9]); };
   auto uread_bar = [&](int b) { return smem_u32(&bars[2 * kStages + 14 + b]); };
   const uint32_t qpass_bar = smem_u32(&bars[2 * kStages + 16]);   // streamed class: the producer passed the image wait
+  const uint32_t zst_bar = smem_u32(&bars[2 * kStages + 17]);     // the z tiles' bulk copies into the slots
   auto ufull_bar = [&](int b) { return smem_u32(&bars[2 * kStages + 10 + b]); };
   const uint32_t vmma_bar = smem_u32(&bars[2 * kStages + 12]);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMisc);
@@ -540,6 +541,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
     mbar_init(uread_bar(0), kEpiThreads);
     mbar_init(uread_bar(1), kEpiThreads);
     mbar_init(qpass_bar, 1);
+    mbar_init(zst_bar, 1);
     mbar_init(ufull_bar(0), kAluThreads);
     mbar_init(ufull_bar(1), kAluThreads);
     mbar_init(vmma_bar, 1);
@@ -1403,6 +1405,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
         if (nseg > 1) load_words(t_first + 1, uw1);
         bool ok = true, zwaited = false;
         int zgroup = -1;                                 // z chunks [zgroup S, zgroup S + S) are in the slots
+        int zstagings = 0;                               // thread 0: stagings done (zst_bar's phase)
         int uses0 = 0, uses1 = 0;                        // MMA rounds issued on each A buffer
         // wait (lane 0 of each warp) until the MMAs that last read A buffer `buf` are done
         auto buffer_free = [&](int buf, int uses) {
@@ -1435,25 +1438,30 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
             buffer_free(1, uses1);
             named_barrier(kBarAlu, kAluThreads);
           }
-          uint4* zt4 = reinterpret_cast<uint4*>(smem + L::kUZ);
-          const uint4* src = reinterpret_cast<const uint4*>(p.ztiles + static_cast<size_t>(grp) * S * L::kUN * 128);
-          constexpr int kZR = 8;
-          const int n16 = min(S, nuc - grp * S) * L::kUN * 8;
-          for (int base = 0; base < n16; base += kAluThreads * kZR) {
-            uint4 t4[kZR];
-#pragma unroll
-            for (int e = 0; e < kZR; ++e) {
-              const int idx = base + e * kAluThreads + tid;
-              t4[e] = (idx < n16) ? __ldcg(src + idx) : make_uint4(0u, 0u, 0u, 0u);
+          // thread 0 copies the chunks' tiles into the slots with bulk copies (the
+          // CTAs that computed z wrote them through the generic proxy) and waits for
+          // them: it alone reads the slots (its MMAs); the other threads go on to
+          // expand the chunk's signs meanwhile
+          if (tid == 0) {
+            constexpr uint32_t kChunkBytes = L::kUN * 128;
+            const int nch = min(S, nuc - grp * S);
+            fence_proxy_async_global();
+            mbar_arrive_expect_tx(zst_bar, static_cast<uint32_t>(nch) * kChunkBytes);
+            for (int c = 0; c < nch; ++c)
+              bulk_load(smem_u32(smem + L::kUZ + c * kChunkBytes),
+                        p.ztiles + static_cast<size_t>(grp * S + c) * kChunkBytes, kChunkBytes, zst_bar);
+            // (not cut short by an abort: the copies must land before anything else
+            // uses the slots or the CTA leaves)
+            const uint64_t t0 = globaltimer_ns();
+            while (!mbar_try_wait(zst_bar, zstagings & 1)) {
+              if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                fail(ctl);
+                ok = false;
+                break;
+              }
             }
-#pragma unroll
-            for (int e = 0; e < kZR; ++e) {
-              const int idx = base + e * kAluThreads + tid;
-              if (idx < n16) zt4[idx] = t4[e];
-            }
+            ++zstagings;
           }
-          fence_proxy_async_smem();
-          named_barrier(kBarAlu, kAluThreads);
           zgroup = grp;
         };
         // The product of segment seg goes to TMEM buffer seg & 1.  The two sides meet
