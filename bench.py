@@ -75,10 +75,10 @@ def kernel_source_digest() -> str:
 
 def ncu_traffic(workload: str, M: int):
     """DRAM bytes (read + write) per launch of the GEMM kernel that serves this
-    workload (decode_kernel for M <= 32, fused_kernel above), from the committed
-    ncu summary, or None when there is none or the kernel sources changed since
-    it was captured."""
-    kernel = "decode_kernel" if M <= 32 else "fused_kernel"
+    workload (decode_kernel for M <= 128 under the default schedule), from the
+    committed ncu summary, or None when there is none or the kernel sources changed
+    since it was captured."""
+    kernel = "decode_kernel" if M <= 128 else "fused_kernel"
     path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
     try:
         fields = {}

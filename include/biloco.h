@@ -182,9 +182,11 @@ int biloco_decompose(const float *W, int N, int K, int r, int T, const uint32_t 
  *   limits  1 <= M <= 128, N % 128 == 0, N <= 2^24, K % 64 == 0, 0 <= r <= 1024,
  *           (N/128) * ceil(K/256) <= 2^24
  * Accumulation is FP32 in an unspecified order; results are deterministic for a
- * fixed shape, mode and GPU.  Decode batches (M <= 32, shared-z schedule) run
- * one kernel that quantises the activation itself; otherwise an activation
- * quantiser runs first for M > 8 (biloco_gemm_kernel_count).
+ * fixed shape, mode and GPU.  Under the shared-z schedule, batches of up to 128
+ * rows run one kernel that quantises the activation itself when each CTA's share
+ * of the weight fits the batch class (ceil(units / G) <= 16 units of 128 x 256
+ * up to 16 rows, <= 64 above); otherwise an activation quantiser runs first for
+ * M > 8 (biloco_gemm_kernel_count).
  * The fused kernel is launched with programmatic dependent launch: it may start
  * while the kernel before it on the stream finishes, and it reads W_fp4 and
  * W_sf before waiting for that kernel (everything else after).  So the weight
@@ -224,11 +226,13 @@ int biloco_gemm(const void *x_bf16, const uint8_t *W_fp4, const uint8_t *W_sf,
  *   N <= BILOCO_NOALLOC_MAX_N, and the call's scratch fits the array.  That
  *   scratch is 16 896 bytes of status and counters plus, each rounded up to 256,
  *   with KC = ceil(K/256), G = min(#SMs, (N/128)*KC) and rpad = 16*ceil(r/16):
- *   decode-batch kernel (M <= 32, shared-z schedule, ceil(units/G) <= 16 for
- *   M <= 16 or <= 64 above; BN = 16 for M <= 16, else 32):
- *     KC * (M <= 16 ? 2304 : 6144)             (quantised activation image)
+ *   decode-batch kernel (M <= 128, shared-z schedule, ceil(units/G) <= 16 for
+ *   M <= 16 or <= 64 above; BN = 16 for M <= 16, else the batch class 32, 64
+ *   or 128 that holds M):
+ *     KC * (M <= 16 ? 2304 : BN * 128 + 2048)  (quantised activation image)
  *     ztile + max(G, ceil(r/128)) * BN * 512   (z tiles, V-side partial sums;
- *                                               ztile = 65536 or 131072)
+ *                                               ztile = 65536 for M <= 16,
+ *                                               else 4096 * BN)
  *     M * rpad * 4                             (z)
  *     2 * G * BN * 512                         (split-K partials)
  *   general kernel (every other shape; BN = 16, 32, 64, 128 for M <= 16, 32,
@@ -236,8 +240,8 @@ int biloco_gemm(const void *x_bf16, const uint8_t *W_fp4, const uint8_t *W_sf,
  *     M > 8:  M*K/2 + KC*2048                  (quantised activation)
  *     r > 0:  (KC + 1) * M * rpad * 4          (z partials and z)
  *     always: 2 * G * BN * 512                 (split-K partials)
- *   On a 148-SM B200 every M <= 32 shape with K <= 13824 and r <= 1024 fits;
- *   M > 64 fits only tiny weights.
+ *   On a 148-SM B200 every M <= 64 shape with K <= 13824 and r <= 1024 fits;
+ *   M > 64 fits only small weights (few units, so a small G).
  * Caveats:
  *   - There is one array per device, shared by all streams and host threads:
  *     calls that overlap in time (on different streams, or from several threads
@@ -338,7 +342,7 @@ const char *biloco_status_string(int status);
 
 /* Number of kernels biloco_gemm would launch per call for this shape under the
  * current schedule setting: 1 when the GEMM kernel quantises the activation
- * itself (the decode-batch kernel, M <= 32, or the general kernel at M <= 8),
+ * itself (the decode-batch kernel, M <= 128, or the general kernel at M <= 8),
  * else 2 (quantiser + GEMM).  BILOCO_ERR_SHAPE for shapes biloco_gemm rejects.
  * Uses the device's SM count (the current device must be set). */
 int biloco_gemm_kernel_count(int M, int N, int K, int r);

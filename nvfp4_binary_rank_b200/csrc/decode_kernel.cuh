@@ -1,5 +1,5 @@
-// Fused NVFP4 GEMM + binary-sign low-rank correction for decode batches
-// (M <= 16 activation rows) on one B200 (sm_100a).
+// Fused NVFP4 GEMM + binary-sign low-rank correction for batches of up to 128
+// activation rows (decode and small prefill batches) on one B200 (sm_100a).
 //
 //   y[m, n] = g * sum_k FP4(x)[m, k] FP4(R)[n, k]  +  sum_i U[n, i] z[m, i],
 //   z[m, i] = alpha_i * sum_k V[k, i] x[m, k]
@@ -14,15 +14,17 @@
 // stream, which is what bounds a decode call:
 //   * Weight stages are requested before that wait: no kernel of this library
 //     writes the weight operand.
-//   * The activation chunks of all the CTA's units land at once in an operand
-//     cache in shared memory: below 8 rows quantised by the CTA itself, from 8
-//     rows up copied from an image the CTAs quantise once between them.  The MMAs
-//     read the activation from there, so the stage ring carries weight bytes only.
+//   * Up to 16 rows the activation chunks of all the CTA's units land at once in
+//     an operand cache in shared memory: below 8 rows quantised by the CTA itself,
+//     from 8 rows up copied from an image the CTAs quantise once between them.
+//     The MMAs read the activation from there, so the stage ring carries weight
+//     bytes only.  The classes of 32, 64 and 128 rows (MMA N = 32, 64, 128) stream
+//     each unit's activation chunk from that image with its weight stage.
 //   * z is computed in rank slices: CTA g < Z computes z for the ranks
 //     [g r / Z, (g + 1) r / Z) and publishes them behind one arrival counter
 //     (Z = G - 2 on large grids, see shared_work_ctas).  This is the "side CTAs +
 //     arrival flag" schedule of the README's mode table.  Below 16 rows the slice
-//     is summed over the whole of K on the CUDA cores; with 16, V^T x runs on the
+//     is summed over the whole of K on the CUDA cores; from 16, V^T x runs on the
 //     tensor cores in pieces of 128 ranks x a K slice whose partial sums the slice
 //     owners add up.
 //   * U z: from 4 rows up (tensor-core U side) every contributor of a weight tile
@@ -65,7 +67,7 @@ constexpr int kAluWarp0 = 6;
 constexpr int kAluWarps = 8;
 constexpr int kAluThreads = kAluWarps * 32;
 constexpr int kFinThreads = kEpiThreads + kAluThreads;
-constexpr int kRowsMax = 32;              // activation rows handled (the largest class)
+constexpr int kRowsMax = 128;             // activation rows handled (the largest class)
 constexpr int kTileRows = 128;            // weight rows per tile = MMA M
 constexpr int kUnitK = 256;               // K elements per unit
 constexpr int kUnitBytesA = kTileRows * 128;
@@ -90,14 +92,14 @@ constexpr int kBarZ = 5;                  // epilogue + CUDA cores: z staged (1-
 template <int MC>
 struct Cfg {
   // Up to 16 rows the activation chunks of all of a CTA's units sit in an operand
-  // cache in shared memory (at most kMaxUnits units per CTA).  The 32-row class
-  // streams them instead: each stage carries one weight unit and the matching
-  // activation chunk (codes and scale atoms) from the grid's activation image,
-  // and both sets of block scales go to TMEM per stage.
+  // cache in shared memory (at most kMaxUnits units per CTA).  From 32 rows the
+  // classes stream them instead: each stage carries one weight unit and the
+  // matching activation chunk (codes and scale atoms) from the grid's activation
+  // image, and both sets of block scales go to TMEM per stage.
   static constexpr bool kStream = MC > 16;
-  static constexpr int kBN = kStream ? 32 : 16;            // MMA N (activation rows, padded)
+  static constexpr int kBN = kStream ? MC : 16;            // MMA N (activation rows, padded)
   static constexpr int kMaxUnits = kStream ? 64 : 16;      // units per CTA
-  static constexpr int kStages = kStream ? 5 : ((MC >= 16) ? 4 : 6);
+  static constexpr int kStages = kStream ? (MC >= 128 ? 3 : 5) : ((MC >= 16) ? 4 : 6);
   static constexpr int kRankGroup = 4;                     // ranks per V-side pass
   // V-side load ring depth (blocks in flight per warp); below 8 rows a warp walks
   // only two or three K blocks
@@ -118,19 +120,30 @@ struct Cfg {
   // x a slice of K, with the partial sums reduced across CTAs (with 8 the CUDA-core
   // loop is faster, measured on B200)
   static constexpr bool kTensorV = MC >= 16;
+  // The U side's product: up to 32 rows the high and low BF16 parts of z go to
+  // separate TMEM columns (one MMA of N = 2 MC per K step, added by the epilogue);
+  // from 64 rows both parts accumulate into the same MC columns (two MMAs of N = MC),
+  // which halves the product's tensor memory.  The 128-row class keeps one product
+  // buffer (its accumulators take half of TMEM), the others two.
+  static constexpr bool kUSum = MC >= 64;
+  static constexpr int kUBufs = MC >= 128 ? 1 : 2;
   // z tiles of the tensor-core U side held in shared memory at once (64 ranks
-  // each); the 32-row class cycles larger ranks through them
-  static constexpr int kZSlots = kStream ? 8 : 16;
+  // each); the streamed classes cycle larger ranks through them
+  static constexpr int kZSlots = !kStream ? 16 : (MC <= 32 ? 8 : (MC <= 64 ? 3 : 2));
+  // from 64 rows the epilogue reads the accumulator and the U-side product 16
+  // columns at a time (a thread cannot hold a whole row of either)
+  static constexpr bool kChunkedEpi = MC > 32;
 };
 
 // Global activation image (8+ rows), per 256-element K chunk:
 //  * classes 8 and 16: the 16 x 128 B code rows exactly as the operand cache holds
 //    them (128-byte swizzle), then 256 B of block scales, 64 B per 64-element K
 //    step (row m at byte 4 m, block b of the step at byte b);
-//  * class 32: the 32 x 128 B code rows (128-byte swizzle), then the block scales
-//    as four 512-byte scale atoms, one per K step, in the layout the tensor
-//    memory copy expects (row m's four scales at bytes 16 m .. 16 m + 3, the other
-//    12 bytes of the row zero).  A stage's activation part is one bulk copy of it.
+//  * classes 32, 64, 128: the MC x 128 B code rows (128-byte swizzle), then the
+//    block scales as four 512-byte scale atoms, one per K step, in the layout the
+//    tensor memory copy expects: 32 lines of 16 bytes, row m's four scales at
+//    bytes 16 (m % 32) + 4 (m / 32) .. + 3 (bytes no row of the class uses are
+//    zero).  A stage's activation part is one bulk copy of it.
 template <int MC>
 struct QImg {
   static constexpr int kCodes = Cfg<MC>::kBN * 128;
@@ -182,14 +195,18 @@ struct Layout {
   static constexpr int kAlloc = kTotal + 1024;
   // TMEM columns.  Cache classes: accumulators [0, 32), activation scales per unit
   // [32, 288), weight scales per stage [288, 384), the two U-side product buffers
-  // [384, 384 + 2 kUN), the V-side product [448, 464).  Streamed class:
-  // accumulators [0, 64), weight and activation scales per stage, then the two
-  // U-side product buffers (2 x 64) and the V-side product (32).
+  // [384, 384 + 2 kUN), the V-side product [448, 464).  Streamed classes:
+  // accumulators [0, 2 MC), weight and activation scales per stage, then the U-side
+  // product buffers (kUBufs x kUCols) and the V-side product (MC columns; from 64
+  // rows it shares the first U-side buffer: the V pieces are read out before this
+  // CTA's z exists, and no U-side MMA runs before z does).
+  static constexpr int kUCols = Cfg<MC>::kUSum ? MC : kUN;             // columns per U-side buffer
   static constexpr int kTmSfb = kStream ? 2 * kBN + kStages * 16 : 32;
   static constexpr int kTmSfa = kStream ? 2 * kBN : kTmSfb + kMaxUnits * 16;
-  static constexpr int kTmU = kStream ? kTmSfb + kStages * 16 : 384;   // two buffers of kUN columns
-  static constexpr int kTmV = kStream ? kTmU + 2 * kUN : 448;
-  static_assert(!Cfg<MC>::kTensorU || kTmU + 2 * kUN <= kTmV, "two U-side product buffers");
+  static constexpr int kTmU = kStream ? kTmSfb + kStages * 16 : 384;
+  static constexpr int kTmV = kStream ? (Cfg<MC>::kUSum ? kTmU : kTmU + Cfg<MC>::kUBufs * kUCols) : 448;
+  static_assert(!Cfg<MC>::kTensorU || kTmU + Cfg<MC>::kUBufs * kUCols <= (Cfg<MC>::kUSum ? kTmemCols : kTmV),
+                "U-side product buffers");
   static_assert(kTmV + kBN <= kTmemCols, "tensor memory budget");
   static_assert(kStream || kTmSfa + kStages * 16 <= kTmU, "tensor memory budget");
   static_assert(kSFA % 1024 == 0 && kB % 1024 == 0 && kUA % 1024 == 0 && kUZ % 1024 == 0 &&
@@ -657,14 +674,14 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
       // cache classes: stage s at kA + s 16 KB (codes) and kSFA + s 2 KB (scales),
       // activation unit k in the operand cache; streamed class: everything in
       // stage s at s * kStageBytes
-      const uint64_t a_desc0 = smem_desc(smem_u32(smem + (kStream ? L::kStageA : L::kA)), 16, 1024, 2);
-      const uint64_t b_desc0 = smem_desc(smem_u32(smem + (kStream ? L::kStageB : L::kB)), 16, 1024, 2);
-      const uint64_t sfa_desc0 = smem_desc(smem_u32(smem + (kStream ? L::kStageSFA : L::kSFA)), 0, 128, 0);
-      const uint64_t sfb_desc0 = smem_desc(smem_u32(smem + L::kStageSFB), 0, 128, 0);
-      constexpr uint64_t kAtom = 512 >> 4;
-      constexpr uint64_t kUnitSf = (kStream ? L::kStageBytes : kSfBytes) >> 4;
-      constexpr uint64_t kUnitA = (kStream ? L::kStageBytes : kUnitBytesA) >> 4;
-      constexpr uint64_t kUnitB = (kBN * 128) >> 4, kStageB = L::kStageBytes >> 4;
+      const SmemDesc a_desc0 = make_sdesc(smem_u32(smem + (kStream ? L::kStageA : L::kA)), 16, 1024, 2);
+      const SmemDesc b_desc0 = make_sdesc(smem_u32(smem + (kStream ? L::kStageB : L::kB)), 16, 1024, 2);
+      const SmemDesc sfa_desc0 = make_sdesc(smem_u32(smem + (kStream ? L::kStageSFA : L::kSFA)), 0, 128, 0);
+      const SmemDesc sfb_desc0 = make_sdesc(smem_u32(smem + L::kStageSFB), 0, 128, 0);
+      constexpr uint32_t kAtom = 512 >> 4;
+      constexpr uint32_t kUnitSf = (kStream ? L::kStageBytes : kSfBytes) >> 4;
+      constexpr uint32_t kUnitA = (kStream ? L::kStageBytes : kUnitBytesA) >> 4;
+      constexpr uint32_t kUnitB = (kBN * 128) >> 4, kStageB = L::kStageBytes >> 4;
       // cache classes: the weight scales of the stages already requested go to
       // TMEM while the activation is still being quantised
       const int pre = kStream ? 0 : min(nunits, kStages);
@@ -676,10 +693,10 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
           break;
         }
         tc_fence_after();
-        const uint64_t sfa_d = sfa_desc0 + static_cast<uint64_t>(j) * kUnitSf;
+        const SmemDesc sfa_d = sdesc_at(sfa_desc0, static_cast<uint32_t>(j) * kUnitSf);
 #pragma unroll
         for (int q = 0; q < 4; ++q)
-          tc_cp_32x128b_warpx4(tmem + L::kTmSfa + j * 16 + 4 * q, sfa_d + kAtom * q);
+          tc_cp_32x128b_warpx4(tmem + L::kTmSfa + j * 16 + 4 * q, sdesc_at(sfa_d, kAtom * q));
       }
       // the activation codes (shared memory) and scales (TMEM) are in place
       if (!kStream && ok && !mbar_wait(actr_bar, 0, abort_flag)) {
@@ -710,21 +727,21 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
               break;
             }
             tc_fence_after();
-            const uint64_t sfa_d = sfa_desc0 + static_cast<uint64_t>(s) * kUnitSf;
+            const SmemDesc sfa_d = sdesc_at(sfa_desc0, static_cast<uint32_t>(s) * kUnitSf);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) tc_cp_32x128b_warpx4(sfa_t + 4 * q, sfa_d + kAtom * q);
+            for (int q = 0; q < 4; ++q) tc_cp_32x128b_warpx4(sfa_t + 4 * q, sdesc_at(sfa_d, kAtom * q));
             if constexpr (kStream) {
-              const uint64_t sfb_d = sfb_desc0 + static_cast<uint64_t>(s) * kStageB;
+              const SmemDesc sfb_d = sdesc_at(sfb_desc0, static_cast<uint32_t>(s) * kStageB);
 #pragma unroll
-              for (int q = 0; q < 4; ++q) tc_cp_32x128b_warpx4(sfb_t + 4 * q, sfb_d + kAtom * q);
+              for (int q = 0; q < 4; ++q) tc_cp_32x128b_warpx4(sfb_t + 4 * q, sdesc_at(sfb_d, kAtom * q));
             }
           }
-          const uint64_t a_d = a_desc0 + static_cast<uint64_t>(s) * kUnitA;
-          const uint64_t b_d = kStream ? b_desc0 + static_cast<uint64_t>(s) * kStageB
-                                       : b_desc0 + static_cast<uint64_t>(k) * kUnitB;
+          const SmemDesc a_d = sdesc_at(a_desc0, static_cast<uint32_t>(s) * kUnitA);
+          const SmemDesc b_d = kStream ? sdesc_at(b_desc0, static_cast<uint32_t>(s) * kStageB)
+                                       : sdesc_at(b_desc0, static_cast<uint32_t>(k) * kUnitB);
 #pragma unroll
           for (int j = 0; j < 4; ++j)
-            tc_mma_nvf4(d_tmem, a_d + 2 * j, b_d + 2 * j, idesc, sfa_t + 4 * j, sfb_t + 4 * j,
+            tc_mma_nvf4(d_tmem, sdesc_at(a_d, 2 * j), sdesc_at(b_d, 2 * j), idesc, sfa_t + 4 * j, sfb_t + 4 * j,
                         (u > ua || j > 0) ? 1u : 0u);
           tc_commit(empty_bar(s));
           if (++s == kStages) { s = 0; ph ^= 1u; }
@@ -756,13 +773,109 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
       for (int c0 = 0; c0 < MC; c0 += 16) {
         uint32_t raw[16];
         tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(b * kBN + c0), raw);
-        tmem_wait_ld();
 #pragma unroll
         for (int j = 0; j < 16; ++j)
           if (c0 + j < MC) v[c0 + j] = __fmul_rn(gs, __uint_as_float(raw[j]));
       }
     };
-    if constexpr (Cfg<MC>::kUShares) {
+    if constexpr (Cfg<MC>::kChunkedEpi) {
+      // 64+ rows: once the segment's FP4 product and (r > 0) this CTA's share of U z
+      // are both in TMEM, read them 16 columns at a time; a sole owner stores y
+      // directly, a split-K contributor publishes its partial and the last one to
+      // arrive sums every contributor's partial (its own included) from the slots
+      constexpr int kUB = Cfg<MC>::kUBufs;
+      bool ok = true;
+      for (int seg = 0; seg < nseg; ++seg) {
+        const int t = t_first + seg;
+        const int b = seg & 1, ubf = seg % kUB;
+        const int hf = owner_cta(static_cast<uint32_t>(t * p.KC), p.G, p.U);
+        const int hl = owner_cta(static_cast<uint32_t>((t + 1) * p.KC - 1), p.G, p.U);
+        const bool sole = hf == hl;
+        const int which = (t == t_first) ? 0 : 1;
+        const int nuc = (p.r + kUChunk - 1) / kUChunk;
+        const int ua = max(u0, t * p.KC), ub = min(u1, (t + 1) * p.KC);
+        const bool addu = p.r > 0 && (ub - t * p.KC) * nuc / p.KC > (ua - t * p.KC) * nuc / p.KC;
+        if (ok) ok = group_wait(accf_bar(b), (seg >> 1) & 1, kBarEpi, kEpiThreads, ctl);
+        if (ok && p.r > 0) ok = group_wait(ud_bar(ubf), (seg / kUB) & 1, kBarEpi, kEpiThreads, ctl);
+        uint16_t* yb = p.y + static_cast<size_t>(t) * kTileRows + row;
+        float* my_slot = p.slots + static_cast<size_t>(2 * g + which) * kBN * kTileRows;
+        if (ok) {
+          tc_fence_after();
+          const uint32_t lane_base = tmem + (static_cast<uint32_t>(q * 32) << 16);
+  #pragma unroll 1
+          for (int c0 = 0; c0 < MC; c0 += 16) {
+            uint32_t ra[16], ru[16];
+            if (addu) {
+              tmem_ld16x2(lane_base + static_cast<uint32_t>(b * kBN + c0), ra,
+                          lane_base + L::kTmU + static_cast<uint32_t>(ubf * L::kUCols + c0), ru);
+            } else {
+              tmem_ld16(lane_base + static_cast<uint32_t>(b * kBN + c0), ra);
+            }
+  #pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              float v = __fmul_rn(gs, __uint_as_float(ra[j]));
+              if (addu) v += __uint_as_float(ru[j]);
+              if (c0 + j < p.M) {
+                if (sole) yb[static_cast<size_t>(c0 + j) * p.N] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+                else my_slot[(c0 + j) * kTileRows + row] = v;
+              }
+            }
+          }
+          tc_fence_before();
+          mbar_arrive(acce_bar(b));
+        }
+        // the U-side buffer may take its next product (arrived on every path, so
+        // that the phases stay in step)
+        if (p.r > 0) {
+          tc_fence_before();
+          mbar_arrive(uread_bar(ubf));
+        }
+        if (!ok) break;
+        if (sole) continue;
+        named_barrier(kBarEpi, kEpiThreads);
+        if (etid == 0) {
+          // release: this CTA's partial; acquire: every earlier contributor's
+          const uint32_t nh = static_cast<uint32_t>(hl - hf + 1);
+          const uint32_t old = atom_add_acq_rel_gpu(p.tickets + t, 1u);
+          const bool last = old == nh - 1;
+          if (last) atomicExch(p.tickets + t, 0u);
+          *epi_last = last ? 1 : 0;
+        }
+        named_barrier(kBarEpi, kEpiThreads);
+        const bool fin = *epi_last != 0;
+        named_barrier(kBarEpi, kEpiThreads);
+        if (!fin) continue;
+        // every contributor's partial, summed in contributor order, 16 rows at a
+        // time, two contributors per batch of loads
+        const int wh_first = (t == first_unit(hf, p.G, p.U) / p.KC) ? 0 : 1;
+  #pragma unroll 1
+        for (int j0 = 0; j0 < MC && j0 < p.M; j0 += 16) {
+          float acc[16];
+  #pragma unroll
+          for (int jj = 0; jj < 16; ++jj) acc[jj] = 0.0f;
+          for (int h0 = hf; h0 <= hl; h0 += 2) {
+            float part[2][16];
+  #pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int h = h0 + e;
+              const float* sl = p.slots + static_cast<size_t>(2 * h + ((h == hf) ? wh_first : 0)) * kBN * kTileRows;
+  #pragma unroll
+              for (int jj = 0; jj < 16; ++jj)
+                part[e][jj] = (h <= hl && j0 + jj < p.M) ? __ldcg(sl + (j0 + jj) * kTileRows + row) : 0.0f;
+            }
+  #pragma unroll
+            for (int e = 0; e < 2; ++e)
+              if (h0 + e <= hl) {
+  #pragma unroll
+                for (int jj = 0; jj < 16; ++jj) acc[jj] += part[e][jj];
+              }
+          }
+  #pragma unroll
+          for (int jj = 0; jj < 16; ++jj)
+            if (j0 + jj < p.M) yb[static_cast<size_t>(j0 + jj) * p.N] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[jj]));
+        }
+      }
+    } else if constexpr (Cfg<MC>::kUShares) {
       bool ok = true;
       for (int seg = 0; seg < nseg; ++seg) {
         const int t = t_first + seg;
@@ -793,12 +906,13 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
               tc_fence_after();
               const uint32_t ucol = L::kTmU + static_cast<uint32_t>(b * L::kUN);
               if constexpr (L::kUN <= 32) {
-                uint32_t du[L::kUN];
-                tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + ucol, *reinterpret_cast<uint32_t(*)[16]>(du));
+                uint32_t du[32];
                 if constexpr (L::kUN > 16)
-                  tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + ucol + 16,
-                            *reinterpret_cast<uint32_t(*)[16]>(du + 16));
-                tmem_wait_ld();
+                  tmem_ld16x2(tmem + (static_cast<uint32_t>(q * 32) << 16) + ucol, *reinterpret_cast<uint32_t(*)[16]>(du),
+                              tmem + (static_cast<uint32_t>(q * 32) << 16) + ucol + 16,
+                              *reinterpret_cast<uint32_t(*)[16]>(du + 16));
+                else
+                  tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + ucol, *reinterpret_cast<uint32_t(*)[16]>(du));
     #pragma unroll
                 for (int j = 0; j < MC; ++j) v[j] += __uint_as_float(du[j]) + __uint_as_float(du[MC + j]);
               } else {
@@ -806,9 +920,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
     #pragma unroll
                 for (int c0 = 0; c0 < MC; c0 += 16) {
                   uint32_t hi[16], lo[16];
-                  tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + ucol + c0, hi);
-                  tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + ucol + MC + c0, lo);
-                  tmem_wait_ld();
+                  tmem_ld16x2(tmem + (static_cast<uint32_t>(q * 32) << 16) + ucol + c0, hi,
+                              tmem + (static_cast<uint32_t>(q * 32) << 16) + ucol + MC + c0, lo);
     #pragma unroll
                   for (int j = 0; j < 16; ++j) v[c0 + j] += __uint_as_float(hi[j]) + __uint_as_float(lo[j]);
                 }
@@ -1066,17 +1179,21 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
             img[kImgCodes + (blk >> 2) * 64 + m * 4 + (blk & 3)] = static_cast<uint8_t>(sc);
           }
         } else {
-          // Streamed class: items of (chunk, row, 64-element K step), I = 128 KC of
-          // them, CTA g < Z taking [g I / Z, (g + 1) I / Z).  An item is four blocks:
-          // 32 code bytes (two 16-byte pieces of the swizzled row) and the row's line
-          // of the step's scale atom (four scales, twelve zero bytes).  Rows >= M and
+          // Streamed classes: items of (chunk, row, 64-element K step), I = 4 kBN KC
+          // of them, CTA g < Z taking [g I / Z, (g + 1) I / Z).  An item is four
+          // blocks: 32 code bytes (two 16-byte pieces of the swizzled row) and the
+          // row's four scales in the step's scale atom (the 32-row class writes the
+          // whole 16-byte line, twelve bytes of it zero; at 64 rows the rows below 32
+          // zero the line's last eight bytes, which no row uses).  Rows >= M and
           // steps past K are written as zeros.
-          const uint32_t items = static_cast<uint32_t>(p.KC) * 128u;
+          constexpr uint32_t kItemsPerChunk = 4u * kBN;
+          const uint32_t items = static_cast<uint32_t>(p.KC) * kItemsPerChunk;
           const uint32_t q0 = g < zg ? static_cast<uint32_t>(static_cast<uint64_t>(g) * items / static_cast<uint32_t>(zg)) : 0u;
           const uint32_t q1 = g < zg ? static_cast<uint32_t>(static_cast<uint64_t>(g + 1) * items / static_cast<uint32_t>(zg)) : 0u;
 #pragma unroll 1
           for (uint32_t it = q0 + static_cast<uint32_t>(tid); it < q1; it += kAluThreads) {
-            const int kc = static_cast<int>(it >> 7), m = static_cast<int>((it >> 2) & 31u), st = static_cast<int>(it & 3u);
+            const int kc = static_cast<int>(it / kItemsPerChunk);
+            const int m = static_cast<int>((it >> 2) & static_cast<uint32_t>(kBN - 1)), st = static_cast<int>(it & 3u);
             const int kk = kc * kUnitK + st * 64;
             const bool live = m < p.M && kk < p.K;
             uint4 xv[8];
@@ -1099,7 +1216,15 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
             // elements 64 st .. 64 st + 63 = bytes 32 st .. 32 st + 31 of the row: pieces 2 st, 2 st + 1
             *reinterpret_cast<uint4*>(img + m * 128 + (((2 * st) ^ (m & 7)) << 4)) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
             *reinterpret_cast<uint4*>(img + m * 128 + (((2 * st + 1) ^ (m & 7)) << 4)) = make_uint4(cw[4], cw[5], cw[6], cw[7]);
-            *reinterpret_cast<uint4*>(img + kImgCodes + st * 512 + m * 16) = make_uint4(sc4, 0u, 0u, 0u);
+            uint8_t* line = img + kImgCodes + st * 512 + (m & 31) * 16;
+            if constexpr (kBN == 32) {
+              *reinterpret_cast<uint4*>(line) = make_uint4(sc4, 0u, 0u, 0u);
+            } else {
+              *reinterpret_cast<uint32_t*>(line + 4 * (m >> 5)) = sc4;
+              if constexpr (kBN == 64) {
+                if (m < 32) *reinterpret_cast<uint2*>(line + 8) = make_uint2(0u, 0u);
+              }
+            }
           }
           // the producers read the image with bulk copies (the async proxy); this
           // CTA's part is published at once, ahead of the V pieces
@@ -1184,13 +1309,13 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
                 bool okv = true;
                 if (tid == 0) {
                   tc_fence_after();
-                  const uint64_t a_d = smem_desc(smem_u32(va), 16, 1024, 2);
-                  const uint64_t b_d = smem_desc(smem_u32(vbt), 16, 1024, 2);
+                  const SmemDesc a_d = make_sdesc(smem_u32(va), 16, 1024, 2);
+                  const SmemDesc b_d = make_sdesc(smem_u32(vbt), 16, 1024, 2);
                   for (int j = 0; j < nb; ++j)
 #pragma unroll
                     for (int k4 = 0; k4 < 4; ++k4)
-                      tc_mma_bf16(tmem + L::kTmV, a_d + static_cast<uint64_t>(j) * ((kTileRows * 128) >> 4) + 2 * k4,
-                                  b_d + static_cast<uint64_t>(j) * ((kBN * 128) >> 4) + 2 * k4, idesc_v,
+                      tc_mma_bf16(tmem + L::kTmV, sdesc_at(a_d, static_cast<uint32_t>(j) * ((kTileRows * 128) >> 4) + 2 * k4),
+                                  sdesc_at(b_d, static_cast<uint32_t>(j) * ((kBN * 128) >> 4) + 2 * k4), idesc_v,
                                   (b0 > a0 || j > 0 || k4 > 0) ? 1u : 0u);
                   tc_commit(vmma_bar);
                   okv = mbar_wait(vmma_bar, vuses & 1, abort_flag);
@@ -1211,7 +1336,6 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
                 for (int c0 = 0; c0 < kBN; c0 += 16) {
                   uint32_t v[16];
                   tmem_ld16(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + L::kTmV + c0, v);
-                  tmem_wait_ld();
 #pragma unroll
                   for (int j = 0; j < 4; ++j)
                     dst[c0 / 4 + j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
@@ -1389,8 +1513,9 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
         const int nuc = (p.r + kUChunk - 1) / kUChunk;
         const int row = tid & (kTileRows - 1), half = tid >> 7;
         const uint32_t idesc_u = (1u << 4) | (1u << 7) | (1u << 10) |
-                                 (static_cast<uint32_t>(L::kUN >> 3) << 17) |
+                                 (static_cast<uint32_t>(L::kUCols >> 3) << 17) |
                                  (static_cast<uint32_t>(kTileRows >> 4) << 24);
+        constexpr int kUB = Cfg<MC>::kUBufs;
         // this thread expands word 2 c + half of row `row` for chunk c
         auto load_words = [&](int t, uint32_t (&uw)[kUChunksMax]) {
           const uint32_t* ur = p.Ubits + (static_cast<size_t>(t) * kTileRows + row) * p.RW;
@@ -1464,19 +1589,20 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
           }
           zgroup = grp;
         };
-        // The product of segment seg goes to TMEM buffer seg & 1.  The two sides meet
-        // only through mbarriers (bounded waits): ud_bar(b) when a segment's MMAs are
-        // done (committed, also for an empty share), uread_bar(b) when the epilogue
-        // has read buffer b, which the next product of that buffer waits for.  So the
-        // share of a CTA's second tile runs while the epilogue still finishes its first.
+        // The product of segment seg goes to TMEM buffer seg % kUB.  The two sides
+        // meet only through mbarriers (bounded waits): ud_bar(b) when a segment's MMAs
+        // are done (committed, also for an empty share), uread_bar(b) when the
+        // epilogue has read buffer b, which the next product of that buffer waits
+        // for.  With two buffers the share of a CTA's second tile runs while the
+        // epilogue still finishes its first.
         for (int seg = 0; seg < nseg; ++seg) {
           const int t = t_first + seg;
-          const int ub_ = seg & 1;
+          const int ub_ = seg % kUB;
           const int ua = max(u0, t * p.KC), ub = min(u1, (t + 1) * p.KC);
           const int cs0 = (ua - t * p.KC) * nuc / p.KC;
           const int cs1 = (ub - t * p.KC) * nuc / p.KC;
           if (seg >= 2) load_words(t_first + seg, uw1);    // segments past the second: load now
-          if (seg >= 2 && tid == 0 && !mbar_wait(uread_bar(ub_), ((seg >> 1) - 1) & 1, abort_flag)) {
+          if (seg >= kUB && tid == 0 && !mbar_wait(uread_bar(ub_), ((seg / kUB) - 1) & 1, abort_flag)) {
             fail(ctl);
             ok = false;
           }
@@ -1524,13 +1650,17 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
               if (tid == 0) {
                 if (mbar_wait(ufull_bar(buf), uses & 1, abort_flag)) {
                   tc_fence_after();
-                  const uint64_t a_d = smem_desc(smem_u32(smem + L::kUA + buf * (kTileRows * 128)), 16, 1024, 2);
-                  const uint64_t b_d =
-                      smem_desc(smem_u32(smem + L::kUZ + (c % Cfg<MC>::kZSlots) * L::kUN * 128), 16, 1024, 2);
+                  const SmemDesc a_d = make_sdesc(smem_u32(smem + L::kUA + buf * (kTileRows * 128)), 16, 1024, 2);
+                  const SmemDesc b_d =
+                      make_sdesc(smem_u32(smem + L::kUZ + (c % Cfg<MC>::kZSlots) * L::kUN * 128), 16, 1024, 2);
+                  const uint32_t d_u = tmem + L::kTmU + static_cast<uint32_t>(ub_ * L::kUCols);
   #pragma unroll
-                  for (int j = 0; j < 4; ++j)
-                    tc_mma_bf16(tmem + L::kTmU + static_cast<uint32_t>(ub_ * L::kUN), a_d + 2 * j, b_d + 2 * j, idesc_u,
-                                (c > cs0 || j > 0) ? 1u : 0u);
+                  for (int j = 0; j < 4; ++j) {
+                    tc_mma_bf16(d_u, sdesc_at(a_d, 2 * j), sdesc_at(b_d, 2 * j), idesc_u, (c > cs0 || j > 0) ? 1u : 0u);
+                    // the low parts (rows MC .. 2 MC - 1 of the tile) into the same columns
+                    if constexpr (Cfg<MC>::kUSum)
+                      tc_mma_bf16(d_u, sdesc_at(a_d, 2 * j), sdesc_at(b_d, (MC * 128 >> 4) + 2 * j), idesc_u, 1u);
+                  }
                   tc_commit(ubuf_bar(buf));
                 } else {
                   fail(ctl);

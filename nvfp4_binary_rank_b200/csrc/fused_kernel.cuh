@@ -894,14 +894,14 @@ fused_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
           const uint32_t sfb_s = smem_u32(smem + L::kSFB + s * kSfBytes);
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            tc_cp_32x128b_warpx4(sfa_t + 4 * j, smem_desc(sfa_s + 512 * j, 0, 128, 0));
-            tc_cp_32x128b_warpx4(sfb_t + 4 * j, smem_desc(sfb_s + 512 * j, 0, 128, 0));
+            tc_cp_32x128b_warpx4(sfa_t + 4 * j, make_sdesc(sfa_s + 512 * j, 0, 128, 0));
+            tc_cp_32x128b_warpx4(sfb_t + 4 * j, make_sdesc(sfb_s + 512 * j, 0, 128, 0));
           }
-          const uint64_t adesc = smem_desc(smem_u32(smem + L::kA + s * kUnitBytesA), 16, 1024, 2);
-          const uint64_t bdesc = smem_desc(smem_u32(smem + L::kB + s * BN * 128), 16, 1024, 2);
+          const SmemDesc adesc = make_sdesc(smem_u32(smem + L::kA + s * kUnitBytesA), 16, 1024, 2);
+          const SmemDesc bdesc = make_sdesc(smem_u32(smem + L::kB + s * BN * 128), 16, 1024, 2);
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            tc_mma_nvf4(d_tmem, adesc + 2 * j, bdesc + 2 * j, idesc, sfa_t + 4 * j, sfb_t + 4 * j,
+            tc_mma_nvf4(d_tmem, sdesc_at(adesc, 2 * j), sdesc_at(bdesc, 2 * j), idesc, sfa_t + 4 * j, sfb_t + 4 * j,
                         (u > ua || j > 0) ? 1u : 0u);
           }
           tc_commit(empty_bar(s));
@@ -944,12 +944,10 @@ fused_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
           const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) +
                                  static_cast<uint32_t>(b * BN + m0);
           tmem_ld16(taddr, raw);
-          tmem_wait_ld();
 #pragma unroll
           for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(raw[j]);
           if (BN >= 32) {
             tmem_ld16(taddr + 16, raw);
-            tmem_wait_ld();
 #pragma unroll
             for (int j = 0; j < 16; ++j) v[16 + j] = __uint_as_float(raw[j]);
           } else {

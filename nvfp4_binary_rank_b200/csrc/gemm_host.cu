@@ -149,8 +149,8 @@ GemmPlan plan_gemm(const GemmArgs& a) {
   const int ranks_per_tile = (r + p.T - 1) / p.T;
   p.fast = p.unit_alu && p.BN <= 32 && K % 128 == 0 && (!p.shared_z || ranks_per_tile <= kVStageRanks);
 
-  // decode batches (up to 32 rows) take the decode kernel when a CTA's units fit
-  // its class (ceil(U / G) units: the operand cache up to 16 rows)
+  // batches up to 128 rows take the decode kernel when a CTA's units fit its class
+  // (ceil(U / G) units: the operand cache up to 16 rows, 64 units when streamed)
   p.decode = M <= kDecodeMaxRows && (r == 0 || p.shared_z) && (p.U + p.G - 1) / p.G <= decode_max_units(M);
 
   ScratchNeed& need = p.need;
@@ -226,7 +226,9 @@ int launch_gemm(const GemmArgs& a, const GemmPlan& p, const Scratch& scr, cudaSt
     else if (M <= 4) e = launch_decode<4>(tw, dp, s, o);
     else if (M <= 8) e = launch_decode<8>(tw, dp, s, o);
     else if (M <= 16) e = launch_decode<16>(tw, dp, s, o);
-    else e = launch_decode<32>(tw, dp, s, o);
+    else if (M <= 32) e = launch_decode<32>(tw, dp, s, o);
+    else if (M <= 64) e = launch_decode<64>(tw, dp, s, o);
+    else e = launch_decode<128>(tw, dp, s, o);
     return launch_status(e);
   }
   if (!inq) {

@@ -161,63 +161,106 @@ __device__ __forceinline__ void tc_commit(uint32_t bar) {
       : "memory");
 }
 
-// Shared-memory matrix descriptor (tcgen05 format): start address, leading and
-// stride byte offsets (16-byte units), fixed version bits 46..47 = 1, swizzle
-// mode in bits 61..63 (0 none, 2 = 128-byte swizzle).
-__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo_bytes, uint32_t sbo_bytes,
-                                              uint32_t swizzle) {
-  uint64_t d = 0;
-  d |= static_cast<uint64_t>((addr >> 4) & 0x3FFF);
-  d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFF) << 16;
-  d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFF) << 32;
-  d |= 1ull << 46;
-  d |= static_cast<uint64_t>(swizzle & 7) << 61;
+// Shared-memory matrix descriptor (tcgen05 format), kept as its two 32-bit words:
+//   lo: start address in 16-byte units (bits 0..13), leading byte offset in
+//       16-byte units (bits 16..29);
+//   hi: stride byte offset in 16-byte units (bits 0..13), the fixed version bit
+//       (bit 14, descriptor bit 46) and the swizzle mode (bits 29..31: 0 none,
+//       2 = 128-byte swizzle).
+// The 64-bit operand is assembled inside each tcgen05 asm statement, and a
+// matrix further on in shared memory only moves the address field of `lo`
+// (sdesc_at).  Descriptors built with 64-bit adds of run-time offsets came out of
+// some builds with the high word cleared (the MMA then read the operands as
+// unswizzled with a zero stride, measured on B200), so no 64-bit arithmetic is
+// done on them.
+struct SmemDesc {
+  uint32_t lo, hi;
+};
+__device__ __forceinline__ SmemDesc make_sdesc(uint32_t addr, uint32_t lbo_bytes, uint32_t sbo_bytes,
+                                               uint32_t swizzle) {
+  SmemDesc d;
+  d.lo = ((addr >> 4) & 0x3FFFu) | (((lbo_bytes >> 4) & 0x3FFFu) << 16);
+  d.hi = ((sbo_bytes >> 4) & 0x3FFFu) | (1u << 14) | ((swizzle & 7u) << 29);
+  return d;
+}
+// The descriptor of the matrix `units` x 16 bytes further on (shared memory ends
+// below 256 KB, so the 14-bit address field never carries).
+__device__ __forceinline__ SmemDesc sdesc_at(SmemDesc d, uint32_t units) {
+  d.lo += units;
   return d;
 }
 
 // Copy 32 rows x 16 bytes of shared memory to TMEM, replicated into all four
 // 32-lane sub-partitions (one 512-byte scale-factor atom -> 4 columns).
-__device__ __forceinline__ void tc_cp_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {
-  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
-               : "memory");
+__device__ __forceinline__ void tc_cp_32x128b_warpx4(uint32_t taddr, SmemDesc s) {
+  asm volatile(
+      "{\n\t.reg .b64 sd;\n\t"
+      "mov.b64 sd, {%1, %2};\n\t"
+      "tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], sd;\n\t}" ::"r"(taddr), "r"(s.lo), "r"(s.hi)
+      : "memory");
 }
 
 // D(tmem) (+)= A(smem) * B(smem)^T with E2M1 operands and UE4M3 scales per 16
 // elements read from TMEM.  M = 128, N from the instruction descriptor, K = 64.
-__device__ __forceinline__ void tc_mma_nvf4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                            uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
-                                            uint32_t accumulate) {
+__device__ __forceinline__ void tc_mma_nvf4(uint32_t d_tmem, SmemDesc a, SmemDesc b, uint32_t idesc,
+                                            uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %6, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%4], [%5], p;\n\t"
+      "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
+      "mov.b64 da, {%1, %2};\n\t"
+      "mov.b64 db, {%3, %4};\n\t"
+      "setp.ne.b32 p, %8, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], da, db, %5, [%6], [%7], p;\n\t"
       "}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
+      "r"(a.lo), "r"(a.hi), "r"(b.lo), "r"(b.hi), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
       : "memory");
 }
 
 // D(tmem) (+)= A(smem) * B(smem)^T with BF16 operands (both BF16) and FP32
 // accumulation; M = 128, N from the instruction descriptor, K = 16.
-__device__ __forceinline__ void tc_mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+__device__ __forceinline__ void tc_mma_bf16(uint32_t d_tmem, SmemDesc a, SmemDesc b, uint32_t idesc,
                                             uint32_t accumulate) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t"
+      "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
+      "mov.b64 da, {%1, %2};\n\t"
+      "mov.b64 db, {%3, %4};\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %5, p;\n\t"
       "}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      "r"(a.lo), "r"(a.hi), "r"(b.lo), "r"(b.hi), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 
-// Load 16 consecutive 32-bit columns of this warp's 32 TMEM lanes.
+// Load 16 consecutive 32-bit columns of this warp's 32 TMEM lanes.  The wait for
+// the load is part of the same asm statement: tcgen05.ld fills its destination
+// registers asynchronously, so no instruction may read them before
+// tcgen05.wait::ld, and with the wait in a separate statement the compiler is free
+// to move register copies (or spills) of them above it.
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
       : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
         "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
         "=r"(v[14]), "=r"(v[15])
-      : "r"(taddr));
+      : "r"(taddr)
+      : "memory");
+}
+// Two such loads (16 columns at ta into a, 16 at tb into b) behind one wait.
+__device__ __forceinline__ void tmem_ld16x2(uint32_t ta, uint32_t (&a)[16], uint32_t tb, uint32_t (&b)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%32];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%33];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3]), "=r"(a[4]), "=r"(a[5]), "=r"(a[6]),
+        "=r"(a[7]), "=r"(a[8]), "=r"(a[9]), "=r"(a[10]), "=r"(a[11]), "=r"(a[12]), "=r"(a[13]),
+        "=r"(a[14]), "=r"(a[15]), "=r"(b[0]), "=r"(b[1]), "=r"(b[2]), "=r"(b[3]), "=r"(b[4]),
+        "=r"(b[5]), "=r"(b[6]), "=r"(b[7]), "=r"(b[8]), "=r"(b[9]), "=r"(b[10]), "=r"(b[11]),
+        "=r"(b[12]), "=r"(b[13]), "=r"(b[14]), "=r"(b[15])
+      : "r"(ta), "r"(tb)
+      : "memory");
 }
 // Store 16 consecutive 32-bit columns of this warp's 32 TMEM lanes.
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
@@ -230,9 +273,6 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16
 }
 __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_wait_ld() {
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
 // Make generic-proxy shared-memory writes visible to the async proxy (TMA / tensor core).
@@ -247,7 +287,14 @@ __device__ __forceinline__ void fence_proxy_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
+// Named barriers.  bar.sync and bar.red are warp-aligned: all lanes of a warp must
+// execute them together, and a warp counts as arrived as soon as any lane does.
+// The compiler does not see an inline-asm barrier as one, so after a branch that
+// only some lanes take (one lane issuing MMAs and waiting for them, say) nothing
+// would reconverge the warp first: its other lanes would release the barrier
+// early.  Each barrier therefore joins its warp's lanes before arriving.
 __device__ __forceinline__ void named_barrier(uint32_t id, uint32_t nthreads) {
+  __syncwarp();
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
@@ -255,6 +302,7 @@ __device__ __forceinline__ void named_barrier(uint32_t id, uint32_t nthreads) {
 // thread gets the same answer, so a group can leave a loop together.
 __device__ __forceinline__ bool named_barrier_or(uint32_t id, uint32_t nthreads, bool v) {
   uint32_t r;
+  __syncwarp();
   asm volatile(
       "{\n\t.reg .pred p, q;\n\t"
       "setp.ne.u32 q, %1, 0;\n\t"

@@ -89,9 +89,11 @@ def test_kernel_count_follows_the_schedule(lib):
     assert lib.biloco_gemm_kernel_count(16, 13824, 5120, 512) == 1
     assert lib.biloco_gemm_kernel_count(32, 5120, 13824, 512) == 1
     assert lib.biloco_gemm_kernel_count(17, 5120, 5120, 1024) == 1
-    # larger batches: quantiser + GEMM
-    assert lib.biloco_gemm_kernel_count(33, 5120, 13824, 512) == 2
-    assert lib.biloco_gemm_kernel_count(128, 5120, 5120, 512) == 2
+    assert lib.biloco_gemm_kernel_count(33, 5120, 13824, 512) == 1
+    assert lib.biloco_gemm_kernel_count(128, 5120, 5120, 512) == 1
+    # more than 64 units per CTA: quantiser + general GEMM
+    assert lib.biloco_gemm_kernel_count(33, 65536, 65536, 512) == 2
+    assert lib.biloco_gemm_kernel_count(128, 65536, 65536, 512) == 2
     # the local-z schedule runs the general kernel (in-kernel quantisation up to M = 8)
     assert lib.biloco_set_mode(_lib.MODE_LOCAL_Z) == 0
     try:

@@ -64,14 +64,16 @@ def _expected_y(x_f32, N, K, sign):
 
 
 # (M, N, K): the decode-batch classes 1, 2, 4 (each CTA quantises its own chunks)
-# and 8, 16 (one activation image shared by the grid), the general kernel quantising
-# per unit (M <= 8 with more than 16 units per CTA) and the activation pre-pass
-# (M > 8 on the general kernel), at full K and with a ragged last chunk.
+# and 8 to 128 (one activation image shared by the grid; from 32 rows streamed with
+# the weight stages), the general kernel quantising per unit (M <= 8 with more than
+# 16 units per CTA) and the activation pre-pass (M > 8 with more units per CTA than
+# the decode classes take), at full K and with a ragged last chunk.
 SHAPES = [
     (1, 5120, 5120), (1, 5248, 5184), (2, 5120, 5120), (3, 5120, 5120), (4, 5248, 5184),
     (5, 5120, 5120), (8, 5120, 5120), (11, 5248, 5184), (16, 5120, 5120),
     (1, 13824, 13824), (4, 13824, 13824), (8, 13824, 13824),
-    (12, 13824, 13824), (17, 5248, 5184), (32, 5120, 5120), (64, 5120, 5120), (128, 5248, 5184),
+    (12, 13824, 13824), (17, 5248, 5184), (32, 5120, 5120), (33, 5120, 5120), (64, 5120, 5120),
+    (100, 5248, 5184), (128, 5248, 5184), (128, 13824, 13824),
 ]
 
 

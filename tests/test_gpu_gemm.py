@@ -210,6 +210,25 @@ def test_batch32_class(nb, M, N, K, r):
         assert np.all(np.abs(y - ref["gemm"]) <= tol)
 
 
+# --- the 64- and 128-row classes of the decode kernel (33 to 128 rows) ------------
+
+@pytest.mark.parametrize("M,N,K,r", [(33, 384, 832, 255), (48, 640, 1344, 0), (64, 1280, 4096, 1024),
+                                     (64, 5120, 13824, 512), (65, 2560, 5184, 600), (96, 128, 64, 3),
+                                     (100, 13824, 5120, 512), (128, 1280, 2560, 1024), (128, 5120, 5120, 0)])
+def test_batch64_128_classes(nb, M, N, K, r):
+    # MMA N = 64 or 128 from the streamed image; the two BF16 parts of z summed in
+    # one TMEM product (the 128-row class with a single product buffer); z tiles
+    # cycled through 3 (64 rows) or 2 (128 rows) slots; the epilogue 16 columns at a
+    # time
+    w = _small(M, N, K, r, seed=M * 13 + r)
+    d, ref = oracle_for(w)
+    y = _run(nb, device_problem(w, d))
+    assert_y_close(y, ref["y"], w.name)
+    if r == 0:
+        tol = np.abs(ref["gemm"]) * 2.0 ** -8 + 1e-6 * np.abs(ref["gemm"]).max()
+        assert np.all(np.abs(y - ref["gemm"]) <= tol)
+
+
 # --- the correction arithmetic of the 1-2-row U side: sign-adds and table lookups ---
 
 @pytest.mark.parametrize("arith", [1, 2])

@@ -73,12 +73,18 @@ def test_dropped_arrivals_expire_inside_the_gemm(nb, entry, mask, M):
 
 
 def test_drop_request_is_consumed_by_one_call(nb):
-    # a request made before a call that does not take the decode kernel is consumed
-    # by that call and affects nothing
+    # a request made before a call that does not take the decode kernel (here the
+    # local-z schedule, which runs the general kernel) is consumed by that call and
+    # affects nothing
     w = workloads.Workload("drop_general", 40, 256, 512, 32, 77)
     d, ref = oracle_for(w)
     prob = device_problem(w, d)
-    nb.selftest_drop_arrivals(1)
-    y = nb.gemm(prob["x"], prob["W"], prob["sf"], prob["g"], prob["Ub"], prob["Vb"], prob["alpha"])
+    nb.set_mode(nb.MODE_LOCAL_Z)
+    try:
+        assert nb.gemm_kernel_count(w.M, w.N, w.K, w.r) == 2
+        nb.selftest_drop_arrivals(1)
+        y = nb.gemm(prob["x"], prob["W"], prob["sf"], prob["g"], prob["Ub"], prob["Vb"], prob["alpha"])
+    finally:
+        nb.set_mode(nb.MODE_AUTO)
     assert nb.last_error() == 0
     assert_y_close(y_to_numpy(y), ref["y"], w.name)
