@@ -408,6 +408,14 @@ EXTRA_CONFIGS = [
 ]
 
 
+def selected_workload(args):
+    """The timed workload: a named configuration, or a sweep point (--sweep M,r)."""
+    if args.sweep:
+        M, r = (int(v) for v in args.sweep.split(","))
+        return workloads.sweep_config(M, r)
+    return workloads.CONFIGS[args.workload]
+
+
 def workload_config(w, world):
     """The `config` object of both arms: the workload and how it is laid out."""
     return {"workload": w.name, "M": w.M, "N": w.N, "K": w.K, "r": w.r, "seed": w.seed,
@@ -439,7 +447,7 @@ def run_ours(args):
     nb.load()
     stream = torch.cuda.Stream()
     l2 = torch.cuda.get_device_properties(ctx.local).L2_cache_size
-    w = workloads.CONFIGS[args.workload]
+    w = selected_workload(args)
     peak, peak_kind = hbm_peak()
 
     prob = setup_problem(w, n_copies_for(w, l2), torch.device("cuda", ctx.local))
@@ -560,7 +568,7 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    w = workloads.CONFIGS[args.workload]
+    w = selected_workload(args)
     # Each step is a bounded sample of the workload (output rows, a K slice in
     # multiples of 256, a rank slice), shrunk by halving until one step fits
     # 100 s / (steps + warm-up), so that the whole run stays within about 2 minutes.
@@ -622,6 +630,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=200)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(workloads.CONFIGS), default="decode")
+    ap.add_argument("--sweep", metavar="M,r", default=None,
+                    help="time the sweep point with M rows and rank r at N = K = 5120 instead of --workload "
+                         "(for profiler runs of one batch class)")
     ap.add_argument("--no-extra", action="store_true", help="skip the other workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--timed-only", action="store_true",

@@ -287,14 +287,7 @@ __device__ __forceinline__ void fence_proxy_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
-// Named barriers.  bar.sync and bar.red are warp-aligned: all lanes of a warp must
-// execute them together, and a warp counts as arrived as soon as any lane does.
-// The compiler does not see an inline-asm barrier as one, so after a branch that
-// only some lanes take (one lane issuing MMAs and waiting for them, say) nothing
-// would reconverge the warp first: its other lanes would release the barrier
-// early.  Each barrier therefore joins its warp's lanes before arriving.
 __device__ __forceinline__ void named_barrier(uint32_t id, uint32_t nthreads) {
-  __syncwarp();
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
@@ -302,7 +295,6 @@ __device__ __forceinline__ void named_barrier(uint32_t id, uint32_t nthreads) {
 // thread gets the same answer, so a group can leave a loop together.
 __device__ __forceinline__ bool named_barrier_or(uint32_t id, uint32_t nthreads, bool v) {
   uint32_t r;
-  __syncwarp();
   asm volatile(
       "{\n\t.reg .pred p, q;\n\t"
       "setp.ne.u32 q, %1, 0;\n\t"
