@@ -42,14 +42,22 @@ def test_expired_wait_is_reported_and_cleared(nb):
     assert_y_close(y_to_numpy(y), ref["y"], "tiny after a timeout")
 
 
-# (mask, M): 1 drops the z arrivals (1 row: the completing CTA's U side waits;
-# 16 rows: the per-contributor tensor-core U side waits), 2 the activation-image
-# arrivals (8 rows), 3 both.
+# (mask, M, N, K): 1 drops the z arrivals (1 row: the completing CTA's U side
+# waits; 16 rows: the per-contributor tensor-core U side waits), 2 the
+# activation-image arrivals (8 rows; from 17 rows the producers' wait on the
+# streamed image), 3 both.  The 64- and 128-row cases run the column-chunked
+# epilogue's abort path; at N = K = 5120 their CTAs hold two tiles, so the
+# 128-row class's single U-side product buffer is waited on for a second segment.
 @pytest.mark.timeout(120, method="thread")
 @pytest.mark.parametrize("entry", ["gemm", "gemm_noalloc"])
-@pytest.mark.parametrize("mask,M", [(1, 1), (1, 16), (2, 8), (3, 16), (2, 24), (1, 32)])
-def test_dropped_arrivals_expire_inside_the_gemm(nb, entry, mask, M):
-    w = workloads.Workload(f"drop_{M}", M, 1280, 2048, 256, 60 + M)
+@pytest.mark.parametrize("mask,M,N,K", [(1, 1, 1280, 2048), (1, 16, 1280, 2048), (2, 8, 1280, 2048),
+                                        (3, 16, 1280, 2048), (2, 24, 1280, 2048), (1, 32, 1280, 2048),
+                                        (1, 64, 1280, 2048), (3, 64, 5120, 5120), (2, 100, 1280, 2048),
+                                        (1, 128, 5120, 5120)])
+def test_dropped_arrivals_expire_inside_the_gemm(nb, entry, mask, M, N, K):
+    if entry == "gemm_noalloc" and M > 64 and N * K > 1280 * 2048:
+        pytest.skip("the 128-row class's scratch at this size exceeds the no-allocation array")
+    w = workloads.Workload(f"drop_{M}", M, N, K, 256, 60 + M)
     d, ref = oracle_for(w)
     prob = device_problem(w, d)
     args = (prob["x"], prob["W"], prob["sf"], prob["g"], prob["Ub"], prob["Vb"], prob["alpha"])
