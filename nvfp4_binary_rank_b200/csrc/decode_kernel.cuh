@@ -23,8 +23,8 @@
 //   * z is computed in rank slices: CTA g < Z computes z for the ranks
 //     [g r / Z, (g + 1) r / Z) and publishes them behind one arrival counter
 //     (Z = G - 2 on large grids, see shared_work_ctas).  This is the "side CTAs +
-//     arrival flag" schedule of the README's mode table.  Below 16 rows the slice
-//     is summed over the whole of K on the CUDA cores; from 16, V^T x runs on the
+//     arrival flag" schedule of the README's mode table.  Below 8 rows the slice
+//     is summed over the whole of K on the CUDA cores; from 8, V^T x runs on the
 //     tensor cores in pieces of 128 ranks x a K slice whose partial sums the slice
 //     owners add up.
 //   * U z: from 4 rows up (tensor-core U side) every contributor of a weight tile
@@ -116,10 +116,10 @@ struct Cfg {
   // image behind an arrival counter) instead of each CTA quantising the chunks of
   // all its units
   static constexpr bool kGlobalQ = MC >= 8;
-  // with 16 rows the V side runs on the tensor cores, cut into pieces of 128 ranks
-  // x a slice of K, with the partial sums reduced across CTAs (with 8 the CUDA-core
-  // loop is faster, measured on B200)
-  static constexpr bool kTensorV = MC >= 16;
+  // from 8 rows the V side runs on the tensor cores, cut into pieces of 128 ranks
+  // x a slice of K, with the partial sums reduced across CTAs (at 8 rows 13-22%
+  // faster than the CUDA-core loop, measured on B200; below 8 that loop stays)
+  static constexpr bool kTensorV = MC >= 8;
   // The U side's product: up to 32 rows the high and low BF16 parts of z go to
   // separate TMEM columns (one MMA of N = 2 MC per K step, added by the epilogue);
   // from 64 rows both parts accumulate into the same MC columns (two MMAs of N = MC),
