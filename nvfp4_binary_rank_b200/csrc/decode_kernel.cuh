@@ -766,7 +766,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
     const int etid = threadIdx.x - kEpiWarp0 * 32;
     griddep_wait();
     const float gs = __ldcg(p.gscale);
-    constexpr int kHB = (MC <= 2) ? 16 : (MC <= 4 ? 8 : (MC <= 8 ? 4 : (MC <= 16 ? 2 : 1)));   // partials loaded per batch
+    constexpr int kHB = (MC <= 2) ? 16 : (MC <= 4 ? 8 : (MC <= 8 ? 6 : (MC <= 16 ? 3 : 1)));   // partials loaded per batch
     // the accumulator of buffer b for this warp's lane quarter, times g
     auto load_acc = [&](int b, float (&v)[MC]) {
 #pragma unroll
@@ -959,12 +959,12 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
           named_barrier(kBarEpi, kEpiThreads);
           if (!fin) continue;
           // every contributor's partial, summed in contributor order (the 32-row
-          // class in two halves of 16 rows, two contributors per batch of loads)
+          // class in two halves of 16 rows, three contributors per batch of loads)
   #pragma unroll
           for (int j = 0; j < MC; ++j) acc[j] = 0.0f;
           const int wh_first = (t == first_unit(hf, p.G, p.U) / p.KC) ? 0 : 1;
           constexpr int kRC = (MC > 16) ? 16 : MC;
-          constexpr int kHBc = (MC > 16) ? 2 : kHB;
+          constexpr int kHBc = (MC > 16) ? 3 : kHB;
   #pragma unroll
           for (int j0 = 0; j0 < MC; j0 += kRC) {
             for (int h0 = hf; h0 <= hl; h0 += kHBc) {
