@@ -194,7 +194,7 @@ int biloco_decompose(const float *W, int N, int K, int r, int T, const uint32_t 
  * of its dependents (griddepcontrol.launch_dependents); kernels without that
  * trigger, biloco_pack_weight's included, are fully ordered before the call.
  *
- * Residency: the GEMM kernel runs one CTA per SM on G = min(#SMs, units) CTAs
+ * Residency: the GEMM kernel runs one CTA per SM on G <= min(#SMs, units) CTAs
  * that exchange data behind grid-wide arrival counters, so all G CTAs must be
  * resident together.  The host checks that one CTA per SM fits
  * (BILOCO_ERR_RESIDENCY otherwise).  With the default launch form
@@ -225,7 +225,9 @@ int biloco_gemm(const void *x_bf16, const uint8_t *W_fp4, const uint8_t *W_sf,
  * checked on the host before anything is launched (BILOCO_ERR_SHAPE otherwise):
  *   N <= BILOCO_NOALLOC_MAX_N, and the call's scratch fits the array.  That
  *   scratch is 16 896 bytes of status and counters plus, each rounded up to 256,
- *   with KC = ceil(K/256), G = min(#SMs, (N/128)*KC) and rpad = 16*ceil(r/16):
+ *   with KC = ceil(K/256), G = min(#SMs, (N/128)*KC) (for 65..128 rows on the
+ *   decode-batch kernel at most 5*(N/128)/2 where that keeps <= 64 units per
+ *   CTA) and rpad = 16*ceil(r/16):
  *   decode-batch kernel (M <= 128, shared-z schedule, ceil(units/G) <= 16 for
  *   M <= 16 or <= 64 above; BN = 16 for M <= 16, else the batch class 32, 64
  *   or 128 that holds M):

@@ -152,6 +152,17 @@ GemmPlan plan_gemm(const GemmArgs& a) {
   // batches up to 128 rows take the decode kernel when a CTA's units fit its class
   // (ceil(U / G) units: the operand cache up to 16 rows, 64 units when streamed)
   p.decode = M <= kDecodeMaxRows && (r == 0 || p.shared_z) && (p.U + p.G - 1) / p.G <= decode_max_units(M);
+  // The 128-row class takes at most about 2.5 CTAs per weight tile: its split-K
+  // partials are 64 KB per contributor, and fewer contributors per tile shorten the
+  // final sums more than the lost SMs slow the weight stream.  Timed on a B200
+  // (N, K, r; us per call, 148 -> capped grid): 5120, 5120, 512: 61.0 -> 48.1;
+  // 5120, 5120, 0: 36.8 -> 32.3; 5120, 13824, 512: 68.7 -> 60.1; M = 96, 5120,
+  // 5120, 256: 50.1 -> 38.4; 5120, 5120, 1024: 74.0 -> 75.5.  With many tiles
+  // (N = 13824) the cap does not apply; a fixed 100 CTAs there was slower.
+  if (p.decode && decode_class(M) == 128) {
+    const int g = std::max(1, 5 * p.T / 2);
+    if (g < p.G && (p.U + g - 1) / g <= decode_max_units(M)) p.G = g;
+  }
 
   ScratchNeed& need = p.need;
   if (p.decode) {
