@@ -193,6 +193,23 @@ def test_cooperative_launch(nb, flags, name):
     np.testing.assert_array_equal(y, y_pdl)
 
 
+@pytest.mark.parametrize("M,N,K,r", [(48, 1280, 2048, 256), (128, 5120, 5120, 512)])
+def test_cooperative_launch_large_classes(nb, M, N, K, r):
+    # the cooperative form on the 64- and 128-row classes (the latter on its capped
+    # grid of 2.5 CTAs per tile): same y as the default launch, within tolerance
+    w = _small(M, N, K, r, seed=M * 17 + r)
+    d, ref = oracle_for(w)
+    prob = device_problem(w, d)
+    y_pdl = _run(nb, prob)
+    nb.set_launch(nb.LAUNCH_COOPERATIVE)
+    try:
+        y = _run(nb, prob)
+    finally:
+        nb.set_launch(nb.LAUNCH_PDL)
+    assert_y_close(y, ref["y"], w.name)
+    np.testing.assert_array_equal(y, y_pdl)
+
+
 # --- the 32-row class of the decode kernel (17 to 32 rows) ------------------------
 
 @pytest.mark.parametrize("M,N,K,r", [(17, 384, 832, 255), (20, 640, 1344, 0), (24, 1280, 4096, 1024),
