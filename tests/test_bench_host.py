@@ -52,3 +52,40 @@ def test_ncu_traffic_follows_the_source_digest(monkeypatch):
     monkeypatch.setattr(bench, "kernel_source_digest", lambda: "0000000000000000")
     assert bench.ncu_traffic("decode", 1) is None
     assert bench.ncu_traffic("no_such_workload", 1) is None
+
+
+def test_every_committed_profile_names_its_workload_and_kernel():
+    # each summary under profiles/ carries the two fields the bench reads, and its
+    # workload resolves to a configuration or a sweep point of the bench
+    prof = os.path.join(ROOT, "profiles")
+    names = [f for f in os.listdir(prof) if f.startswith("decode_kernel_") and f.endswith(".md")]
+    assert names
+    for f in names:
+        text = open(os.path.join(prof, f)).read()
+        assert "- source_digest: `" in text and "- dram_bytes_per_launch: " in text, f
+        wl = f[len("decode_kernel_"):-3]
+        if wl.startswith("sweep_M"):
+            M, r = (int(v) for v in wl[len("sweep_M"):].split("_r"))
+            assert workloads.sweep_config(M, r).name == wl
+        else:
+            assert wl in workloads.CONFIGS, f
+
+
+def test_metric_range_reports_the_worst_point():
+    extra = {"sweep_M8_r512": {"us": 17.6, "frac": 0.137}, "sweep_M16_r512": {"us": 19.0, "frac": 0.128},
+             "sweep_M32_r512": {"us": 23.7, "frac": 0.105}, "mlp_up": {"us": 22.0, "frac": 0.293}}
+    got = bench.metric_range(11.4, 0.21, extra)
+    assert sorted(got["points"]) == ["M1", "M16", "M32", "M8"]
+    assert got["worst"] == {"M": 32, "us": 23.7, "frac": 0.105}
+    # with only the headline, the headline is the worst point
+    assert bench.metric_range(11.4, 0.21, {})["worst"]["M"] == 1
+
+
+def test_sweep_option_selects_a_sweep_point():
+    class A:
+        sweep = "64,512"
+        workload = "decode"
+    w = bench.selected_workload(A)
+    assert (w.name, w.M, w.N, w.K, w.r) == ("sweep_M64_r512", 64, 5120, 5120, 512)
+    A.sweep = None
+    assert bench.selected_workload(A).name == "decode"
