@@ -327,9 +327,10 @@ int biloco_selftest_wait_timeout(biloco_stream_t stream);
 /*
  * biloco_selftest_drop_arrivals - exercise the GEMM's own failure path on the GPU
  * without a fault.  The next biloco_gemm or biloco_gemm_noalloc call that runs
- * the decode-batch kernel (M <= 16, shared-z schedule) leaves out the grid-wide
- * arrivals selected by `mask` (1: the z slices, 2: the activation image, 3:
- * both); every other call, and every call after that one, is unaffected.  The
+ * the decode-batch kernel (M <= 128, shared-z schedule) leaves out the grid-wide
+ * arrivals selected by `mask` (1: the z slices, 2: the activation image, which
+ * batches of 8 rows and more share, 3: both); every other call, and every call
+ * after that one, is unaffected.  The
  * CTAs waiting on those arrivals give up after their bounded wait (about 1 s),
  * leave together, drain their copies and tensor-core work, free their tensor
  * memory and record BILOCO_ERR_TIMEOUT; y of that call is not valid.  A following
