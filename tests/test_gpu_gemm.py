@@ -210,6 +210,18 @@ def test_cooperative_launch_large_classes(nb, M, N, K, r):
     np.testing.assert_array_equal(y, y_pdl)
 
 
+@pytest.mark.parametrize("M,N,K,r", [(5, 384, 832, 255), (7, 2560, 1344, 129), (8, 1280, 5184, 1000),
+                                     (6, 13824, 5120, 512), (100, 640, 2624, 300)])
+def test_tensor_v_side_from_8_rows_and_capped_grid(nb, M, N, K, r):
+    # the 8-row class's V side in tensor-core pieces (ragged K, partial rank blocks,
+    # more rank blocks than pieces per CTA), and a 128-row call on a ragged shape
+    # whose grid is capped at 2.5 CTAs per tile (5 tiles -> 12 CTAs)
+    w = _small(M, N, K, r, seed=M * 19 + r)
+    d, ref = oracle_for(w)
+    y = _run(nb, device_problem(w, d))
+    assert_y_close(y, ref["y"], w.name)
+
+
 # --- the 32-row class of the decode kernel (17 to 32 rows) ------------------------
 
 @pytest.mark.parametrize("M,N,K,r", [(17, 384, 832, 255), (20, 640, 1344, 0), (24, 1280, 4096, 1024),
