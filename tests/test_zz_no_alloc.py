@@ -57,6 +57,8 @@ SHAPES = [
     ("m24", workloads.Workload("na_24_640_1344_100", 24, 640, 1344, 100, 14), 1),
     ("m3_r0", workloads.Workload("na_3_256_512_0", 3, 256, 512, 0, 13), 1),
     ("mlp_up", workloads.CONFIGS["mlp_up"], 1),
+    ("m64_full", workloads.sweep_config(64, 512), 1),
+    ("m128_small", workloads.Workload("na_128_640_1280_64", 128, 640, 1280, 64, 15), 1),
 ]
 
 
